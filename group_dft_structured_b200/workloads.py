@@ -1,0 +1,96 @@
+"""Workload shapes and seeded synthetic inputs for the p4 EQ-Linear layer.
+
+This module holds no arithmetic of the method: it only draws random numbers
+and rounds them to the compute dtype.  Both the CUDA path (through the tests
+and the benchmark) and the float64 oracle consume exactly the rounded arrays
+produced here.
+
+Recipe.  Layout x[N,C,4], W[D,C,4], b[D], dy[N,D,4] (group index innermost).
+Values are drawn in float64 with numpy's PCG64 generator and rounded
+(round-to-nearest-even) to the mode dtype:
+
+* x, dy ~ N(0, 1)
+* W ~ N(0, variance 1/(4C)), i.e. std 1/(2 sqrt C): the fan-in of the
+  unrolled 4C-wide layer, so that Var(y) is about 1
+* b ~ N(0, std 0.02)
+
+Seeds: 20260000 + 100 * workload_id + {x: 0, W: 1, b: 2, dy: 3}.
+
+The shapes stand in for the token streams of the networks the paper
+evaluates (Flash EQ-ViT and Flash EQ-Swin, technical summary "Livello di
+Rete"): a ViT MLP fc1 at 64 x 197 tokens and a Swin stage-1 stream at
+128 x 3136 tokens; no dataset is involved.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+T = 4
+
+
+@dataclass(frozen=True)
+class Workload:
+    wid: int            # workload id (used in the seeds)
+    name: str
+    N: int              # tokens
+    C: int              # input channels per group element
+    D: int              # output channels per group element
+    dtype: str          # "fp16" or "fp32"
+    passes: tuple       # subset of ("fwd", "dx", "dw")
+    note: str
+
+
+WORKLOADS = {
+    1: Workload(1, "p4_fwd_fp32_N256_C16_D16", 256, 16, 16, "fp32", ("fwd",),
+                "small forward, fp32 (64->64 unrolled)"),
+    2: Workload(2, "p4_fwd_fp16_vit_fc1_N12608_C48_D192", 12608, 48, 192, "fp16", ("fwd",),
+                "ViT MLP fc1-like forward, 64x197 tokens (192->768 unrolled)"),
+    3: Workload(3, "p4_fwd_fp16_square_N65536_C192_D192", 65536, 192, 192, "fp16", ("fwd",),
+                "square forward (768->768 unrolled); also run in fp32 mode"),
+    4: Workload(4, "p4_bwd_fp16_N32768_C256_D256", 32768, 256, 256, "fp16", ("dx", "dw"),
+                "backward dX and dW (1024->1024 unrolled)"),
+    5: Workload(5, "p4_fwdbwd_fp16_swin_N401408_C24_D96", 401408, 24, 96, "fp16",
+                ("fwd", "dx", "dw"),
+                "Swin stage-1-like forward+backward, 128x3136 tokens (96->384 unrolled)"),
+}
+
+
+def np_dtype(dtype: str):
+    return {"fp16": np.float16, "fp32": np.float32, "fp64": np.float64}[dtype]
+
+
+def _normal(seed: int, shape, std: float, dtype: str) -> np.ndarray:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    v = rng.standard_normal(size=shape, dtype=np.float64)
+    if std != 1.0:
+        v *= std
+    return v.astype(np_dtype(dtype))
+
+
+def make_inputs(wid: int, N: int, C: int, D: int, dtype: str,
+                which=("x", "W", "b", "dy")) -> dict:
+    """Seeded, dtype-rounded inputs for a layer of the given shape.
+
+    ``wid`` selects the seed block; any shape may be drawn with it (small
+    parity cases reuse a workload's seeds at reduced sizes).
+    """
+    base = 20260000 + 100 * wid
+    out = {}
+    if "x" in which:
+        out["x"] = _normal(base + 0, (N, C, T), 1.0, dtype)
+    if "W" in which:
+        out["W"] = _normal(base + 1, (D, C, T), 1.0 / (2.0 * np.sqrt(C)), dtype)
+    if "b" in which:
+        out["b"] = _normal(base + 2, (D,), 0.02, dtype)
+    if "dy" in which:
+        out["dy"] = _normal(base + 3, (N, D, T), 1.0, dtype)
+    return out
+
+
+def workload_inputs(wid: int, dtype: str | None = None, N: int | None = None,
+                    which=("x", "W", "b", "dy")) -> dict:
+    w = WORKLOADS[wid]
+    return make_inputs(wid, w.N if N is None else N, w.C, w.D, dtype or w.dtype, which)
