@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the p4 Flash EQ-Linear hot path on B200 (one JSON line).
+
+A step is one pass of the whole path on one batch: weight transform
+(feql_weight_fft), forward (feql_forward), input gradient (feql_backward_dx)
+and weight gradient (feql_backward_dw), all through the C ABI, fp16 data with
+fp32 accumulation, on the Swin stage-1-like forward+backward workload
+N = 128 x 3136 tokens, C = 24, D = 96 (96 -> 384 unrolled).  Inputs are
+resident in HBM; each pass reads/writes ~385 MB, more than the 126 MB L2, so
+no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the full workload on
+its own tokens (weak scaling); the data-parallel weight gradient is summed
+with one NCCL all-reduce per step.  --impl reference times the float64 CPU
+oracle (the unrolled dense method) on the host cores, on a bounded sample.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "p4 EQ-Linear fwd/bwd tokens/s, effective TFLOP/s and % of roofline (fp16)"
+WORKLOAD_ID = 5
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def workload_bytes(w, elt):
+    """Algorithmic HBM bytes per launch of each pass (inputs read once, outputs
+    written once; Fourier weights counted as their 4*D*C values)."""
+    N, C, D = w.N, w.C, w.D
+    x, y, what, b = 4 * N * C * elt, 4 * N * D * elt, 4 * D * C * elt, D * elt
+    return {
+        "wfft": 4 * D * C * elt + what,
+        "fwd": x + what + b + y,
+        "dx": y + what + x,
+        "dw": x + y + 4 * D * C * elt + b,
+    }
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------- baseline
+def oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def time_oracle(w, n_sample):
+    """Float64 oracle (unrolled dense method) for all passes on n_sample tokens."""
+    import numpy as np
+
+    from group_dft_structured_b200.workloads import make_inputs
+    from oracle import feql_oracle as O
+    inp = make_inputs(w.wid, n_sample, w.C, w.D, w.dtype)
+    f = {k: v.astype(np.float64) for k, v in inp.items()}
+    t0 = time.perf_counter()
+    if "fwd" in w.passes:
+        O.forward(f["x"], f["W"], f["b"])
+    if "dx" in w.passes:
+        O.backward_dx(f["dy"], f["W"])
+    if "dw" in w.passes:
+        O.backward_dw(f["x"], f["dy"])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, target_s=3.0):
+    n = min(w.N, 8192)
+    t = min(time_oracle(w, n), time_oracle(w, n))
+    while t < target_s and n < w.N:
+        n = min(w.N, n * 2)
+        t = time_oracle(w, n)
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
+            "sample": f"{n} of {w.N} tokens, passes {'+'.join(w.passes)}, float64 numpy "
+                      f"(unrolled circulant), one timed run of {t:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from group_dft_structured_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    # size one step so that the whole run stays within about two minutes
+    target = min(1.5, 120.0 / max(1, args.steps + args.warmup))
+    n = min(w.N, 1024)
+    t = min(time_oracle(w, n), time_oracle(w, n))
+    while t < target and n < w.N:
+        n = min(w.N, n * 2)
+        t = time_oracle(w, n)
+    for _ in range(args.warmup):
+        time_oracle(w, n)
+    times = [time_oracle(w, n) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "N": w.N, "C": w.C, "D": w.D,
+                   "passes": list(w.passes), "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_cores(),
+                         "kind": "oracle",
+                         "sample": f"{n} of {w.N} tokens per step, float64 numpy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------- ours
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import group_dft_structured_b200 as F
+    from group_dft_structured_b200 import layer as L
+    from group_dft_structured_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    F.load()
+    mode = F.FEQL_FP16 if w.dtype == "fp16" else F.FEQL_FP32
+    N, C, D = w.N, w.C, w.D
+    elt = 2 if w.dtype == "fp16" else 4
+    inp = make_inputs(w.wid + 1000 * rank, N, C, D, w.dtype)
+    dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    x, W, b, dy = dev["x"], dev["W"], dev["b"], dev["dy"]
+    What = torch.empty(F.feql_weight_fft_bytes(C, D, mode), dtype=torch.uint8, device="cuda")
+    y = torch.empty((N, D, 4), dtype=x.dtype, device="cuda")
+    dx = torch.empty((N, C, 4), dtype=x.dtype, device="cuda")
+    dW = torch.empty((D, C, 4), dtype=x.dtype, device="cuda")
+    db = torch.empty((D,), dtype=x.dtype, device="cuda")
+    ws = L.dw_workspace(N, C, D, mode, "cuda")
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    passes = ["wfft"] + [p for p in ("fwd", "dx", "dw") if p in w.passes]
+    launches_per_step = {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2}
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        F.feql_weight_fft(W, What, C, D, mode, s)
+        if ev is not None:
+            ev[1].record(stream)
+        i = 2
+        if "fwd" in passes:
+            F.feql_forward(x, What, b, y, N, C, D, mode, s)
+            if ev is not None:
+                ev[i].record(stream)
+            i += 1
+        if "dx" in passes:
+            F.feql_backward_dx(dy, What, dx, N, C, D, mode, s)
+            if ev is not None:
+                ev[i].record(stream)
+            i += 1
+        if "dw" in passes:
+            F.feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s)
+            if ev is not None:
+                ev[i].record(stream)
+        if world > 1:
+            dist.all_reduce(dW)
+            dist.all_reduce(db)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if F.feql_device_status(s) != F.FEQL_OK:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    clocks = ClockSampler(local_rank)
+    if rank == 0 or world == 1:
+        clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(passes) + 1)]
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop() if (rank == 0 or world == 1) else None
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    per_pass = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
+                for i, p in enumerate(passes)}
+    if F.feql_device_status(s) != F.FEQL_OK:
+        raise RuntimeError("device-side timeout during timing")
+
+    # ---------------------------------------------------------- e2e (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: torch.from_numpy(v).pin_memory() for k, v in inp.items()}
+        hout = {"y": torch.empty_like(y, device="cpu").pin_memory(),
+                "dx": torch.empty_like(dx, device="cpu").pin_memory(),
+                "dW": torch.empty_like(dW, device="cpu").pin_memory(),
+                "db": torch.empty_like(db, device="cpu").pin_memory()}
+        h2d = sum(hin[k].numel() * hin[k].element_size() for k in ("x", "W", "b")) + \
+            (hin["dy"].numel() * hin["dy"].element_size() if ("dx" in passes or "dw" in passes) else 0)
+        outs = [k for k in ("y", "dx", "dW", "db")
+                if (k == "y" and "fwd" in passes) or (k == "dx" and "dx" in passes)
+                or (k in ("dW", "db") and "dw" in passes)]
+        d2h = sum(hout[k].numel() * hout[k].element_size() for k in outs)
+        src = {"y": y, "dx": dx, "dW": dW, "db": db}
+
+        def e2e_step():
+            x.copy_(hin["x"], non_blocking=True)
+            W.copy_(hin["W"], non_blocking=True)
+            b.copy_(hin["b"], non_blocking=True)
+            if "dx" in passes or "dw" in passes:
+                dy.copy_(hin["dy"], non_blocking=True)
+            step()
+            for k in outs:
+                hout[k].copy_(src[k], non_blocking=True)
+
+        e2e_step()
+        barrier()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z.record(stream)
+        barrier()
+        e_ms = a.elapsed_time(z)
+        if world > 1:
+            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": N * world * args.e2e_steps / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # ------------------------------------------------------------- report
+    value = N * world * args.steps / (ms * 1e-3)
+    peak, peak_src = measured_peaks()
+    nbytes = workload_bytes(w, elt)
+    macs = 6 * N * C * D
+    mean_ms = {p: float(np.mean(v)) for p, v in per_pass.items()}
+    pass_report = {}
+    for p in passes:
+        gbs = nbytes[p] / (mean_ms[p] * 1e-3) / 1e9
+        pass_report[p] = {"ms": round(mean_ms[p], 5), "GB_s": round(gbs, 1),
+                          "frac_hbm": round(gbs / peak, 4), "algorithmic_bytes": nbytes[p]}
+        if p != "wfft":
+            pass_report[p]["alg_TFLOP_s"] = round(2 * macs / (mean_ms[p] * 1e-3) / 1e12, 2)
+            pass_report[p]["dense_equiv_TFLOP_s"] = round(
+                2 * 16 * N * C * D / (mean_ms[p] * 1e-3) / 1e12, 2)
+    dom = max((p for p in passes if p != "wfft"), key=lambda p: mean_ms[p])
+    achieved = nbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get(w.name, {}).get(dom)
+    nkern = sum(launches_per_step[p] for p in passes)
+    step_ms = ms / args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "N": N, "C": C, "D": D, "T": 4,
+                   "passes": passes, "accumulate": "f32", "l2": "inputs larger than L2, no flush",
+                   "global_tokens": N * world,
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "effective_TFLOP_s": round(2 * 16 * N * C * D * len([p for p in passes if p != "wfft"])
+                                   * world / (step_ms * 1e-3) / 1e12, 2),
+        "roofline_pct_step": round(100 * sum(nbytes[p] for p in passes) / (step_ms * 1e-3) / 1e9
+                                   / peak, 2),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": peak_src},
+        "passes": pass_report,
+        "gpu_launches": nkern * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,334 @@
+// feql_api.cu — the C ABI of libfeql.so (declared in include/feql.h).
+//
+// Host side only: argument validation, per-shape plans, TMA tensor maps and
+// kernel launches.  Every arithmetic step runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/feql.h"
+#include "plan.cuh"
+#include "simt.cuh"
+#include "sm100.cuh"
+#include "tc_fwd.cuh"
+#include "wfft.cuh"
+
+using namespace feql;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxChannels = 1 << 16;   // per group element
+constexpr int64_t kMaxTokens = (1ll << 31) - 1;  // TMA coordinates are int32
+
+struct DeviceInfo {
+  int sms = 0;
+  int smem_optin = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ok[kMaxDevices];
+
+int device_info(DeviceInfo *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FEQL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_dev_ok[dev]) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FEQL_ERR_CUDA;
+    g_dev[dev] = d;
+    g_dev_ok[dev] = true;
+  }
+  *out = g_dev[dev];
+  return FEQL_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major fp16 matrix [rows][cols] viewed as a 2-D tensor; box = 64 cols x 128 rows,
+// 128-byte swizzle, zero fill out of range.
+int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return FEQL_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBM)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int dt) { return dt >= FEQL_FP16 && dt <= FEQL_FP16_SIMT; }
+
+// Resolves FEQL_FP32 to the library's fp32 algorithm.
+int resolve(int dt) { return dt == FEQL_FP32 ? FEQL_FP32_SIMT : dt; }
+
+bool is_tc(int dt) { return dt == FEQL_FP16; }
+bool is_half(int dt) { return dt == FEQL_FP16 || dt == FEQL_FP16_SIMT; }
+
+int check_shape(int C, int D) {
+  if (C <= 0 || D <= 0 || C > kMaxChannels || D > kMaxChannels) return FEQL_ERR_INVALID_ARG;
+  return FEQL_OK;
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FEQL_OK : FEQL_ERR_CUDA;
+}
+
+int grid_for(int64_t work, int threads, int sms) {
+  int64_t g = cdiv(work, threads);
+  const int64_t cap = static_cast<int64_t>(sms) * 8;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
+
+// ---------------------------------------------------------------- tc launch
+int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __half *bias,
+                   void *out, int64_t N, cudaStream_t stream) {
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
+  TcFwdParams p;
+  p.wt = wt;
+  p.bias = bias;
+  p.N = N;
+  p.Ci = P.Ci;
+  p.Do = P.Do;
+  p.BD = P.BD;
+  p.nD = P.nD;
+  p.nK = P.nK;
+  p.chunk_bytes = P.chunk_bytes;
+  const int64_t nM = cdiv(N, kBM);
+  if (nM * P.nD > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  p.n_units = static_cast<int>(nM * P.nD);
+  p.nacc = (4 * P.BD <= 256) ? 2 : 1;
+  p.acc_stride = p.nacc == 2 ? 256 : 0;
+  p.stage_bytes = kXChunkBytes + static_cast<int>(align_up(P.chunk_bytes, 1024));
+  p.bias_floats = P.nD * P.BD;
+  const int budget = dev.smem_optin - 1024;  // 1 KB for aligning the base
+  p.stages = 8;
+  while (p.stages > 2 && tc_fwd_smem(p).total > budget) --p.stages;
+  if (tc_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  const int smem = tc_fwd_smem(p).total + 1024;
+
+  CUtensorMap tm_in, tm_out;
+  st = make_tmap_f16(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT);
+  if (st != FEQL_OK) return st;
+  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT);
+  if (st != FEQL_OK) return st;
+  if (cudaFuncSetAttribute(tc_fourier_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return FEQL_ERR_CUDA;
+  const int grid = p.n_units < dev.sms ? p.n_units : dev.sms;
+  tc_fourier_gemm_kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, tm_out, p);
+  return launch_status();
+}
+
+template <typename T>
+int launch_simt_fwd(const void *in, const float *Wp, const void *bias, void *out, int64_t N,
+                    int Ci, int Do, cudaStream_t stream) {
+  const int64_t gx = cdiv(N, kSimtTile);
+  if (gx > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(cdiv(Do, kSimtTile)));
+  if (grid.y > 65535) return FEQL_ERR_UNSUPPORTED;
+  simt_fwd_kernel<T><<<grid, kSimtThreads, 0, stream>>>(
+      static_cast<const T *>(in), Wp, static_cast<const T *>(bias), static_cast<T *>(out), N, Ci,
+      Do);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- dW plan
+struct DwPlan {
+  int splits;
+  int64_t split_len;
+  int64_t ws_floats;
+};
+
+DwPlan make_dw_plan(int64_t N, int C, int D, int sms) {
+  DwPlan q;
+  const int64_t tiles = cdiv(D, kSimtTile) * cdiv(C, kSimtTile);
+  int64_t s = cdiv(2ll * sms, tiles);
+  const int64_t max_s = cdiv(N, kSimtK) > 0 ? cdiv(N, kSimtK) : 1;
+  if (s > max_s) s = max_s;
+  if (s > 1024) s = 1024;
+  if (s < 1) s = 1;
+  q.split_len = align_up(cdiv(N > 0 ? N : 1, s), kSimtK);
+  q.splits = static_cast<int>(cdiv(N > 0 ? N : 1, q.split_len));
+  q.ws_floats = static_cast<int64_t>(q.splits) * (4ll * C * D + D);
+  return q;
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+size_t feql_weight_fft_bytes(int C, int D, int dtype) {
+  if (!valid_dtype(dtype) || check_shape(C, D) != FEQL_OK) return 0;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return 0;
+  return static_cast<size_t>(make_what_layout(C, D, is_tc(dt)).bytes);
+}
+
+int feql_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_stream stream) {
+  if (!valid_dtype(dtype) || W == nullptr || What == nullptr) return FEQL_ERR_INVALID_ARG;
+  if (check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WhatLayout L = make_what_layout(C, D, is_tc(dt));
+  if (is_tc(dt)) {
+    const int64_t elems = (L.fwd.bytes + L.dx.bytes) / 2;
+    wfft_tc_kernel<<<grid_for(elems, 256, dev.sms), 256, 0, s>>>(
+        static_cast<const __half *>(W), static_cast<uint8_t *>(What), L, C);
+  } else if (is_half(dt)) {
+    wfft_simt_kernel<__half><<<grid_for(2ll * C * D, 256, dev.sms), 256, 0, s>>>(
+        static_cast<const __half *>(W), static_cast<float *>(What), C, D);
+  } else {
+    wfft_simt_kernel<float><<<grid_for(2ll * C * D, 256, dev.sms), 256, 0, s>>>(
+        static_cast<const float *>(W), static_cast<float *>(What), C, D);
+  }
+  return launch_status();
+}
+
+static int pass_common(const void *in, const void *What, const void *bias, void *out, int64_t N,
+                       int C, int D, int dtype, feql_stream stream, int dir) {
+  if (!valid_dtype(dtype) || in == nullptr || What == nullptr || out == nullptr)
+    return FEQL_ERR_INVALID_ARG;
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
+  if (N == 0) return FEQL_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WhatLayout L = make_what_layout(C, D, is_tc(dt));
+  const int Ci = dir == 0 ? C : D, Do = dir == 0 ? D : C;
+  if (is_tc(dt)) {
+    const uint8_t *wt = static_cast<const uint8_t *>(What) + (dir == 0 ? L.off_fwd : L.off_dx);
+    return launch_tc_gemm(in, wt, dir == 0 ? L.fwd : L.dx, static_cast<const __half *>(bias), out,
+                          N, s);
+  }
+  const float *Wp = static_cast<const float *>(What) + (dir == 0 ? L.off_fwd : L.off_dx) / 4;
+  if (is_half(dt)) return launch_simt_fwd<__half>(in, Wp, bias, out, N, Ci, Do, s);
+  return launch_simt_fwd<float>(in, Wp, bias, out, N, Ci, Do, s);
+}
+
+int feql_forward(const void *x, const void *What, const void *b, void *y, int64_t N, int C, int D,
+                 int dtype, feql_stream stream) {
+  return pass_common(x, What, b, y, N, C, D, dtype, stream, 0);
+}
+
+int feql_backward_dx(const void *dy, const void *What, void *dx, int64_t N, int C, int D,
+                     int dtype, feql_stream stream) {
+  return pass_common(dy, What, nullptr, dx, N, C, D, dtype, stream, 1);
+}
+
+size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
+  if (!valid_dtype(dtype) || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
+  DeviceInfo dev;
+  if (device_info(&dev) != FEQL_OK) return 0;
+  return static_cast<size_t>(make_dw_plan(N, C, D, dev.sms).ws_floats) * 4;
+}
+
+int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws, size_t ws_bytes,
+                     int64_t N, int C, int D, int dtype, feql_stream stream) {
+  if (!valid_dtype(dtype) || x == nullptr || dy == nullptr || dW == nullptr || ws == nullptr)
+    return FEQL_ERR_INVALID_ARG;
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws))
+    return FEQL_ERR_INVALID_ARG;
+  if (db != nullptr && !aligned16(db)) return FEQL_ERR_INVALID_ARG;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  const DwPlan q = make_dw_plan(N, C, D, dev.sms);
+  if (ws_bytes < static_cast<size_t>(q.ws_floats) * 4) return FEQL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float *wsf = static_cast<float *>(ws);
+  float *wsdb = wsf + static_cast<int64_t>(q.splits) * 4 * C * D;
+  dim3 grid(static_cast<unsigned>(cdiv(D, kSimtTile)), static_cast<unsigned>(cdiv(C, kSimtTile)),
+            static_cast<unsigned>(q.splits));
+  if (grid.y > 65535) return FEQL_ERR_UNSUPPORTED;
+  const int64_t red = static_cast<int64_t>(C) * D + D;
+  if (is_half(dt)) {
+    simt_dw_partial_kernel<__half><<<grid, kSimtThreads, 0, s>>>(
+        static_cast<const __half *>(x), static_cast<const __half *>(dy), wsf, wsdb, N, C, D,
+        q.split_len);
+    dw_reduce_kernel<__half><<<grid_for(red, 256, dev.sms), 256, 0, s>>>(
+        wsf, wsdb, static_cast<__half *>(dW), static_cast<__half *>(db), q.splits, C, D);
+  } else {
+    simt_dw_partial_kernel<float><<<grid, kSimtThreads, 0, s>>>(
+        static_cast<const float *>(x), static_cast<const float *>(dy), wsf, wsdb, N, C, D,
+        q.split_len);
+    dw_reduce_kernel<float><<<grid_for(red, 256, dev.sms), 256, 0, s>>>(
+        wsf, wsdb, static_cast<float *>(dW), static_cast<float *>(db), q.splits, C, D);
+  }
+  return launch_status();
+}
+
+int feql_device_status(feql_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FEQL_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, feql::g_status, sizeof(v)) != cudaSuccess) return FEQL_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(feql::g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return FEQL_ERR_CUDA;
+  return (v & kStatusTimeout) ? FEQL_ERR_TIMEOUT : FEQL_OK;
+}
+
+const char *feql_status_string(int status) {
+  switch (status) {
+    case FEQL_OK: return "ok";
+    case FEQL_ERR_INVALID_ARG: return "invalid argument";
+    case FEQL_ERR_UNSUPPORTED: return "unsupported shape or mode";
+    case FEQL_ERR_CUDA: return "CUDA error";
+    case FEQL_ERR_TIMEOUT: return "device-side bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

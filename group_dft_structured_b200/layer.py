@@ -1,0 +1,61 @@
+"""Torch-facing convenience around the C ABI: allocates outputs, the Fourier
+weight buffer and the dW workspace with torch (device memory only) and calls
+the library.  No arithmetic happens here.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward_dw, feql_backward_dw_workspace_bytes,
+               feql_backward_dx, feql_forward, feql_weight_fft, feql_weight_fft_bytes)
+
+
+def torch_dtype(mode: int):
+    return torch.float16 if mode in (FEQL_FP16, FEQL_FP16_SIMT) else torch.float32
+
+
+def weight_fft(W: torch.Tensor, mode: int, stream=None) -> torch.Tensor:
+    D, C, _ = W.shape
+    nbytes = feql_weight_fft_bytes(C, D, mode)
+    if nbytes == 0:
+        raise ValueError("unsupported (C, D, mode)")
+    What = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    feql_weight_fft(W, What, C, D, mode, stream)
+    return What
+
+
+def forward(x: torch.Tensor, What: torch.Tensor, b, D: int, mode: int, out=None,
+            stream=None) -> torch.Tensor:
+    N, C, _ = x.shape
+    y = out if out is not None else torch.empty((N, D, 4), dtype=x.dtype, device=x.device)
+    feql_forward(x, What, b, y, N, C, D, mode, stream)
+    return y
+
+
+def backward_dx(dy: torch.Tensor, What: torch.Tensor, C: int, mode: int, out=None,
+                stream=None) -> torch.Tensor:
+    N, D, _ = dy.shape
+    dx = out if out is not None else torch.empty((N, C, 4), dtype=dy.dtype, device=dy.device)
+    feql_backward_dx(dy, What, dx, N, C, D, mode, stream)
+    return dx
+
+
+def dw_workspace(N: int, C: int, D: int, mode: int, device) -> torch.Tensor:
+    nbytes = feql_backward_dw_workspace_bytes(N, C, D, mode)
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, ws=None, out=None,
+                with_db: bool = True, stream=None):
+    N, C, _ = x.shape
+    D = dy.shape[1]
+    if ws is None:
+        ws = dw_workspace(N, C, D, mode, x.device)
+    if out is None:
+        dW = torch.empty((D, C, 4), dtype=x.dtype, device=x.device)
+        db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
+    else:
+        dW, db = out
+    feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
+    return dW, db

@@ -1,0 +1,127 @@
+/*
+ * feql.h — C ABI of the B200 (sm_100a) p4 Flash EQ-Linear library (libfeql.so).
+ *
+ * The layer (Flash EQ-Linear, technical summary "Intuizione Centrale"; arXiv
+ * abstract): the p4 equivariant linear layer is a circular convolution along
+ * the group axis (T = 4) composed with a linear map along the channels,
+ *
+ *     y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod 4] * x[n,c,s],
+ *
+ * computed exactly through a real DFT along the group axis: bins 0 and 2 are
+ * real channel contractions and bin 1 is one complex contraction (bin 3 is its
+ * conjugate), six real GEMMs of N x C x D instead of sixteen (technical
+ * summary "Specializzazione per il Gruppo di Rotazione p4"; abstract, cost
+ * 2(T-1)/T^2 of the dense form).
+ *
+ * Layouts (all row-major, contiguous, group index innermost):
+ *     x  [N][C][4]     y  [N][D][4]     W  [D][C][4]     b [D]
+ *     dy [N][D][4]     dx [N][C][4]     dW [D][C][4]     db [D]
+ * C and D count channels per group element (the unrolled widths are 4C, 4D).
+ *
+ * Conventions shared by every entry point:
+ *  - Every data pointer is a DEVICE pointer on the current CUDA device,
+ *    owned by the caller; the library allocates no device memory and keeps no
+ *    per-call state (it caches only per-device properties).
+ *  - Calls only enqueue work on `stream` (NULL = legacy default stream) and
+ *    never synchronise, except feql_device_status.
+ *  - Element type of x, y, W, b, dy, dx, dW, db follows `dtype`:
+ *    FEQL_FP16* -> IEEE binary16, FEQL_FP32* -> binary32.  Accumulation is
+ *    fp32 in every mode.
+ *  - Pointers must be 16-byte aligned.  Inputs and outputs must not overlap.
+ *  - Return value: FEQL_OK, or an feql_status code; on an error nothing is
+ *    enqueued (FEQL_ERR_CUDA: a launch failed; see feql_status_string).
+ *  - N == 0 is a valid no-op (for feql_backward_dw it zeroes dW and db).
+ */
+#ifndef FEQL_H
+#define FEQL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *feql_stream;
+
+/* Arithmetic mode. */
+typedef enum {
+  FEQL_FP16 = 0,        /* fp16 data, fp32 accumulate, tcgen05 tensor cores */
+  FEQL_FP32 = 1,        /* fp32 data; the library picks FEQL_FP32_SIMT or FEQL_FP32_3XTF32 */
+  FEQL_FP32_SIMT = 2,   /* fp32 data, fp32 FMA on CUDA cores */
+  FEQL_FP32_3XTF32 = 3, /* fp32 data, split-TF32 (hi*hi + hi*lo + lo*hi) on tensor cores */
+  FEQL_FP16_SIMT = 4    /* fp16 data, fp32 FMA on CUDA cores (cross-check path) */
+} feql_dtype;
+
+typedef enum {
+  FEQL_OK = 0,
+  FEQL_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad dtype, misaligned, workspace too small */
+  FEQL_ERR_UNSUPPORTED = 2, /* shape/mode the kernels do not cover (e.g. odd C or D in fp16) */
+  FEQL_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a launch failed */
+  FEQL_ERR_TIMEOUT = 4      /* a kernel's bounded wait expired (reported by feql_device_status) */
+} feql_status;
+
+/* Size in bytes of the opaque Fourier-weight buffer What for (C, D, dtype);
+ * 0 on invalid arguments.  The layout is private to the library and depends
+ * only on (C, D, dtype). */
+size_t feql_weight_fft_bytes(int C, int D, int dtype);
+
+/* a1 — weight transform, run once per weight update (technical summary
+ * "Approccio Algoritmico": the convolution theorem needs W in the Fourier
+ * domain).  Computes the non-redundant bins of the 4-point real DFT of W
+ * along the group axis,
+ *     What0 = W0+W1+W2+W3,  What2 = W0-W1+W2-W3,  What1 = (W0-W2) + i(W3-W1),
+ * and stores them, for both the forward and the dX pass (conjugated and
+ * transposed), in the kernels' tile layout.
+ *   W    : device, [D][C][4] of dtype (read only)
+ *   What : device, feql_weight_fft_bytes(C, D, dtype) bytes (written)
+ */
+int feql_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_stream stream);
+
+/* a2–a4 — forward: 4-point rDFT of x along the group axis, the six real
+ * per-frequency channel contractions, inverse rDFT, + bias; the Fourier
+ * intermediates never leave the chip (technical summary "Implementazione":
+ * fused dataflow without intermediate global writes).
+ *   x    : device [N][C][4]           What : from feql_weight_fft (same C, D, dtype)
+ *   b    : device [D] or NULL (no bias)
+ *   y    : device [N][D][4] (written)
+ */
+int feql_forward(const void *x, const void *What, const void *b, void *y,
+                 int64_t N, int C, int D, int dtype, feql_stream stream);
+
+/* a5 — backward input gradient: dx[n,c,s] = sum_{d,t} W[d,c,(t-s) mod 4] dy[n,d,t],
+ * the same structure as the forward with conj(What)^T (contraction over D),
+ * no bias.
+ *   dy : device [N][D][4]   dx : device [N][C][4] (written) */
+int feql_backward_dx(const void *dy, const void *What, void *dx,
+                     int64_t N, int C, int D, int dtype, feql_stream stream);
+
+/* Workspace (bytes) feql_backward_dw needs for these sizes on the current device. */
+size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype);
+
+/* a6 — backward weight gradient of the loss <dy, y>:
+ *     dW[d,c,u] = sum_n sum_t dy[n,d,t] x[n,c,(t-u) mod 4],   db[d] = sum_{n,t} dy[n,d,t].
+ * Per frequency bin G_k[d,c] = sum_n dY_k[n,d] conj(X_k[n,c]) is accumulated
+ * over N in a split-K reduction, reduced in a fixed order (bit-identical run
+ * to run), then inverse-transformed.
+ *   x  : device [N][C][4]    dy : device [N][D][4]
+ *   dW : device [D][C][4] (written)    db : device [D] or NULL (written)
+ *   ws : device scratch of ws_bytes >= feql_backward_dw_workspace_bytes(...) */
+int feql_backward_dw(const void *x, const void *dy, void *dW, void *db,
+                     void *ws, size_t ws_bytes,
+                     int64_t N, int C, int D, int dtype, feql_stream stream);
+
+/* Synchronises `stream`, then returns and clears the device-side status word
+ * of the current device: FEQL_OK, or FEQL_ERR_TIMEOUT when some kernel gave up
+ * on a bounded wait since the last call (its outputs are then undefined). */
+int feql_device_status(feql_stream stream);
+
+/* Static description of a status code. */
+const char *feql_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FEQL_H */

@@ -1,0 +1,101 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/feql.h declares, validates its arguments before any
+CUDA call, and sizes the Fourier-weight buffer as documented."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import group_dft_structured_b200 as F
+from group_dft_structured_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return F.load()
+
+
+def header_functions():
+    src = open(F.HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(feql_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = header_functions()
+    for n in ["feql_weight_fft", "feql_forward", "feql_backward_dx", "feql_backward_dw",
+              "feql_weight_fft_bytes", "feql_backward_dw_workspace_bytes",
+              "feql_device_status", "feql_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_status_strings(lib):
+    assert F.feql_status_string(F.FEQL_OK) == "ok"
+    assert "invalid" in F.feql_status_string(F.FEQL_ERR_INVALID_ARG)
+    assert "timed out" in F.feql_status_string(F.FEQL_ERR_TIMEOUT)
+    assert F.feql_status_string(99) == "unknown status"
+
+
+def test_invalid_arguments_rejected_before_cuda(lib):
+    st = lib.feql_forward(None, None, None, None, 10, 4, 4, F.FEQL_FP16, None)
+    assert st == F.FEQL_ERR_INVALID_ARG
+    p = 1 << 20  # aligned fake address; never dereferenced because N < 0
+    assert lib.feql_forward(p, p, None, p, -1, 4, 4, F.FEQL_FP16, None) == F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_forward(p, p, None, p, 8, 0, 4, F.FEQL_FP16, None) == F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_forward(p, p, None, p, 8, 4, 4, 17, None) == F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_forward(p + 4, p, None, p, 8, 4, 4, F.FEQL_FP16, None) == F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_backward_dx(p, None, p, 8, 4, 4, F.FEQL_FP16, None) == F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_backward_dw(p, p, p, None, None, 0, 8, 4, 4, F.FEQL_FP16, None) == \
+        F.FEQL_ERR_INVALID_ARG
+    assert lib.feql_weight_fft(None, p, 4, 4, F.FEQL_FP16, None) == F.FEQL_ERR_INVALID_ARG
+    # odd channel counts cannot be tiled by TMA in fp16 (row stride not a multiple of 16 B)
+    assert lib.feql_forward(p, p, None, p, 8, 3, 4, F.FEQL_FP16, None) == F.FEQL_ERR_UNSUPPORTED
+    assert lib.feql_weight_fft(p, p, 4, 5, F.FEQL_FP16, None) == F.FEQL_ERR_UNSUPPORTED
+
+
+def _tc_plan(Ci, Do):
+    nD = -(-Do // 128)
+    BD = -(-(-(-Do // nD)) // 16) * 16
+    nK = -(-Ci // 16)
+    return nD, BD, nK, nD * nK * 6 * BD * 16 * 2
+
+
+@pytest.mark.parametrize("C,D", [(16, 16), (48, 192), (192, 192), (256, 256), (24, 96), (6, 40)])
+def test_weight_buffer_sizes(lib, C, D):
+    def al(v):
+        return -(-v // 1024) * 1024
+    tc = al(_tc_plan(C, D)[3]) + al(_tc_plan(D, C)[3])
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16) == tc
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32_SIMT) == 2 * 4 * C * D * 4
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32) == 2 * 4 * C * D * 4
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16_SIMT) == 2 * 4 * C * D * 4
+    assert F.feql_weight_fft_bytes(0, D, F.FEQL_FP16) == 0
+
+
+def test_tile_plans_cover_the_workloads():
+    # output-channel tiles of at most 128 (complex-bin MMA N = 2*BD <= 256)
+    assert _tc_plan(48, 192)[:2] == (2, 96)
+    assert _tc_plan(192, 192)[:2] == (2, 96)
+    assert _tc_plan(256, 256)[:2] == (2, 128)
+    assert _tc_plan(24, 96)[:2] == (1, 96)
+    assert _tc_plan(96, 24)[:2] == (1, 32)
+    assert _tc_plan(16, 16)[:2] == (1, 16)
+
+
+def test_product_path_has_no_oracle_dependency():
+    pkg = os.path.dirname(F.__file__)
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(root, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), f
+                assert "feql_oracle" not in src, f
