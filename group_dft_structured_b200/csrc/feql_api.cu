@@ -14,6 +14,7 @@
 #include "plan.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
+#include "tc_dw.cuh"
 #include "tc_fwd.cuh"
 #include "wfft.cuh"
 
@@ -73,14 +74,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major fp16 matrix [rows][cols] viewed as a 2-D tensor; box = 64 cols x 128 rows,
-// 128-byte swizzle, zero fill out of range.
-int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols) {
+// Row-major fp16 matrix [rows][cols] viewed as a 2-D tensor; box = 64 cols x box_rows
+// rows, 128-byte swizzle, zero fill out of range.
+int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                  int box_rows = kBM) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return FEQL_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBM)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -192,6 +194,76 @@ DwPlan make_dw_plan(int64_t N, int C, int D, int sms) {
   return q;
 }
 
+// Tensor-core dW plan: d tiles of 128 rows, c tiles of CT <= 128 columns, the
+// token axis split so that tiles x splits fills the SMs once.
+TcDwParams make_tc_dw_plan(int64_t N, int C, int D, int sms) {
+  TcDwParams p;
+  p.N = N;
+  p.C = C;
+  p.D = D;
+  p.Cs = static_cast<int>(align_up(C, 16));
+  const int nct = static_cast<int>(cdiv(C, kDwMaxCT));
+  p.CT = static_cast<int>(align_up(cdiv(C, nct), 16));
+  p.tiles_c = static_cast<int>(cdiv(C, p.CT));
+  p.tiles_d = static_cast<int>(cdiv(D, kDwMT));
+  p.nqd_max = static_cast<int>(cdiv(D, 16) < 8 ? cdiv(D, 16) : 8);
+  p.nqc_max = p.CT / 16;
+  const int nbox = p.nqd_max + p.nqc_max;
+  // tokens per chunk: every (box, token) item of a chunk has one transform
+  // thread slot (kDwItems), and the plane buffer (8 dy chunks per bin for the
+  // M = 128 operand) stays within ~40 KB
+  p.TB = 32;
+  while (p.TB * nbox > kDwItems) p.TB /= 2;
+  const int64_t tiles = static_cast<int64_t>(p.tiles_d) * p.tiles_c;
+  int64_t s = sms / tiles;
+  if (s < 1) s = 1;
+  const int64_t max_s = cdiv(N > 0 ? N : 1, p.TB);
+  if (s > max_s) s = max_s;
+  p.split_len = align_up(cdiv(N > 0 ? N : 1, s), p.TB);
+  p.splits = static_cast<int>(cdiv(N > 0 ? N : 1, p.split_len));
+  p.raw_bytes = nbox * p.TB * 128;
+  p.plane_bytes = 4 * (8 + p.nqc_max) * p.TB * 32;
+  int cols = 32;
+  while (cols < 4 * p.CT) cols *= 2;
+  p.tmem_cols = cols;
+  p.stages = 0;
+  p.ws = nullptr;
+  p.ws_db = nullptr;
+  return p;
+}
+
+int64_t tc_dw_ws_floats(const TcDwParams &p) {
+  return static_cast<int64_t>(p.splits) * (4ll * p.D * p.Cs + p.D);
+}
+
+int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half *db, float *ws,
+                 const DeviceInfo &dev, cudaStream_t stream) {
+  if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
+  p.ws = ws;
+  p.ws_db = ws + static_cast<int64_t>(p.splits) * 4 * p.D * p.Cs;
+  const int64_t red = static_cast<int64_t>(p.C) * p.D + p.D;
+  if (p.N > 0) {
+    const int budget = dev.smem_optin - 1024;
+    p.stages = 8;
+    while (p.stages > 2 && tc_dw_smem(p).total > budget) --p.stages;
+    if (tc_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+    const int smem = tc_dw_smem(p).total + 1024;
+    CUtensorMap tm_dy, tm_x;
+    int st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB);
+    if (st != FEQL_OK) return st;
+    st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB);
+    if (st != FEQL_OK) return st;
+    if (cudaFuncSetAttribute(tc_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return FEQL_ERR_CUDA;
+    const int grid = p.tiles_d * p.tiles_c * p.splits;
+    tc_dw_kernel<<<grid, kDwThreads, smem, stream>>>(tm_dy, tm_x, p);
+  }
+  dw_tc_reduce_kernel<<<grid_for(red, 256, dev.sms), 256, 0, stream>>>(
+      p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs);
+  return launch_status();
+}
+
 }  // namespace
 
 // =============================================================================
@@ -232,9 +304,9 @@ int feql_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_str
 
 static int pass_common(const void *in, const void *What, const void *bias, void *out, int64_t N,
                        int C, int D, int dtype, feql_stream stream, int dir) {
-  if (!valid_dtype(dtype) || in == nullptr || What == nullptr || out == nullptr)
+  if (!valid_dtype(dtype) || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
     return FEQL_ERR_INVALID_ARG;
-  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
   if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
   const int dt = resolve(dtype);
@@ -268,14 +340,15 @@ size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
   if (!valid_dtype(dtype) || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
+  if (is_tc(resolve(dtype))) return static_cast<size_t>(tc_dw_ws_floats(make_tc_dw_plan(N, C, D, dev.sms))) * 4;
   return static_cast<size_t>(make_dw_plan(N, C, D, dev.sms).ws_floats) * 4;
 }
 
 int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws, size_t ws_bytes,
                      int64_t N, int C, int D, int dtype, feql_stream stream) {
-  if (!valid_dtype(dtype) || x == nullptr || dy == nullptr || dW == nullptr || ws == nullptr)
-    return FEQL_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype) || dW == nullptr || ws == nullptr) return FEQL_ERR_INVALID_ARG;
   if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws))
     return FEQL_ERR_INVALID_ARG;
   if (db != nullptr && !aligned16(db)) return FEQL_ERR_INVALID_ARG;
@@ -285,9 +358,15 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws
   DeviceInfo dev;
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (is_tc(dt)) {
+    TcDwParams p = make_tc_dw_plan(N, C, D, dev.sms);
+    if (ws_bytes < static_cast<size_t>(tc_dw_ws_floats(p)) * 4) return FEQL_ERR_INVALID_ARG;
+    return launch_tc_dw(p, x, dy, static_cast<__half *>(dW), static_cast<__half *>(db),
+                        static_cast<float *>(ws), dev, s);
+  }
   const DwPlan q = make_dw_plan(N, C, D, dev.sms);
   if (ws_bytes < static_cast<size_t>(q.ws_floats) * 4) return FEQL_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float *wsf = static_cast<float *>(ws);
   float *wsdb = wsf + static_cast<int64_t>(q.splits) * 4 * C * D;
   dim3 grid(static_cast<unsigned>(cdiv(D, kSimtTile)), static_cast<unsigned>(cdiv(C, kSimtTile)),

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -214,6 +215,12 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Two floats rounded to fp16 (RN) and packed into one 32-bit word, low half first.
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
 // ----------------------------------------------------------------------------
 // Descriptors
 // ----------------------------------------------------------------------------
@@ -237,9 +244,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 // a_mn / b_mn select MN-major.
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t M, uint32_t N, uint32_t a_fmt,
                                                   uint32_t b_fmt, uint32_t a_mn = 0,
-                                                  uint32_t b_mn = 0) {
+                                                  uint32_t b_mn = 0, uint32_t b_neg = 0) {
   return (1u << 4)              // D format: f32
-         | (a_fmt << 7) | (b_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
+         | (a_fmt << 7) | (b_fmt << 10) | (b_neg << 14) | (a_mn << 15) | (b_mn << 16) |
          ((N >> 3) << 17)       // N / 8
          | ((M >> 4) << 24);    // M / 16
 }

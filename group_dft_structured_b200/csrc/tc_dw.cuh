@@ -1,0 +1,334 @@
+// tc_dw.cuh — weight gradient on the sm_100a tensor cores (fp16 data).
+//
+// The loss <dy, y> has dW[d,c,u] = sum_n sum_t dy[n,d,t] x[n,c,(t-u) mod 4], a
+// circular cross-correlation along the group axis, so per frequency bin
+// (convolution theorem, Flash EQ-Linear technical summary "Approccio
+// Algoritmico"):
+//   G_k[d,c] = sum_n dY_k[n,d] conj(X_k[n,c])
+//   G0 = sum dY0 X0,  G2 = sum dY2 X2,
+//   Re G1 = sum dY1r X1r + dY1i X1i,  Im G1 = sum dY1i X1r - dY1r X1i
+// — six real N-contractions — and dW = irDFT_4(G) (applied by the reduce).
+// db[d] = sum_n dY0[n,d] comes out of the same rDFT.
+//
+// Work unit (one per CTA): a 128-row d tile x a CT-column c tile x a token
+// split.  Per chunk of TB tokens:
+//   warp 0      TMA: the d-tile's dy boxes and the c-tile's x boxes (16
+//               channels x 4 group elements x TB tokens each) into a raw ring
+//   warps 2..5  4-point rDFT of every (token, channel) fibre into fp16 planes
+//               laid out MN-major (channel contiguous, token = K), 32-byte
+//               swizzle; db partial sums in registers
+//   warp 1      TMEM allocator + MMA issuer: per 16 tokens six M=128 x N=CT
+//               MMAs, the -Im X1 term through the B-negate bit
+// After the last chunk warps 2..5 read the four fp32 accumulators out of
+// TMEM and write them to the workspace; dw_tc_reduce_kernel sums the splits
+// in a fixed order (bit-identical run to run) and applies the inverse rDFT.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "plan.cuh"
+#include "sm100.cuh"
+
+namespace feql {
+
+constexpr int kDwThreads = 192;
+constexpr int kDwMT = 128;       // d rows per tile (MMA M)
+constexpr int kDwMaxCT = 128;    // c columns per tile (MMA N; 4 accumulators <= 512 TMEM cols)
+constexpr int kDwItems = 256;    // (box, token) items per chunk: nbox * TB
+
+struct TcDwParams {
+  int64_t N;
+  int C, D, Cs;          // Cs: workspace row stride (C rounded up to 16)
+  int CT;                // c columns per tile
+  int nqd_max, nqc_max;  // 16-channel boxes per tile (dy, x) in the plane layout
+  int tiles_d, tiles_c, splits;
+  int64_t split_len;     // tokens per split (multiple of TB)
+  int TB;                // tokens per chunk
+  int stages;            // raw ring depth
+  int raw_bytes;         // (nqd_max + nqc_max) * TB * 128
+  int plane_bytes;       // 4 * (8 + nqc_max) * TB * 32
+  int tmem_cols;
+  float *ws;             // [splits][4][D][Cs]
+  float *ws_db;          // [splits][D]
+};
+
+struct DwSmem {
+  int raw0, plane0, bars, total;
+};
+
+__host__ __device__ inline DwSmem tc_dw_smem(const TcDwParams &p) {
+  DwSmem s;
+  s.raw0 = 0;
+  s.plane0 = p.stages * p.raw_bytes;
+  s.bars = s.plane0 + 2 * p.plane_bytes;
+  s.total = s.bars + (2 * p.stages + 2 * 2 + 1) * 8 + 16;
+  return s;
+}
+
+__global__ void __launch_bounds__(kDwThreads, 1)
+tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
+             const TcDwParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const DwSmem L = tc_dw_smem(p);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *full = bars;                 // raw slot landed (TMA tx)
+  uint64_t *empty = bars + p.stages;     // raw slot read by the transform (4 warps)
+  uint64_t *pfull = bars + 2 * p.stages; // plane buffer written (4 warps)
+  uint64_t *pempty = pfull + 2;          // plane buffer consumed (MMA commit)
+  uint64_t *acc_full = pempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int u = blockIdx.x;
+  const int tiles = p.tiles_d * p.tiles_c;
+  const int split = u / tiles, ti = (u % tiles) / p.tiles_c, tj = u % p.tiles_c;
+  const int64_t t_begin = static_cast<int64_t>(split) * p.split_len;
+  int64_t t_end = t_begin + p.split_len;
+  if (t_end > p.N) t_end = p.N;
+  const int nchunks = t_begin < t_end ? static_cast<int>(cdiv(t_end - t_begin, p.TB)) : 0;
+  int nqd = static_cast<int>(cdiv(p.D - ti * kDwMT, 16));
+  if (nqd > p.nqd_max) nqd = p.nqd_max;
+  int nqc = static_cast<int>(cdiv(p.C - tj * p.CT, 16));
+  if (nqc > p.nqc_max) nqc = p.nqc_max;
+  const int nbox = nqd + nqc;
+  const int chunk_plane = p.TB * 32;  // bytes of one 16-channel plane chunk
+  const int x_off = 4 * 8 * chunk_plane;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pfull[b], 4);
+      mbar_init(&pempty[b], 1);
+    }
+    mbar_init(acc_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_dy);
+      tma_prefetch_desc(&tm_x);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ch = 0; ch < nchunks; ++ch) {
+        if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
+        if (ok) {
+          uint8_t *raw = smem + L.raw0 + s * p.raw_bytes;
+          const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * p.TB);
+          mbar_arrive_expect_tx(&full[s], nbox * p.TB * 128);
+          for (int q = 0; q < nqd; ++q)
+            tma_load_2d(raw + q * p.TB * 128, &tm_dy, (ti * kDwMT + q * 16) * kT, row, &full[s]);
+          for (int q = 0; q < nqc; ++q)
+            tma_load_2d(raw + (nqd + q) * p.TB * 128, &tm_x, (tj * p.CT + q * 16) * kT, row,
+                        &full[s]);
+        }
+        if (++s == p.stages) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id = instr_desc(kDwMT, p.CT, 0, 0, 1, 1);
+      const uint32_t id_neg = instr_desc(kDwMT, p.CT, 0, 0, 1, 1, 1);
+      const uint32_t lbo = chunk_plane, sbo = 256;
+      const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
+      const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
+      for (int ch = 0; ch < nchunks; ++ch) {
+        const int pb = ch & 1;
+        if (ok) ok = mbar_wait(&pfull[pb], (ch >> 1) & 1);
+        tc_fence_after();
+        if (ok) {
+          const uint32_t pl = smem_u32(smem + L.plane0 + pb * p.plane_bytes);
+          for (int k = 0; k < p.TB / 16; ++k) {
+            const uint32_t ko = k * 512;  // 16 tokens x 32 B
+            auto A = [&](int bin) { return smem_desc(pl + bin * 8 * chunk_plane + ko, lbo, sbo, kSw32); };
+            auto B = [&](int bin) {
+              return smem_desc(pl + x_off + bin * p.nqc_max * chunk_plane + ko, lbo, sbo, kSw32);
+            };
+            const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
+            mma_f16_ss(acc0, A(0), B(0), id, first);
+            mma_f16_ss(acc2, A(1), B(1), id, first);
+            mma_f16_ss(acc1r, A(2), B(2), id, first);
+            mma_f16_ss(acc1r, A(3), B(3), id, 1u);
+            mma_f16_ss(acc1i, A(3), B(2), id, first);
+            mma_f16_ss(acc1i, A(2), B(3), id_neg, 1u);
+          }
+          mma_commit(&pempty[pb]);
+        }
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    // ---------------------------------------------------------- transform
+    const int t = threadIdx.x - 64;
+    const bool do_db = tj == 0;
+    float db_acc[2][16];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) db_acc[k][c] = 0.f;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int ch = 0; ch < nchunks; ++ch) {
+      const int pb = ch & 1;
+      if (ok) ok = mbar_wait(&full[s], ph);
+      if (ok) ok = mbar_wait(&pempty[pb], ((ch >> 1) & 1) ^ 1);
+      const uint8_t *raw = smem + L.raw0 + s * p.raw_bytes;
+      uint8_t *planes = smem + L.plane0 + pb * p.plane_bytes;
+#pragma unroll
+      for (int k = 0; k < kDwItems / 128; ++k) {
+        const int e = t + 128 * k;
+        const int b = e / p.TB, r = e % p.TB;
+        if (b >= nbox) continue;
+        const uint8_t *src = raw + b * p.TB * 128 + r * 128;
+        uint32_t pl[4][8];
+        float y0[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
+          const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+          float f[2][4];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float2 lo = __half22float2(h[2 * c]), hi = __half22float2(h[2 * c + 1]);
+            const float a = lo.x + hi.x, bb = lo.y + hi.y;
+            f[c][0] = a + bb;
+            f[c][1] = a - bb;
+            f[c][2] = lo.x - hi.x;
+            f[c][3] = hi.y - lo.y;
+          }
+          y0[2 * q] = f[0][0];
+          y0[2 * q + 1] = f[1][0];
+#pragma unroll
+          for (int pp = 0; pp < 4; ++pp) pl[pp][q] = pack_half2(f[0][pp], f[1][pp]);
+        }
+        uint8_t *dst = b < nqd ? planes + b * chunk_plane
+                               : planes + x_off + (b - nqd) * chunk_plane;
+        const int pstride = b < nqd ? 8 * chunk_plane : p.nqc_max * chunk_plane;
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          uint8_t *row = dst + pp * pstride + r * 32;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            *reinterpret_cast<uint4 *>(row + (((hh ^ (r >> 2)) & 1) << 4)) =
+                make_uint4(pl[pp][4 * hh + 0], pl[pp][4 * hh + 1], pl[pp][4 * hh + 2],
+                           pl[pp][4 * hh + 3]);
+        }
+        if (do_db && b < nqd) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) db_acc[k][c] += y0[c];
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) {
+        mbar_arrive(&empty[s]);
+        mbar_arrive(&pfull[pb]);
+      }
+      if (++s == p.stages) { s = 0; ph ^= 1; }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait(acc_full, 0);
+    tc_fence_after();
+    const int quad = warp & 3;
+    const int d = ti * kDwMT + quad * 32 + lane;
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const int ncol = p.CT / 16;
+    for (int bin = 0; bin < 4; ++bin) {
+      float *dst = p.ws + ((static_cast<int64_t>(split) * 4 + bin) * p.D + d) * p.Cs +
+                   static_cast<int64_t>(tj) * p.CT;
+      for (int g = 0; g < ncol; ++g) {
+        uint32_t v[16];
+        tmem_ld16(tl + bin * p.CT + g * 16, v);
+        tmem_ld_wait();
+        if (d < p.D && tj * p.CT + g * 16 < p.C) {
+          float4 *o = reinterpret_cast<float4 *>(dst + g * 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+
+    // db: fixed-order reduction of the per-thread partials through shared memory
+    if (do_db) {
+      named_bar_sync(3, 128);  // raw ring is free: every chunk has been consumed
+      float *sdb = reinterpret_cast<float *>(smem + L.raw0);  // [kDwItems][16]
+#pragma unroll
+      for (int k = 0; k < kDwItems / 128; ++k)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) sdb[(t + 128 * k) * 16 + c] = db_acc[k][c];
+      named_bar_sync(3, 128);
+      if (t < nqd * 16) {
+        const int b = t / 16, c = t % 16;
+        float sum = 0.f;
+        for (int r = 0; r < p.TB; ++r) sum += sdb[(b * p.TB + r) * 16 + c];
+        const int dd = ti * kDwMT + b * 16 + c;
+        if (dd < p.D) p.ws_db[static_cast<int64_t>(split) * p.D + dd] = sum;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+// Sum of the split partials in a fixed order, inverse rDFT, fp16 cast:
+//   dW[d][c][u] = (G0 + (-1)^u G2)/4 + Re(G1 i^u)/2,   db[d] = sum of partials.
+__global__ void dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
+                                    __half *__restrict__ dW, __half *__restrict__ db, int splits,
+                                    int C, int D, int Cs) {
+  const int64_t plane = static_cast<int64_t>(D) * Cs;
+  const int64_t n = static_cast<int64_t>(D) * C;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n + D;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (e < n) {
+      const int64_t d = e / C, c = e % C;
+      const float *src = ws + d * Cs + c;
+      float g0 = 0.f, g2 = 0.f, g1r = 0.f, g1i = 0.f;
+      for (int s = 0; s < splits; ++s) {
+        const float *q = src + static_cast<int64_t>(s) * 4 * plane;
+        g0 += q[0];
+        g2 += q[plane];
+        g1r += q[2 * plane];
+        g1i += q[3 * plane];
+      }
+      const float ev = 0.25f * (g0 + g2), od = 0.25f * (g0 - g2);
+      __half2 lo = __floats2half2_rn(ev + 0.5f * g1r, od - 0.5f * g1i);
+      __half2 hi = __floats2half2_rn(ev - 0.5f * g1r, od + 0.5f * g1i);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t *>(&lo);
+      pk.y = *reinterpret_cast<uint32_t *>(&hi);
+      *reinterpret_cast<uint2 *>(dW + e * kT) = pk;
+    } else if (db != nullptr) {
+      const int d = static_cast<int>(e - n);
+      float sum = 0.f;
+      for (int s = 0; s < splits; ++s) sum += ws_db[static_cast<int64_t>(s) * D + d];
+      db[d] = __float2half_rn(sum);
+    }
+  }
+}
+
+}  // namespace feql

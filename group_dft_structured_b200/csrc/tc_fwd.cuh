@@ -66,11 +66,6 @@ __host__ __device__ inline TcSmem tc_fwd_smem(const TcFwdParams &p) {
   return s;
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
-
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
                        const __grid_constant__ CUtensorMap tm_out, const TcFwdParams p) {

@@ -30,7 +30,8 @@
  *  - Pointers must be 16-byte aligned.  Inputs and outputs must not overlap.
  *  - Return value: FEQL_OK, or an feql_status code; on an error nothing is
  *    enqueued (FEQL_ERR_CUDA: a launch failed; see feql_status_string).
- *  - N == 0 is a valid no-op (for feql_backward_dw it zeroes dW and db).
+ *  - N == 0 is a valid no-op (for feql_backward_dw it zeroes dW and db); the
+ *    token-indexed pointers (x, y, dy, dx) may then be NULL.
  */
 #ifndef FEQL_H
 #define FEQL_H
