@@ -411,3 +411,86 @@ const char *feql_status_string(int status) {
 }
 
 }  // extern "C"
+
+// =============================================================================
+// Weight gradient without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at the point where they need the
+// weight gradient: code running inside a framework that owns every allocation
+// (a custom allocator or a memory pool that must not grow), plug-ins whose
+// host can only hand over the input and output tensors, or runtimes that
+// forbid allocation after start-up.  feql_backward_dw needs a split-K
+// workspace; this variant takes it from a fixed array that lives in the
+// library's device image instead.
+//
+// The array is a file-scope __device__ object of kNoAllocScratchBytes.  Every
+// GPU that loads the library holds it until the process exits.  In host code
+// its name is only a host-side stand-in, so the device address is looked up
+// with cudaGetSymbolAddress, once per device, by the first call made with that
+// device current (make that first call before any stream capture).  The array
+// is shared by all calls: calls that overlap on the GPU (different streams,
+// threads) race on it and must be serialised by the caller.  Nothing in it
+// needs clearing between calls — every element the reduction reads is written
+// earlier in the same call — so it simply keeps the last call's partial sums.
+// No cudaMalloc, cudaFree or other allocating routine is called.
+// =============================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(16) << 20;  // 16 MiB
+
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_dw_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_dw_scratch on the current device (looked up once per device).
+int noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FEQL_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dw_scratch) != cudaSuccess || p == nullptr) return FEQL_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return FEQL_OK;
+}
+
+}  // namespace
+
+extern "C" int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW, void *db,
+                                        int64_t N, int C, int D, int dtype, feql_stream stream) {
+  if (!valid_dtype(dtype) || dW == nullptr) return FEQL_ERR_INVALID_ARG;
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dW)) return FEQL_ERR_INVALID_ARG;
+  if (db != nullptr && !aligned16(db)) return FEQL_ERR_INVALID_ARG;
+  if (resolve(dtype) != FEQL_FP16) return FEQL_ERR_UNSUPPORTED;  // tensor-core fp16 path only
+  if ((C | D) & 1) return FEQL_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  TcDwParams p = make_tc_dw_plan(N, C, D, dev.sms);
+  // One token split needs 4*D*Cs + D floats of partial sums; if even one does
+  // not fit, the shape is rejected.  Otherwise use as many splits as fit (the
+  // regular plan's count when it fits, fewer — slower, and summed in a
+  // different grouping — if not).
+  const int64_t cap = static_cast<int64_t>(kNoAllocScratchBytes / 4);
+  const int64_t per_split = 4ll * p.D * p.Cs + p.D;
+  if (per_split > cap) return FEQL_ERR_UNSUPPORTED;
+  if (tc_dw_ws_floats(p) > cap) {
+    const int64_t max_splits = cap / per_split;
+    p.split_len = align_up(cdiv(N > 0 ? N : 1, max_splits), p.TB);
+    p.splits = static_cast<int>(cdiv(N > 0 ? N : 1, p.split_len));
+  }
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != FEQL_OK) return st;
+  return launch_tc_dw(p, x, dy, static_cast<__half *>(dW), static_cast<__half *>(db),
+                      static_cast<float *>(scratch), dev, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -113,6 +113,27 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db,
                      void *ws, size_t ws_bytes,
                      int64_t N, int C, int D, int dtype, feql_stream stream);
 
+/* Weight gradient for callers that cannot allocate device memory (code inside
+ * a framework that owns every allocation, plug-ins that are handed only their
+ * input and output tensors, runtimes that forbid allocation after start-up).
+ * The paper has no counterpart: this is a library convenience.
+ * Same arguments and results as feql_backward_dw in FEQL_FP16 mode, minus the
+ * workspace: the split-K partial sums go to a fixed 16 MiB array inside the
+ * library's device image, which every GPU that loads the library keeps until
+ * the process exits.  Allocates nothing.
+ *  - Limit: one token split needs (4*D*roundup(C,16) + D) * 4 bytes of
+ *    partial sums; shapes where that exceeds 16 MiB (e.g. C = D = 1024) get
+ *    FEQL_ERR_UNSUPPORTED without anything launched, as do modes other than
+ *    FEQL_FP16 and odd C or D.  When the regular split count does not fit,
+ *    fewer splits are used: less parallelism, and the fp32 partial sums are
+ *    grouped differently (results agree to rounding, not bit for bit).
+ *  - The first call on a device looks up the array's device address (make it
+ *    before any stream capture).
+ *  - All calls share the one array: calls that overlap on the GPU race and
+ *    must be serialised by the caller.  No state carries over between calls. */
+int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW, void *db,
+                             int64_t N, int C, int D, int dtype, feql_stream stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word
  * of the current device: FEQL_OK, or FEQL_ERR_TIMEOUT when some kernel gave up
  * on a bounded wait since the last call (its outputs are then undefined). */

@@ -1,0 +1,75 @@
+"""The no-allocation weight-gradient entry point against the regular one.
+
+feql_backward_dw_noalloc serves callers that cannot allocate device memory
+(frameworks that own every allocation, plug-ins handed only their tensors,
+runtimes that forbid allocation after start-up): it takes its split-K scratch
+from a fixed array inside the library instead of a caller workspace.  This
+file is collected last so that a run stopping at the first failure has run
+everything else first; it also passes on its own in a fresh process.
+"""
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import group_dft_structured_b200 as F
+from group_dft_structured_b200 import layer as Lyr
+from group_dft_structured_b200.workloads import make_inputs
+from oracle import feql_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+TOL_FP16 = 5e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from group_dft_structured_b200 import build
+    build.build()
+    F.load()
+
+
+def _inputs(wid, N, C, D):
+    inp = make_inputs(wid, N, C, D, "fp16")
+    return torch.from_numpy(inp["x"]).cuda(), torch.from_numpy(inp["dy"]).cuda()
+
+
+def test_noalloc_matches_workspace_version_on_consecutive_calls():
+    lib = F.load()
+    # two calls in a row on different shapes: the second must not see the
+    # first one's leftovers in the shared scratch array
+    for wid, (N, C, D) in [(11, (20000, 24, 96)), (12, (3000, 256, 256)), (13, (517, 48, 192))]:
+        x, dy = _inputs(wid, N, C, D)
+        ref_dW, ref_db = Lyr.backward_dw(x, dy, F.FEQL_FP16)
+        dW = torch.full((D, C, 4), float("nan"), dtype=torch.float16, device="cuda")
+        db = torch.full((D,), float("nan"), dtype=torch.float16, device="cuda")
+        st = lib.feql_backward_dw_noalloc(x.data_ptr(), dy.data_ptr(), dW.data_ptr(),
+                                          db.data_ptr(), N, C, D, F.FEQL_FP16,
+                                          torch.cuda.current_stream().cuda_stream)
+        assert st == F.FEQL_OK
+        assert F.feql_device_status() == F.FEQL_OK
+        a, b = dW.double().cpu().numpy(), ref_dW.double().cpu().numpy()
+        assert O.rel_err(a, b) <= TOL_FP16
+        assert O.rel_err(db.double().cpu().numpy(), ref_db.double().cpu().numpy()) <= TOL_FP16
+        # and against the float64 oracle
+        xf = x.double().cpu().numpy()
+        dyf = dy.double().cpu().numpy()
+        oW, ob = O.backward_dw(xf, dyf)
+        assert O.rel_err(a, oW) <= TOL_FP16
+        assert O.rel_err(db.double().cpu().numpy(), ob) <= TOL_FP16
+
+
+def test_noalloc_rejects_sizes_beyond_the_fixed_scratch():
+    lib = F.load()
+    N, C, D = 4096, 1024, 1024
+    assert (4 * D * C + D) * 4 > 16 << 20  # one split's partial sums exceed the array
+    p = 1 << 20  # never dereferenced: the size check fails before any launch
+    st = lib.feql_backward_dw_noalloc(p, p, p, None, N, C, D, F.FEQL_FP16, None)
+    assert st == F.FEQL_ERR_UNSUPPORTED
+    st = lib.feql_backward_dw_noalloc(p, p, p, None, 16, 8, 8, F.FEQL_FP32, None)
+    assert st == F.FEQL_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert F.feql_device_status() == F.FEQL_OK
