@@ -136,26 +136,44 @@ int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __h
   p.chunk_bytes = P.chunk_bytes;
   const int64_t nM = cdiv(N, kBM);
   if (nM * P.nD > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  p.nM = static_cast<int>(nM);
   p.n_units = static_cast<int>(nM * P.nD);
   p.nacc = (4 * P.BD <= 256) ? 2 : 1;
   p.acc_stride = p.nacc == 2 ? 256 : 0;
-  p.stage_bytes = kXChunkBytes + static_cast<int>(align_up(P.chunk_bytes, 1024));
   p.bias_floats = P.nD * P.BD;
   const int budget = dev.smem_optin - 1024;  // 1 KB for aligning the base
+  // Resident weights when the CTA's slice fits beside >= 4 input stages and
+  // there are enough CTAs for one fixed output tile each.
+  p.resident = 1;
+  p.wres_bytes = static_cast<int>(align_up(static_cast<int64_t>(P.nK) * P.chunk_bytes, 1024));
+  p.stage_bytes = kXChunkBytes;
   p.stages = 8;
-  while (p.stages > 2 && tc_fwd_smem(p).total > budget) --p.stages;
-  if (tc_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  while (p.stages > 4 && tc_fwd_smem(p).total > budget) --p.stages;
+  if (tc_fwd_smem(p).total > budget || dev.sms < P.nD) {
+    p.resident = 0;
+    p.wres_bytes = 0;
+    p.stage_bytes = kXChunkBytes + static_cast<int>(align_up(P.chunk_bytes, 1024));
+    p.stages = 8;
+    while (p.stages > 2 && tc_fwd_smem(p).total > budget) --p.stages;
+    if (tc_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  }
   const int smem = tc_fwd_smem(p).total + 1024;
+  int grid;
+  if (p.resident) {
+    const int64_t per_tile = nM < dev.sms / P.nD ? nM : dev.sms / P.nD;  // CTAs per output tile
+    grid = static_cast<int>(per_tile * P.nD);
+  } else {
+    grid = p.n_units < dev.sms ? p.n_units : dev.sms;
+  }
 
   CUtensorMap tm_in, tm_out;
   st = make_tmap_f16(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT);
   if (st != FEQL_OK) return st;
-  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT);
+  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT, kOutRows);
   if (st != FEQL_OK) return st;
   if (cudaFuncSetAttribute(tc_fourier_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return FEQL_ERR_CUDA;
-  const int grid = p.n_units < dev.sms ? p.n_units : dev.sms;
   tc_fourier_gemm_kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, tm_out, p);
   return launch_status();
 }
@@ -241,7 +259,6 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
   if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
   p.ws = ws;
   p.ws_db = ws + static_cast<int64_t>(p.splits) * 4 * p.D * p.Cs;
-  const int64_t red = static_cast<int64_t>(p.C) * p.D + p.D;
   if (p.N > 0) {
     const int budget = dev.smem_optin - 1024;
     p.stages = 8;
@@ -259,7 +276,9 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     const int grid = p.tiles_d * p.tiles_c * p.splits;
     tc_dw_kernel<<<grid, kDwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  dw_tc_reduce_kernel<<<grid_for(red, 256, dev.sms), 256, 0, stream>>>(
+  const int64_t rblocks = dw_reduce_blocks(p.C, p.D);
+  if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dw_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), kRedOut * kRedGroups, 0, stream>>>(
       p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs);
   return launch_status();
 }

@@ -29,13 +29,17 @@ struct TcPlan {
   int64_t bytes;     // nD * nK * chunk_bytes
 };
 
+// Output-channel tile: short contractions (<= 4 chunks) are epilogue-bound, so
+// they take BD <= 64 and the four accumulators (4*BD <= 256 columns) can be
+// double-buffered in TMEM; long contractions take BD up to 128 so that fewer
+// tiles re-read and re-transform the input.
 __host__ __device__ inline TcPlan make_tc_plan(int Ci, int Do) {
   TcPlan p;
   p.Ci = Ci;
   p.Do = Do;
-  p.nD = static_cast<int>(cdiv(Do, kMaxBD));
-  p.BD = static_cast<int>(align_up(cdiv(Do, p.nD), 16));
   p.nK = static_cast<int>(cdiv(Ci, kCK));
+  p.nD = static_cast<int>(cdiv(Do, p.nK <= 4 ? kMaxBD / 2 : kMaxBD));
+  p.BD = static_cast<int>(align_up(cdiv(Do, p.nD), 16));
   p.chunk_bytes = 6 * p.BD * kCK * 2;
   p.bytes = static_cast<int64_t>(p.nD) * p.nK * p.chunk_bytes;
   return p;
@@ -51,7 +55,8 @@ __host__ __device__ inline int sw32_offset(int row, int k) {
 // Layout of the opaque What buffer.
 //   fp16 tensor-core modes: [fwd chunks][dx chunks], each direction laid out
 //       [tile j][chunk kc][rows 0..6BD) with rows
-//       [0,BD) What0 | [BD,2BD) What2 | [2BD,4BD) (Re1 ; Im1) | [4BD,6BD) (-Im1 ; Re1)
+//       [0,BD) What0 | [BD,2BD) What2 | [2BD,4BD) (Re1 ; Im1) | [4BD,6BD) (Im1 ; -Re1)
+//   (the last block multiplies the stored -Im X1 plane)
 //   SIMT modes: fp32 planes [dir][bin p][Do][Ci], p = (0, 2, Re 1, Im 1).
 struct WhatLayout {
   bool tc;

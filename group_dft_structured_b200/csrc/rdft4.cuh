@@ -1,0 +1,38 @@
+// rdft4.cuh — the p4 group-axis butterflies on packed fp16 pairs.
+//
+// Flash EQ-Linear, technical summary "Specializzazione per il Gruppo di
+// Rotazione p4": the 4-point DFT has entries 0 and +-1 only, so the
+// non-redundant bins of a real fibre (v0, v1, v2, v3) are sums and
+// differences:
+//   V0 = (v0+v2) + (v1+v3),  V2 = (v0+v2) - (v1+v3),
+//   Re V1 = v0 - v2,         Im V1 = v3 - v1.
+// The kernels store -Im V1 = v1 - v3 (one subtraction fewer per pair); every
+// consumer of that plane carries the sign instead (weight tiles, MMA negate
+// bits).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace feql {
+
+__device__ __forceinline__ __half2 as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+__device__ __forceinline__ uint32_t as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// One 16-byte chunk = two channels x four group elements (fp16), i.e. words
+// (c0: v0 v1), (c0: v2 v3), (c1: v0 v1), (c1: v2 v3).  Returns the four bins of
+// both channels as packed pairs (channel c0 in the low half):
+//   b0 = V0, b2 = V2, b1r = Re V1, b1n = -Im V1.
+__device__ __forceinline__ void rdft4_pair(const uint4 &v, uint32_t &b0, uint32_t &b2,
+                                           uint32_t &b1r, uint32_t &b1n) {
+  const __half2 a0 = as_h2(v.x), c0 = as_h2(v.y), a1 = as_h2(v.z), c1 = as_h2(v.w);
+  const __half2 s0 = __hadd2(a0, c0), d0 = __hsub2(a0, c0);  // (v0+v2, v1+v3), (v0-v2, v1-v3)
+  const __half2 s1 = __hadd2(a1, c1), d1 = __hsub2(a1, c1);
+  const __half2 p = __lows2half2(s0, s1), q = __highs2half2(s0, s1);
+  b0 = as_u32(__hadd2(p, q));
+  b2 = as_u32(__hsub2(p, q));
+  b1r = as_u32(__lows2half2(d0, d1));
+  b1n = as_u32(__highs2half2(d0, d1));
+}
+
+}  // namespace feql

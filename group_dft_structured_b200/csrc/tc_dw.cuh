@@ -14,12 +14,13 @@
 // split.  Per chunk of TB tokens:
 //   warp 0      TMA: the d-tile's dy boxes and the c-tile's x boxes (16
 //               channels x 4 group elements x TB tokens each) into a raw ring
-//   warps 2..5  4-point rDFT of every (token, channel) fibre into fp16 planes
-//               laid out MN-major (channel contiguous, token = K), 32-byte
-//               swizzle; db partial sums in registers
+//   warps 2..9  4-point rDFT (packed fp16 pairs) of every (token, channel)
+//               fibre into planes X0, X2, Re X1, -Im X1 laid out MN-major
+//               (channel contiguous, token = K), 32-byte swizzle; one
+//               (16-channel box, token) item per thread; db partial sums
 //   warp 1      TMEM allocator + MMA issuer: per 16 tokens six M=128 x N=CT
-//               MMAs, the -Im X1 term through the B-negate bit
-// After the last chunk warps 2..5 read the four fp32 accumulators out of
+//               MMAs, one of them through the B-negate bit
+// After the last chunk warps 2..9 read the four fp32 accumulators out of
 // TMEM and write them to the workspace; dw_tc_reduce_kernel sums the splits
 // in a fixed order (bit-identical run to run) and applies the inverse rDFT.
 #pragma once
@@ -27,14 +28,16 @@
 #include <cuda_fp16.h>
 
 #include "plan.cuh"
+#include "rdft4.cuh"
 #include "sm100.cuh"
 
 namespace feql {
 
-constexpr int kDwThreads = 192;
+constexpr int kDwXfWarps = 8;     // transform (then epilogue) warps
+constexpr int kDwThreads = 64 + kDwXfWarps * 32;
 constexpr int kDwMT = 128;       // d rows per tile (MMA M)
 constexpr int kDwMaxCT = 128;    // c columns per tile (MMA N; 4 accumulators <= 512 TMEM cols)
-constexpr int kDwItems = 256;    // (box, token) items per chunk: nbox * TB
+constexpr int kDwItems = kDwXfWarps * 32;  // (box, token) items per chunk: nbox * TB
 
 struct TcDwParams {
   int64_t N;
@@ -74,8 +77,8 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
   const DwSmem L = tc_dw_smem(p);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *full = bars;                 // raw slot landed (TMA tx)
-  uint64_t *empty = bars + p.stages;     // raw slot read by the transform (4 warps)
-  uint64_t *pfull = bars + 2 * p.stages; // plane buffer written (4 warps)
+  uint64_t *empty = bars + p.stages;     // raw slot read by the transform warps
+  uint64_t *pfull = bars + 2 * p.stages; // plane buffer written by the transform warps
   uint64_t *pempty = pfull + 2;          // plane buffer consumed (MMA commit)
   uint64_t *acc_full = pempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
@@ -99,10 +102,10 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 4);
+      mbar_init(&empty[s], kDwXfWarps);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&pfull[b], 4);
+      mbar_init(&pfull[b], kDwXfWarps);
       mbar_init(&pempty[b], 1);
     }
     mbar_init(acc_full, 1);
@@ -142,6 +145,9 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
+    // The planes hold -Im of bin 1 (for dy and x alike), so
+    //   Re G1 = dY1r X1r + (-dY1i)(-X1i),   Im G1 = -(-dY1i) X1r + dY1r (-X1i),
+    // the first Im term through the B-negate bit.
     if (lane == 0) {
       const uint32_t id = instr_desc(kDwMT, p.CT, 0, 0, 1, 1);
       const uint32_t id_neg = instr_desc(kDwMT, p.CT, 0, 0, 1, 1, 1);
@@ -165,8 +171,8 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
             mma_f16_ss(acc2, A(1), B(1), id, first);
             mma_f16_ss(acc1r, A(2), B(2), id, first);
             mma_f16_ss(acc1r, A(3), B(3), id, 1u);
-            mma_f16_ss(acc1i, A(3), B(2), id, first);
-            mma_f16_ss(acc1i, A(2), B(3), id_neg, 1u);
+            mma_f16_ss(acc1i, A(3), B(2), id_neg, first);
+            mma_f16_ss(acc1i, A(2), B(3), id, 1u);
           }
           mma_commit(&pempty[pb]);
         }
@@ -175,51 +181,32 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     }
   } else {
     // ---------------------------------------------------------- transform
+    // one (box, token) item per thread and chunk
     const int t = threadIdx.x - 64;
-    const bool do_db = tj == 0;
-    float db_acc[2][16];
+    const int b = t / p.TB, r = t % p.TB;
+    const bool active = b < nbox;
+    const bool is_dy = b < nqd;
+    const bool do_db = tj == 0 && is_dy;
+    float db_acc[16];
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-      for (int c = 0; c < 16; ++c) db_acc[k][c] = 0.f;
+    for (int c = 0; c < 16; ++c) db_acc[c] = 0.f;
     int s = 0;
     uint32_t ph = 0;
     for (int ch = 0; ch < nchunks; ++ch) {
       const int pb = ch & 1;
       if (ok) ok = mbar_wait(&full[s], ph);
       if (ok) ok = mbar_wait(&pempty[pb], ((ch >> 1) & 1) ^ 1);
-      const uint8_t *raw = smem + L.raw0 + s * p.raw_bytes;
-      uint8_t *planes = smem + L.plane0 + pb * p.plane_bytes;
-#pragma unroll
-      for (int k = 0; k < kDwItems / 128; ++k) {
-        const int e = t + 128 * k;
-        const int b = e / p.TB, r = e % p.TB;
-        if (b >= nbox) continue;
-        const uint8_t *src = raw + b * p.TB * 128 + r * 128;
+      if (active) {
+        const uint8_t *src = smem + L.raw0 + s * p.raw_bytes + b * p.TB * 128 + r * 128;
+        uint8_t *planes = smem + L.plane0 + pb * p.plane_bytes;
         uint32_t pl[4][8];
-        float y0[16];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint4 v = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-          const __half2 *h = reinterpret_cast<const __half2 *>(&v);
-          float f[2][4];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float2 lo = __half22float2(h[2 * c]), hi = __half22float2(h[2 * c + 1]);
-            const float a = lo.x + hi.x, bb = lo.y + hi.y;
-            f[c][0] = a + bb;
-            f[c][1] = a - bb;
-            f[c][2] = lo.x - hi.x;
-            f[c][3] = hi.y - lo.y;
-          }
-          y0[2 * q] = f[0][0];
-          y0[2 * q + 1] = f[1][0];
-#pragma unroll
-          for (int pp = 0; pp < 4; ++pp) pl[pp][q] = pack_half2(f[0][pp], f[1][pp]);
+          rdft4_pair(v, pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
         }
-        uint8_t *dst = b < nqd ? planes + b * chunk_plane
-                               : planes + x_off + (b - nqd) * chunk_plane;
-        const int pstride = b < nqd ? 8 * chunk_plane : p.nqc_max * chunk_plane;
+        uint8_t *dst = is_dy ? planes + b * chunk_plane : planes + x_off + (b - nqd) * chunk_plane;
+        const int pstride = is_dy ? 8 * chunk_plane : p.nqc_max * chunk_plane;
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
           uint8_t *row = dst + pp * pstride + r * 32;
@@ -229,9 +216,13 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
                 make_uint4(pl[pp][4 * hh + 0], pl[pp][4 * hh + 1], pl[pp][4 * hh + 2],
                            pl[pp][4 * hh + 3]);
         }
-        if (do_db && b < nqd) {
+        if (do_db) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) db_acc[k][c] += y0[c];
+          for (int q = 0; q < 8; ++q) {
+            const float2 f = __half22float2(as_h2(pl[0][q]));
+            db_acc[2 * q] += f.x;
+            db_acc[2 * q + 1] += f.y;
+          }
         }
       }
       fence_proxy_async_smem();
@@ -244,16 +235,17 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     }
 
     // ------------------------------------------------------------ epilogue
+    // two warps per TMEM lane quadrant, alternating 16-column groups
     if (ok) ok = mbar_wait(acc_full, 0);
     tc_fence_after();
-    const int quad = warp & 3;
+    const int quad = warp & 3, half = (warp - 2) / 4;
     const int d = ti * kDwMT + quad * 32 + lane;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const int ncol = p.CT / 16;
     for (int bin = 0; bin < 4; ++bin) {
       float *dst = p.ws + ((static_cast<int64_t>(split) * 4 + bin) * p.D + d) * p.Cs +
                    static_cast<int64_t>(tj) * p.CT;
-      for (int g = 0; g < ncol; ++g) {
+      for (int g = half; g < ncol; g += 2) {
         uint32_t v[16];
         tmem_ld16(tl + bin * p.CT + g * 16, v);
         tmem_ld_wait();
@@ -269,19 +261,17 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     tc_fence_before();
 
     // db: fixed-order reduction of the per-thread partials through shared memory
-    if (do_db) {
-      named_bar_sync(3, 128);  // raw ring is free: every chunk has been consumed
+    if (tj == 0) {
+      named_bar_sync(3, kDwXfWarps * 32);  // raw ring is free: every chunk has been consumed
       float *sdb = reinterpret_cast<float *>(smem + L.raw0);  // [kDwItems][16]
 #pragma unroll
-      for (int k = 0; k < kDwItems / 128; ++k)
-#pragma unroll
-        for (int c = 0; c < 16; ++c) sdb[(t + 128 * k) * 16 + c] = db_acc[k][c];
-      named_bar_sync(3, 128);
+      for (int c = 0; c < 16; ++c) sdb[t * 16 + c] = db_acc[c];
+      named_bar_sync(3, kDwXfWarps * 32);
       if (t < nqd * 16) {
-        const int b = t / 16, c = t % 16;
+        const int bb = t / 16, c = t % 16;
         float sum = 0.f;
-        for (int r = 0; r < p.TB; ++r) sum += sdb[(b * p.TB + r) * 16 + c];
-        const int dd = ti * kDwMT + b * 16 + c;
+        for (int rr = 0; rr < p.TB; ++rr) sum += sdb[(bb * p.TB + rr) * 16 + c];
+        const int dd = ti * kDwMT + bb * 16 + c;
         if (dd < p.D) p.ws_db[static_cast<int64_t>(split) * p.D + dd] = sum;
       }
     }
@@ -297,38 +287,63 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
 
 // Sum of the split partials in a fixed order, inverse rDFT, fp16 cast:
 //   dW[d][c][u] = (G0 + (-1)^u G2)/4 + Re(G1 i^u)/2,   db[d] = sum of partials.
-__global__ void dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
-                                    __half *__restrict__ dW, __half *__restrict__ db, int splits,
-                                    int C, int D, int Cs) {
+// A block takes 32 consecutive (d, c) outputs (the last blocks take db); its
+// 16 warps each sum every 16th split, then warp 0 adds the 16 partial sums in
+// warp order — the same grouping on every run, so the result is bit-stable.
+constexpr int kRedOut = 32, kRedGroups = 16;
+
+__global__ void __launch_bounds__(kRedOut * kRedGroups)
+dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
+                    __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
+                    int Cs) {
+  __shared__ float part[kRedGroups][4][kRedOut];
   const int64_t plane = static_cast<int64_t>(D) * Cs;
   const int64_t n = static_cast<int64_t>(D) * C;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n + D;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t nblk_w = cdiv(n, kRedOut);
+  const int lo = threadIdx.x % kRedOut, grp = threadIdx.x / kRedOut;
+  if (blockIdx.x < nblk_w) {
+    const int64_t e = blockIdx.x * static_cast<int64_t>(kRedOut) + lo;
+    float g[4] = {0.f, 0.f, 0.f, 0.f};
     if (e < n) {
-      const int64_t d = e / C, c = e % C;
-      const float *src = ws + d * Cs + c;
-      float g0 = 0.f, g2 = 0.f, g1r = 0.f, g1i = 0.f;
-      for (int s = 0; s < splits; ++s) {
+      const float *src = ws + (e / C) * Cs + (e % C);
+      for (int s = grp; s < splits; s += kRedGroups) {
         const float *q = src + static_cast<int64_t>(s) * 4 * plane;
-        g0 += q[0];
-        g2 += q[plane];
-        g1r += q[2 * plane];
-        g1i += q[3 * plane];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) g[k] += q[k * plane];
       }
-      const float ev = 0.25f * (g0 + g2), od = 0.25f * (g0 - g2);
-      __half2 lo = __floats2half2_rn(ev + 0.5f * g1r, od - 0.5f * g1i);
-      __half2 hi = __floats2half2_rn(ev - 0.5f * g1r, od + 0.5f * g1i);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) part[grp][k][lo] = g[k];
+    __syncthreads();
+    if (grp == 0 && e < n) {
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < kRedGroups; ++q)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) t[k] += part[q][k][lo];
+      const float ev = 0.25f * (t[0] + t[1]), od = 0.25f * (t[0] - t[1]);
       uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t *>(&lo);
-      pk.y = *reinterpret_cast<uint32_t *>(&hi);
+      pk.x = pack_half2(ev + 0.5f * t[2], od - 0.5f * t[3]);
+      pk.y = pack_half2(ev - 0.5f * t[2], od + 0.5f * t[3]);
       *reinterpret_cast<uint2 *>(dW + e * kT) = pk;
-    } else if (db != nullptr) {
-      const int d = static_cast<int>(e - n);
-      float sum = 0.f;
-      for (int s = 0; s < splits; ++s) sum += ws_db[static_cast<int64_t>(s) * D + d];
-      db[d] = __float2half_rn(sum);
+    }
+  } else if (db != nullptr) {
+    const int64_t d = (blockIdx.x - nblk_w) * kRedOut + lo;
+    float sdb = 0.f;
+    if (d < D)
+      for (int s = grp; s < splits; s += kRedGroups) sdb += ws_db[static_cast<int64_t>(s) * D + d];
+    part[grp][0][lo] = sdb;
+    __syncthreads();
+    if (grp == 0 && d < D) {
+      float t = 0.f;
+      for (int q = 0; q < kRedGroups; ++q) t += part[q][0][lo];
+      db[d] = __float2half_rn(t);
     }
   }
+}
+
+// Blocks for dw_tc_reduce_kernel: the dW outputs, then the db outputs.
+__host__ __device__ inline int64_t dw_reduce_blocks(int C, int D) {
+  return cdiv(static_cast<int64_t>(D) * C, kRedOut) + cdiv(D, kRedOut);
 }
 
 }  // namespace feql

@@ -7,19 +7,26 @@
 // contractions, bin 1 is one complex contraction; the Fourier tiles live only
 // in shared memory / tensor memory (no intermediate global writes).
 //
-// One persistent CTA per SM, warp-specialised (320 threads):
-//   warp 0      TMA producer: input chunk [128 tokens x 16 channels x 4] and
-//               the matching weight chunk into a ring of `stages` slots
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5  transform: 4-point rDFT of the chunk, in place, into four
-//               K-major fp16 operand planes (X0, X2, Re X1, Im X1)
-//   warps 6..9  epilogue: tcgen05.ld of the four fp32 accumulators, inverse
-//               rDFT + bias, fp16 pack, swizzled smem staging, TMA store
+// One persistent CTA per SM, warp-specialised (576 threads):
+//   warp 0       TMA producer: input chunks [128 tokens x 16 channels x 4] into
+//                a ring of `stages` slots; the weight chunks either ride along
+//                in each slot or, when the CTA's whole weight slice fits, are
+//                loaded once into a resident buffer
+//   warp 1       TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..9   transform, two 4-warp teams taking alternate chunks: 4-point
+//                rDFT of the chunk (packed fp16 pairs), in place, into four
+//                K-major operand planes (X0, X2, Re X1, -Im X1)
+//   warps 10..17 epilogue, two 4-warp teams: tcgen05.ld of the four fp32
+//                accumulators, inverse rDFT + bias, fp16 pack, swizzled smem
+//                staging; each warp owns 32 token rows and issues its own TMA
+//                stores
 // Per chunk the MMA warp issues four M=128 x K=16 MMAs:
 //   acc[0, BD)    += X0  * What0^T                (N = BD)
 //   acc[BD, 2BD)  += X2  * What2^T                (N = BD)
-//   acc[2BD, 4BD) += ReX1 * (Re1 ; Im1)^T + ImX1 * (-Im1 ; Re1)^T   (N = 2 BD)
-// so columns [2BD, 3BD) hold Re Y1 and [3BD, 4BD) hold Im Y1.
+//   acc[2BD, 4BD) += ReX1 * (Re1 ; Im1)^T + (-ImX1) * (Im1 ; -Re1)^T   (N = 2 BD)
+// so columns [2BD, 3BD) hold Re Y1 and [3BD, 4BD) hold Im Y1.  When 4*BD <= 256
+// the accumulators are double-buffered in TMEM so the epilogue of one tile
+// overlaps the MMAs of the next.
 // Every wait is bounded (mbar_wait); a timed-out thread stops issuing work but
 // keeps the loop structure so named barriers stay matched.
 #pragma once
@@ -27,15 +34,18 @@
 #include <cuda_fp16.h>
 
 #include "plan.cuh"
+#include "rdft4.cuh"
 #include "sm100.cuh"
 
 namespace feql {
 
-constexpr int kTcThreads = 320;
+constexpr int kTeams = 2;                         // transform teams and epilogue teams
+constexpr int kTcThreads = 64 + 2 * kTeams * 128; // TMA + MMA warps, 4-warp teams
 constexpr int kXChunkBytes = kBM * kCK * kT * 2;  // 16 KB: 128 rows x 128 B
 constexpr int kPlaneBytes = kBM * kCK * 2;        // 4 KB: 128 rows x 32 B
-constexpr int kOutBoxBytes = kBM * 64 * 2;        // 16 KB: 128 rows x (16 ch x 4) fp16
-constexpr int kNumOut = 2;
+constexpr int kOutRows = 32;                      // rows per epilogue TMA store (one warp)
+constexpr int kOutBoxBytes = kOutRows * 64 * 2;   // 4 KB: 32 rows x (16 ch x 4) fp16
+constexpr int kNumOut = 2;                        // staging buffers per epilogue warp
 constexpr int kTmemCols = 512;
 
 struct TcFwdParams {
@@ -43,30 +53,54 @@ struct TcFwdParams {
   const __half *bias;   // [Do] or nullptr
   int64_t N;
   int Ci, Do, BD, nD, nK, chunk_bytes;
-  int n_units;          // ceil(N/128) * nD
+  int nM;               // token tiles: ceil(N / 128)
+  int n_units;          // nM * nD
   int nacc, acc_stride; // accumulator buffers in TMEM and their column stride
+  int resident;         // 1: the CTA's weight slice is loaded once (fixed D tile per CTA)
+  int wres_bytes;       // resident weight buffer: nK * chunk_bytes (1 KB aligned)
   int stages;
-  int stage_bytes;      // 16 KB input chunk + weight chunk (1 KB aligned)
+  int stage_bytes;      // 16 KB input chunk (+ weight chunk unless resident), 1 KB aligned
   int bias_floats;      // nD * BD
 };
 
 struct TcSmem {
   // offsets (bytes) from the 1024-aligned dynamic smem base
-  int stage0, out0, bias, bars, total;
+  int wres, stage0, out0, bias, bars, total;
 };
 
 __host__ __device__ inline TcSmem tc_fwd_smem(const TcFwdParams &p) {
   TcSmem s;
-  s.stage0 = 0;
-  s.out0 = p.stages * p.stage_bytes;
-  s.bias = s.out0 + kNumOut * kOutBoxBytes;
+  s.wres = 0;
+  s.stage0 = p.resident ? p.wres_bytes : 0;
+  s.out0 = s.stage0 + p.stages * p.stage_bytes;
+  s.bias = s.out0 + 4 * kTeams * kNumOut * kOutBoxBytes;
   s.bars = s.bias + static_cast<int>(align_up(p.bias_floats * 4, 16));
-  // full, tready, empty per stage; acc_full, acc_empty per acc buffer; final; tmem slot
-  s.total = s.bars + (3 * p.stages + 2 * 2 + 1) * 8 + 16;
+  // full, tready, empty per stage; acc_full, acc_empty per acc buffer; final; wfull; tmem slot
+  s.total = s.bars + (3 * p.stages + 2 * 2 + 2) * 8 + 16;
   return s;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+// k-th work unit of this CTA: token tile m and output-channel tile j.  With
+// resident weights every CTA keeps one j (neighbouring CTAs share a token tile,
+// so its second read comes from L2); otherwise units are dealt round-robin.
+__device__ __forceinline__ bool tc_unit(const TcFwdParams &p, int k, int &m, int &j) {
+  if (p.resident) {
+    const int g = gridDim.x / p.nD;
+    if (static_cast<int>(blockIdx.x) >= g * p.nD) return false;
+    j = blockIdx.x % p.nD;
+    m = blockIdx.x / p.nD + k * g;
+    return m < p.nM;
+  }
+  const int u = blockIdx.x + k * gridDim.x;
+  if (u >= p.n_units) return false;
+  m = u / p.nD;
+  j = u % p.nD;
+  return true;
+}
+
+// 18 warps over the 4 SM sub-partitions put 5 warps on one 16K-register
+// slice: 5 x 32 x 96 = 15,360 registers fits, 104 would not.
+__global__ void __maxnreg__(96)
 tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
                        const __grid_constant__ CUtensorMap tm_out, const TcFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -81,7 +115,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
   uint64_t *acc_full = bars + 3 * p.stages;
   uint64_t *acc_empty = acc_full + 2;
   uint64_t *final_bar = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(final_bar + 1);
+  uint64_t *wfull = final_bar + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wfull + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
@@ -93,9 +128,10 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], p.nacc == 1 ? 4 * kTeams : 4);  // single buffer: all teams release
     }
     mbar_init(final_bar, 1);
+    mbar_init(wfull, 1);
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < p.bias_floats; i += blockDim.x)
@@ -108,8 +144,6 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  const int first = blockIdx.x, step = gridDim.x;
   bool ok = true;
 
   if (warp == 0) {
@@ -117,27 +151,32 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
       tma_prefetch_desc(&tm_out);
+      int m, j;
+      if (p.resident && tc_unit(p, 0, m, j)) {
+        mbar_arrive_expect_tx(wfull, p.nK * p.chunk_bytes);
+        bulk_load(smem + L.wres, p.wt + static_cast<int64_t>(j) * p.nK * p.chunk_bytes,
+                  p.nK * p.chunk_bytes, wfull);
+      }
       int s = 0;
       uint32_t ph = 0;
-      for (int u = first; u < p.n_units; u += step) {
-        const int m = u / p.nD, j = u % p.nD;
+      for (int k = 0; tc_unit(p, k, m, j); ++k) {
         for (int kc = 0; kc < p.nK; ++kc) {
           if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
           if (ok) {
             uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
-            mbar_arrive_expect_tx(&full[s], kXChunkBytes + p.chunk_bytes);
-            tma_load_2d(st, &tm_in, kc * (kCK * kT), m * kBM, &full[s]);
-            bulk_load(st + kXChunkBytes,
-                      p.wt + (static_cast<int64_t>(j) * p.nK + kc) * p.chunk_bytes,
-                      p.chunk_bytes, &full[s]);
+            if (p.resident) {
+              mbar_arrive_expect_tx(&full[s], kXChunkBytes);
+              tma_load_2d(st, &tm_in, kc * (kCK * kT), m * kBM, &full[s]);
+            } else {
+              mbar_arrive_expect_tx(&full[s], kXChunkBytes + p.chunk_bytes);
+              tma_load_2d(st, &tm_in, kc * (kCK * kT), m * kBM, &full[s]);
+              bulk_load(st + kXChunkBytes,
+                        p.wt + (static_cast<int64_t>(j) * p.nK + kc) * p.chunk_bytes,
+                        p.chunk_bytes, &full[s]);
+            }
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }
         }
-      }
-      // drain: the last loads must land before the CTA may exit
-      for (int i = 0; i < p.stages; ++i) {
-        if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
-        if (++s == p.stages) { s = 0; ph ^= 1; }
       }
     }
   } else if (warp == 1) {
@@ -146,10 +185,11 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       const uint32_t id_bd = instr_desc(kBM, p.BD, 0, 0);
       const uint32_t id_2bd = instr_desc(kBM, 2 * p.BD, 0, 0);
       const uint32_t wrow = 32;  // bytes per weight row (16 fp16)
+      int m, j;
+      if (p.resident && tc_unit(p, 0, m, j)) ok = mbar_wait(wfull, 0);
       int s = 0;
       uint32_t ph = 0;
-      int it = 0;
-      for (int u = first; u < p.n_units; u += step, ++it) {
+      for (int it = 0; tc_unit(p, it, m, j); ++it) {
         const int a = it % p.nacc;
         const uint32_t aph = (it / p.nacc) & 1;
         if (ok) ok = mbar_wait(&acc_empty[a], aph ^ 1);
@@ -161,7 +201,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
           tc_fence_after();
           if (ok) {
             const uint32_t xs = smem_u32(smem + L.stage0 + s * p.stage_bytes);
-            const uint32_t ws = xs + kXChunkBytes;
+            const uint32_t ws = p.resident ? smem_u32(smem + L.wres) + kc * p.chunk_bytes
+                                           : xs + kXChunkBytes;
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
             mma_f16_ss(acc, smem_desc(xs + 0 * kPlaneBytes, 16, 256, kSw32),
                        smem_desc(ws, 16, 256, kSw32), id_bd, acc_in);
@@ -177,17 +218,24 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
         }
         if (ok) mma_commit(&acc_full[a]);
       }
-      // all MMAs must be complete before TMEM is released
+      // all MMAs (and hence all loads they consumed) complete before exit
       mma_commit(final_bar);
       mbar_wait(final_bar, 0);
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + 4 * kTeams) {
     // ---------------------------------------------------------- transform
-    const int r = threadIdx.x - 64;  // row of the chunk (token within the tile)
-    int s = 0;
+    // kTeams teams of 4 warps take alternate chunks of the ring.
+    const int team = (warp - 2) / 4;
+    const int r = (threadIdx.x - 64) % 128;  // row of the chunk (token within the tile)
+    int s = 0, c = 0;
     uint32_t ph = 0;
-    for (int u = first; u < p.n_units; u += step) {
-      for (int kc = 0; kc < p.nK; ++kc) {
+    int m, j;
+    for (int k = 0; tc_unit(p, k, m, j); ++k) {
+      for (int kc = 0; kc < p.nK; ++kc, ++c) {
+        if (c % kTeams != team) {
+          if (++s == p.stages) { s = 0; ph ^= 1; }
+          continue;
+        }
         if (ok) ok = mbar_wait(&full[s], ph);
         uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
         // row r: 8 x 16 B, logical chunk q = channels 2q, 2q+1 (x 4 group elements)
@@ -195,25 +243,10 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           raw[q] = *reinterpret_cast<const uint4 *>(st + r * 128 + ((q ^ (r & 7)) << 4));
-        uint32_t pl[4][8];  // [plane][channel pair] packed half2
+        uint32_t pl[4][8];  // [plane][channel pair] packed half2: V0, V2, Re V1, -Im V1
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const __half2 *h = reinterpret_cast<const __half2 *>(&raw[q]);
-          float f[2][4];
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const float2 lo = __half22float2(h[2 * c]), hi = __half22float2(h[2 * c + 1]);
-            const float v0 = lo.x, v1 = lo.y, v2 = hi.x, v3 = hi.y;
-            const float a = v0 + v2, b = v1 + v3;
-            f[c][0] = a + b;
-            f[c][1] = a - b;
-            f[c][2] = v0 - v2;
-            f[c][3] = v3 - v1;
-          }
-#pragma unroll
-          for (int pp = 0; pp < 4; ++pp) pl[pp][q] = pack_half2(f[0][pp], f[1][pp]);
-        }
-        named_bar_sync(2, 128);  // every row read before the planes overwrite it
+        for (int q = 0; q < 8; ++q) rdft4_pair(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+        named_bar_sync(2 + team, 128);  // every row read before the planes overwrite it
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
           uint8_t *plane = st + pp * kPlaneBytes + r * 32;
@@ -231,59 +264,77 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    // kTeams teams of 4 warps.  With double-buffered accumulators each team
+    // owns one TMEM buffer (alternate tiles); with a single buffer the teams
+    // split each tile's 16-column groups.  Each warp owns one TMEM lane
+    // quadrant (32 token rows) and stores its rows with its own TMA stores.
+    const int ew = warp - 2 - 4 * kTeams;   // epilogue warp index
+    const int eteam = ew / 4;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;       // token within the tile
-    const int et = threadIdx.x - 192;       // 0..127 among epilogue threads
-    int it = 0, oi = 0;
-    for (int u = first; u < p.n_units; u += step, ++it) {
-      const int m = u / p.nD, j = u % p.nD;
+    uint8_t *obase = smem + L.out0 + ew * kNumOut * kOutBoxBytes;
+    const int groups = p.BD / 16;
+    const bool split = p.nacc == 1;
+    const int g0 = split ? eteam : 0, gstep = split ? kTeams : 1;
+    int last_g = -1;
+    for (int g = g0; g < groups; g += gstep) last_g = g;
+    int oi = 0, m, j;
+    for (int it = 0; tc_unit(p, it, m, j); ++it) {
+      if (!split && it % kTeams != eteam) continue;
       const int a = it % p.nacc;
       const uint32_t aph = (it / p.nacc) & 1;
       if (ok) ok = mbar_wait(&acc_full[a], aph);
       tc_fence_after();
+      if (last_g < 0) {  // this team reads nothing of the tile
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
+      }
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
-      const int groups = p.BD / 16;
-      for (int g = 0; g < groups; ++g) {
-        uint32_t y0[16], y2[16], y1r[16], y1i[16];
-        tmem_ld16(tl + g * 16, y0);
-        tmem_ld16(tl + p.BD + g * 16, y2);
-        tmem_ld16(tl + 2 * p.BD + g * 16, y1r);
-        tmem_ld16(tl + 3 * p.BD + g * 16, y1i);
-        tmem_ld_wait();
-        if (g == groups - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
-        }
+      for (int g = g0; g < groups; g += gstep) {
         const int d0 = j * p.BD + g * 16;
         uint32_t packed[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-          const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-          const float bv = sbias[d0 + i];
-          const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
-          packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-          packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+        for (int h = 0; h < 2; ++h) {  // 8 columns at a time keeps registers low
+          uint32_t y0[8], y2[8], y1r[8], y1i[8];
+          const uint32_t col = tl + g * 16 + h * 8;
+          tmem_ld8(col, y0);
+          tmem_ld8(col + p.BD, y2);
+          tmem_ld8(col + 2 * p.BD, y1r);
+          tmem_ld8(col + 3 * p.BD, y1i);
+          tmem_ld_wait();
+          if (h == 1 && g == last_g) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
+            const float bv = sbias[d0 + h * 8 + i];
+            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
+            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+          }
         }
-        if (d0 >= p.Do) continue;  // uniform across the epilogue warps
-        uint8_t *ob = smem + L.out0 + (oi % kNumOut) * kOutBoxBytes;
-        if (et == 0) bulk_wait_read<kNumOut - 1>();
-        named_bar_sync(1, 128);
+        if (d0 >= p.Do) continue;  // whole group is padding
+        uint8_t *ob = obase + (oi % kNumOut) * kOutBoxBytes;
+        if (lane == 0) bulk_wait_read<kNumOut - 1>();  // this buffer's last store has read it
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4 *>(ob + row * 128 + ((q ^ (row & 7)) << 4)) =
+          *reinterpret_cast<uint4 *>(ob + lane * 128 + ((q ^ (lane & 7)) << 4)) =
               make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (et == 0) {
-          tma_store_2d(&tm_out, d0 * kT, m * kBM, ob);
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_out, d0 * kT, m * kBM + quad * 32, ob);
           bulk_commit();
         }
         ++oi;
       }
     }
-    if (et == 0) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();

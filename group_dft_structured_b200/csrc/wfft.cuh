@@ -65,8 +65,8 @@ __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict
       weight_bins(W, C, dir, o, i, b0, b2, b1r, b1i);
       if (sub == 0) v = b0;
       else if (sub == 1) v = b2;
-      else if (sub == 2) v = hi ? b1i : b1r;    // rows (Re1 ; Im1): multiplies Re X1
-      else v = hi ? b1r : -b1i;                 // rows (-Im1 ; Re1): multiplies Im X1
+      else if (sub == 2) v = hi ? b1i : b1r;    // rows (Re1 ; Im1): multiply Re X1
+      else v = hi ? -b1r : b1i;                 // rows (Im1 ; -Re1): multiply -Im X1
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);

@@ -63,9 +63,9 @@ def test_invalid_arguments_rejected_before_cuda(lib):
 
 
 def _tc_plan(Ci, Do):
-    nD = -(-Do // 128)
-    BD = -(-(-(-Do // nD)) // 16) * 16
     nK = -(-Ci // 16)
+    nD = -(-Do // (64 if nK <= 4 else 128))
+    BD = -(-(-(-Do // nD)) // 16) * 16
     return nD, BD, nK, nD * nK * 6 * BD * 16 * 2
 
 
@@ -82,11 +82,12 @@ def test_weight_buffer_sizes(lib, C, D):
 
 
 def test_tile_plans_cover_the_workloads():
-    # output-channel tiles of at most 128 (complex-bin MMA N = 2*BD <= 256)
-    assert _tc_plan(48, 192)[:2] == (2, 96)
+    # output-channel tiles of at most 128 (complex-bin MMA N = 2*BD <= 256);
+    # at most 64 (double-buffered TMEM) when the contraction is <= 64 channels
+    assert _tc_plan(48, 192)[:2] == (3, 64)
     assert _tc_plan(192, 192)[:2] == (2, 96)
     assert _tc_plan(256, 256)[:2] == (2, 128)
-    assert _tc_plan(24, 96)[:2] == (1, 96)
+    assert _tc_plan(24, 96)[:2] == (2, 48)
     assert _tc_plan(96, 24)[:2] == (1, 32)
     assert _tc_plan(16, 16)[:2] == (1, 16)
 
