@@ -67,6 +67,20 @@ def workload_bytes(w, elt):
     }
 
 
+def kernel_source_hash():
+    """Hash of the CUDA sources; DRAM counters in profiles/traffic.json are only
+    reported while it matches the hash they were taken with."""
+    import hashlib
+    d = os.path.join(ROOT, "group_dft_structured_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -359,7 +373,9 @@ def main():
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
-            traffic = json.load(f).get(w.name, {}).get(dom)
+            tj = json.load(f)
+        if tj.get("source_hash") == kernel_source_hash():
+            traffic = tj.get(w.name, {}).get(dom)
     nkern = sum(launches_per_step[p] for p in passes)
     step_ms = ms / args.steps
     line = {
