@@ -54,6 +54,29 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def rank_seed_id(wid: int, rank: int) -> int:
+    """Seed block of a rank's own tokens (weak scaling: every rank has a full batch)."""
+    return wid + 1000 * rank
+
+
+def dp_allreduce_grads(dW, db):
+    """Data-parallel weight gradient: every rank holds dW/db of its own tokens;
+    the layer's gradient is their sum (the path's one exchange step)."""
+    import torch.distributed as dist
+    dist.all_reduce(dW)
+    if db is not None:
+        dist.all_reduce(db)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The slowest rank's time (all ranks take part)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_bytes(w, elt):
     """Algorithmic HBM bytes per launch of each pass (inputs read once, outputs
     written once; Fourier weights counted as their 4*D*C values)."""
@@ -229,7 +252,7 @@ def main():
     mode = F.FEQL_FP16 if w.dtype == "fp16" else F.FEQL_FP32
     N, C, D = w.N, w.C, w.D
     elt = 2 if w.dtype == "fp16" else 4
-    inp = make_inputs(w.wid + 1000 * rank, N, C, D, w.dtype)
+    inp = make_inputs(rank_seed_id(w.wid, rank), N, C, D, w.dtype)
     dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
     x, W, b, dy = dev["x"], dev["W"], dev["b"], dev["dy"]
     What = torch.empty(F.feql_weight_fft_bytes(C, D, mode), dtype=torch.uint8, device="cuda")
@@ -265,8 +288,7 @@ def main():
             if ev is not None:
                 ev[i].record(stream)
         if world > 1:
-            dist.all_reduce(dW)
-            dist.all_reduce(db)
+            dp_allreduce_grads(dW, db)
 
     def barrier():
         if world > 1:
@@ -295,9 +317,7 @@ def main():
     clk = clocks.stop() if (rank == 0 or world == 1) else None
     ms = t_start.elapsed_time(t_end)
     if world > 1:
-        tt = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, "cuda")
     per_pass = {p: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)]
                 for i, p in enumerate(passes)}
     if F.feql_device_status(s) != F.FEQL_OK:
@@ -339,9 +359,7 @@ def main():
         barrier()
         e_ms = a.elapsed_time(z)
         if world > 1:
-            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+            e_ms = max_over_ranks(e_ms, "cuda")
         e2e = {"value": N * world * args.e2e_steps / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps}
