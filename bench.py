@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--separate-backward", action="store_true",
+                    help="run dX and dW as two passes instead of the fused backward")
     return ap.parse_args()
 
 
@@ -87,6 +89,7 @@ def workload_bytes(w, elt):
         "fwd": x + what + b + y,
         "dx": y + what + x,
         "dw": x + y + 4 * D * C * elt + b,
+        "bwd": x + y + what + x + 4 * D * C * elt + b,  # x, dy, What in; dx, dW, db out
     }
 
 
@@ -263,30 +266,29 @@ def main():
     ws = L.dw_workspace(N, C, D, mode, "cuda")
     stream = torch.cuda.current_stream()
     s = stream.cuda_stream
-    passes = ["wfft"] + [p for p in ("fwd", "dx", "dw") if p in w.passes]
-    launches_per_step = {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2}
+    # One step = every row of the path: weight rDFT, forward, and the backward
+    # (dX and dW/db, fused into one pass over dy unless --separate-backward).
+    calls = {
+        "wfft": lambda: F.feql_weight_fft(W, What, C, D, mode, s),
+        "fwd": lambda: F.feql_forward(x, What, b, y, N, C, D, mode, s),
+        "dx": lambda: F.feql_backward_dx(dy, What, dx, N, C, D, mode, s),
+        "dw": lambda: F.feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
+        "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode, s),
+    }
+    passes = ["wfft"] + (["fwd"] if "fwd" in w.passes else [])
+    if "dx" in w.passes and "dw" in w.passes and not args.separate_backward:
+        passes.append("bwd")
+    else:
+        passes += [p for p in ("dx", "dw") if p in w.passes]
+    launches_per_step = {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2, "bwd": 2}
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        F.feql_weight_fft(W, What, C, D, mode, s)
-        if ev is not None:
-            ev[1].record(stream)
-        i = 2
-        if "fwd" in passes:
-            F.feql_forward(x, What, b, y, N, C, D, mode, s)
+        for i, p in enumerate(passes):
+            calls[p]()
             if ev is not None:
-                ev[i].record(stream)
-            i += 1
-        if "dx" in passes:
-            F.feql_backward_dx(dy, What, dx, N, C, D, mode, s)
-            if ev is not None:
-                ev[i].record(stream)
-            i += 1
-        if "dw" in passes:
-            F.feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s)
-            if ev is not None:
-                ev[i].record(stream)
+                ev[i + 1].record(stream)
         if world > 1:
             dp_allreduce_grads(dW, db)
 
@@ -331,11 +333,13 @@ def main():
                 "dx": torch.empty_like(dx, device="cpu").pin_memory(),
                 "dW": torch.empty_like(dW, device="cpu").pin_memory(),
                 "db": torch.empty_like(db, device="cpu").pin_memory()}
+        has_bwd = any(p in passes for p in ("dx", "dw", "bwd"))
         h2d = sum(hin[k].numel() * hin[k].element_size() for k in ("x", "W", "b")) + \
-            (hin["dy"].numel() * hin["dy"].element_size() if ("dx" in passes or "dw" in passes) else 0)
+            (hin["dy"].numel() * hin["dy"].element_size() if has_bwd else 0)
         outs = [k for k in ("y", "dx", "dW", "db")
-                if (k == "y" and "fwd" in passes) or (k == "dx" and "dx" in passes)
-                or (k in ("dW", "db") and "dw" in passes)]
+                if (k == "y" and "fwd" in passes)
+                or (k == "dx" and ("dx" in passes or "bwd" in passes))
+                or (k in ("dW", "db") and ("dw" in passes or "bwd" in passes))]
         d2h = sum(hout[k].numel() * hout[k].element_size() for k in outs)
         src = {"y": y, "dx": dx, "dW": dW, "db": db}
 
@@ -343,7 +347,7 @@ def main():
             x.copy_(hin["x"], non_blocking=True)
             W.copy_(hin["W"], non_blocking=True)
             b.copy_(hin["b"], non_blocking=True)
-            if "dx" in passes or "dw" in passes:
+            if has_bwd:
                 dy.copy_(hin["dy"], non_blocking=True)
             step()
             for k in outs:
@@ -376,15 +380,17 @@ def main():
     nbytes = workload_bytes(w, elt)
     macs = 6 * N * C * D
     mean_ms = {p: float(np.mean(v)) for p, v in per_pass.items()}
+    gemm_passes = {"wfft": 0, "fwd": 1, "dx": 1, "dw": 1, "bwd": 2}  # layer contractions per pass
     pass_report = {}
     for p in passes:
         gbs = nbytes[p] / (mean_ms[p] * 1e-3) / 1e9
         pass_report[p] = {"ms": round(mean_ms[p], 5), "GB_s": round(gbs, 1),
                           "frac_hbm": round(gbs / peak, 4), "algorithmic_bytes": nbytes[p]}
         if p != "wfft":
-            pass_report[p]["alg_TFLOP_s"] = round(2 * macs / (mean_ms[p] * 1e-3) / 1e12, 2)
+            g = gemm_passes[p]
+            pass_report[p]["alg_TFLOP_s"] = round(2 * macs * g / (mean_ms[p] * 1e-3) / 1e12, 2)
             pass_report[p]["dense_equiv_TFLOP_s"] = round(
-                2 * 16 * N * C * D / (mean_ms[p] * 1e-3) / 1e12, 2)
+                2 * 16 * N * C * D * g / (mean_ms[p] * 1e-3) / 1e12, 2)
     dom = max((p for p in passes if p != "wfft"), key=lambda p: mean_ms[p])
     achieved = nbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
     traffic = None
@@ -405,7 +411,7 @@ def main():
                    "passes": passes, "accumulate": "f32", "l2": "inputs larger than L2, no flush",
                    "global_tokens": N * world,
                    "parallelism": f"dp{world}" if world > 1 else "single"},
-        "effective_TFLOP_s": round(2 * 16 * N * C * D * len([p for p in passes if p != "wfft"])
+        "effective_TFLOP_s": round(2 * 16 * N * C * D * sum(gemm_passes[p] for p in passes)
                                    * world / (step_ms * 1e-3) / 1e12, 2),
         "roofline_pct_step": round(100 * sum(nbytes[p] for p in passes) / (step_ms * 1e-3) / 1e9
                                    / peak, 2),

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "feql_backward_dx": (_I, [_VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
     "feql_backward_dw_workspace_bytes": (_SZ, [_I64, _I, _I, _I]),
     "feql_backward_dw": (_I, [_VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
+    "feql_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
     "feql_backward_dw_noalloc": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
     "feql_device_status": (_I, [_VP]),
     "feql_status_string": (ctypes.c_char_p, [_I]),
@@ -129,6 +130,13 @@ def feql_backward_dw(x, dy, dW, db, ws, ws_bytes: int, N: int, C: int, D: int, d
                      stream=None) -> None:
     _check(load().feql_backward_dw(_ptr(x), _ptr(dy), _ptr(dW), _ptr(db), _ptr(ws), ws_bytes,
                                    N, C, D, dtype, _stream(stream)), "feql_backward_dw")
+
+
+def feql_backward(x, dy, What, dx, dW, db, ws, ws_bytes: int, N: int, C: int, D: int,
+                  dtype: int, stream=None) -> None:
+    _check(load().feql_backward(_ptr(x), _ptr(dy), _ptr(What), _ptr(dx), _ptr(dW), _ptr(db),
+                                _ptr(ws), ws_bytes, N, C, D, dtype, _stream(stream)),
+           "feql_backward")
 
 
 def feql_backward_dw_noalloc(x, dy, dW, db, N: int, C: int, D: int, dtype: int,

@@ -14,6 +14,7 @@
 #include "plan.cuh"
 #include "simt.cuh"
 #include "sm100.cuh"
+#include "tc_bwd.cuh"
 #include "tc_dw.cuh"
 #include "tc_fwd.cuh"
 #include "wfft.cuh"
@@ -283,6 +284,63 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
   return launch_status();
 }
 
+// Fused backward plan; false when the shape is outside the fused kernel's
+// range (then feql_backward runs the dX and dW kernels one after the other).
+bool make_tc_bwd_plan(int64_t N, int C, int D, const WhatLayout &L, const DeviceInfo &dev,
+                      TcBwdParams &p) {
+  if (N <= 0 || L.dx.nD != 1) return false;
+  p.N = N;
+  p.C = C;
+  p.D = D;
+  p.Cs = static_cast<int>(align_up(C, 16));
+  p.nqd = static_cast<int>(cdiv(D, 16));
+  p.nqc = static_cast<int>(cdiv(C, 16));
+  if (p.nqd + p.nqc > kBwMaxItems / kBwTB) return false;
+  p.slots = p.nqd + p.nqc > 8 ? p.nqd + p.nqc : 8;
+  p.CT = 16 * p.nqc;
+  p.BD = L.dx.BD;
+  p.chunk_bytes = L.dx.chunk_bytes;
+  if (4 * p.CT + 4 * p.BD > 512) return false;
+  p.ndx = (4 * p.CT + 8 * p.BD <= 512) ? 2 : 1;
+  p.wres_bytes = static_cast<int>(align_up(static_cast<int64_t>(p.nqd) * p.chunk_bytes, 1024));
+  int64_t s = dev.sms;
+  if (s > cdiv(N, kBwTB)) s = cdiv(N, kBwTB);
+  p.split_len = align_up(cdiv(N, s), kBwTB);
+  p.splits = static_cast<int>(cdiv(N, p.split_len));
+  const int budget = dev.smem_optin - 1024;
+  p.stages = 4;
+  while (p.stages > 2 && tc_bwd_smem(p).total > budget) --p.stages;
+  if (tc_bwd_smem(p).total > budget) return false;
+  p.ws = nullptr;
+  p.ws_db = nullptr;
+  return true;
+}
+
+int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *wt, __half *dx,
+                  __half *dW, __half *db, float *ws, const DeviceInfo &dev, cudaStream_t stream) {
+  if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
+  p.wt = wt;
+  p.ws = ws;
+  p.ws_db = ws + static_cast<int64_t>(p.splits) * 4 * p.D * p.Cs;
+  const int smem = tc_bwd_smem(p).total + 1024;
+  CUtensorMap tm_dy, tm_x, tm_dx;
+  int st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, kBwTB);
+  if (st != FEQL_OK) return st;
+  st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB);
+  if (st != FEQL_OK) return st;
+  st = make_tmap_f16(&tm_dx, dx, p.N, static_cast<int64_t>(p.C) * kT, kBwOutRows);
+  if (st != FEQL_OK) return st;
+  if (cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FEQL_ERR_CUDA;
+  tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, tm_dx, p);
+  const int64_t rblocks = dw_reduce_blocks(p.C, p.D);
+  if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dw_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), kRedOut * kRedGroups, 0, stream>>>(
+      p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs);
+  return launch_status();
+}
+
 }  // namespace
 
 // =============================================================================
@@ -361,6 +419,40 @@ size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
   if (device_info(&dev) != FEQL_OK) return 0;
   if (is_tc(resolve(dtype))) return static_cast<size_t>(tc_dw_ws_floats(make_tc_dw_plan(N, C, D, dev.sms))) * 4;
   return static_cast<size_t>(make_dw_plan(N, C, D, dev.sms).ws_floats) * 4;
+}
+
+int feql_backward(const void *x, const void *dy, const void *What, void *dx, void *dW, void *db,
+                  void *ws, size_t ws_bytes, int64_t N, int C, int D, int dtype,
+                  feql_stream stream) {
+  if (!valid_dtype(dtype) || dW == nullptr || ws == nullptr) return FEQL_ERR_INVALID_ARG;
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || dy == nullptr || What == nullptr || dx == nullptr))
+    return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(What) || !aligned16(dx) || !aligned16(dW) ||
+      !aligned16(ws) || (db != nullptr && !aligned16(db)))
+    return FEQL_ERR_INVALID_ARG;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  if (is_tc(dt) && N > 0) {
+    const WhatLayout L = make_what_layout(C, D, true);
+    TcBwdParams p;
+    if (make_tc_bwd_plan(N, C, D, L, dev, p)) {
+      // the regular dW workspace always covers the fused plan (no more splits)
+      if (ws_bytes < static_cast<size_t>(p.splits) * (4ull * p.D * p.Cs + p.D) * 4)
+        return FEQL_ERR_INVALID_ARG;
+      return launch_tc_bwd(p, x, dy, static_cast<const uint8_t *>(What) + L.off_dx,
+                           static_cast<__half *>(dx), static_cast<__half *>(dW),
+                           static_cast<__half *>(db), static_cast<float *>(ws), dev,
+                           reinterpret_cast<cudaStream_t>(stream));
+    }
+  }
+  st = feql_backward_dx(dy, What, dx, N, C, D, dtype, stream);
+  if (st != FEQL_OK) return st;
+  return feql_backward_dw(x, dy, dW, db, ws, ws_bytes, N, C, D, dtype, stream);
 }
 
 int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws, size_t ws_bytes,

@@ -247,6 +247,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// The start address is the only field that changes between the MMAs of one
+// operand stream, so the issue loops build a descriptor once with address 0
+// and add the 16-byte-unit address (shared addresses are < 256 KB, so it
+// never carries out of the 14-bit field).
+__device__ __forceinline__ uint64_t desc_at(uint64_t base, uint32_t saddr) {
+  return base + static_cast<uint64_t>(saddr >> 4);
+}
+
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.
 // a_fmt/b_fmt: 0 = f16, 1 = bf16, 2 = tf32.  Both operands K-major unless
 // a_mn / b_mn select MN-major.

@@ -1,0 +1,390 @@
+// tc_bwd.cuh — fused backward: dX and the dW/db partial sums from one pass
+// over dy (sm_100a tensor cores, fp16 data).
+//
+// Both gradients need the rDFT of the same dy tile (Flash EQ-Linear,
+// technical summary "Implementazione": fused dataflow), so one kernel reads
+// x and dy once and produces
+//   dX[n,:] = irDFT_4( per-bin dY_k[n,:] . conj(What_k) )          (forward of conj(What)^T)
+//   G_k[d,c] += sum_{n in split} dY_k[n,d] conj(X_k[n,c])          (split-K partials of dW)
+//   db[d]    += sum_{n in split} dY_0[n,d]
+// and dw_tc_reduce_kernel finishes dW/db as for feql_backward_dw.
+//
+// One CTA per token split (a multiple of 64 tokens); shapes with C <= 64 and
+// D <= 128 (one dW tile, one dX output tile).  Per stage of 64 tokens:
+//   warp 0      TMA: every 16-channel box of dy and x for the 64 tokens
+//   warps 2..9  4-point rDFT of every (token, channel) fibre, in place: each
+//               8 KB box becomes four 2 KB planes (V0, V2, Re V1, -Im V1),
+//               rows = tokens, 32-byte swizzle; db sums in registers
+//   warp 1      TMEM allocator + MMA issuer:
+//                 dW: per 16 tokens six M=128 (d) x N=CT (c) MMAs, both
+//                     operands MN-major (the planes read column-wise)
+//                 dX: per 16-channel d chunk four M=64 (tokens) MMAs against
+//                     the resident conj(What)^T tiles, K-major (the same planes
+//                     read row-wise) into a double-buffered accumulator
+//   warps 10..13 dX epilogue: the M=64 accumulator sits in TMEM lanes
+//               (m mod 16) + 32 * (m / 16), so warp q's lanes 0..15 hold
+//               tokens 16q..16q+15; inverse rDFT, fp16, 16-row TMA stores
+// After the last stage warps 2..9 write the dW partials and db to the
+// workspace.  Every wait is bounded.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "plan.cuh"
+#include "rdft4.cuh"
+#include "sm100.cuh"
+
+namespace feql {
+
+constexpr int kBwTB = 64;                    // tokens per stage (dX MMA M)
+constexpr int kBwBox = kBwTB * 128;          // 8 KB: 64 tokens x 16 channels x 4 fp16
+constexpr int kBwPlane = kBwTB * 32;         // 2 KB: one bin of one box
+constexpr int kBwXfWarps = 8;
+constexpr int kBwEpWarps = 4;
+constexpr int kBwThreads = 64 + (kBwXfWarps + kBwEpWarps) * 32;
+constexpr int kBwOutRows = 16;               // tokens per dX TMA store (one warp)
+constexpr int kBwOutBox = kBwOutRows * 128;  // 2 KB
+constexpr int kBwNumOut = 4;                 // staging buffers per dX epilogue warp
+constexpr int kBwMaxItems = 2 * kBwXfWarps * 32;  // (box, token) items a stage may hold
+
+struct TcBwdParams {
+  const uint8_t *wt;   // conj(What)^T tiles of the dX direction (one output tile)
+  int64_t N;
+  int C, D, Cs;        // Cs: workspace row stride
+  int nqd, nqc;        // 16-channel boxes of dy and of x
+  int slots;           // box slots per stage: max(8, nqd + nqc) (dW operand reads 8 d boxes)
+  int CT;              // dW columns: 16 * nqc
+  int BD;              // dX output tile (>= C)
+  int chunk_bytes;     // one dX weight chunk: 6 * BD rows x 32 B
+  int wres_bytes;      // nqd * chunk_bytes, 1 KB aligned
+  int stages;
+  int splits;
+  int64_t split_len;   // tokens per CTA, multiple of 64
+  int ndx;             // dX accumulator buffers (1 or 2)
+  float *ws;           // [splits][4][D][Cs]
+  float *ws_db;        // [splits][D]
+};
+
+struct BwSmem {
+  int wres, stage0, out0, bars, total;
+};
+
+__host__ __device__ inline BwSmem tc_bwd_smem(const TcBwdParams &p) {
+  BwSmem s;
+  s.wres = 0;
+  s.stage0 = p.wres_bytes;
+  s.out0 = s.stage0 + p.stages * p.slots * kBwBox;
+  s.bars = s.out0 + kBwEpWarps * kBwNumOut * kBwOutBox;
+  // full, tready, empty per stage; dxfull, dxempty x2; dwfull; wfull; tmem slot
+  s.total = s.bars + (3 * p.stages + 4 + 2) * 8 + 16;
+  return s;
+}
+
+// 14 warps over the 4 SM sub-partitions put 4 warps on one 16K-register slice:
+// 4 x 32 x 128 = 16,384.
+__global__ void __maxnreg__(128)
+tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
+              const __grid_constant__ CUtensorMap tm_dx, const TcBwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const BwSmem L = tc_bwd_smem(p);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *full = bars;
+  uint64_t *tready = bars + p.stages;
+  uint64_t *empty = bars + 2 * p.stages;
+  uint64_t *dxfull = bars + 3 * p.stages;
+  uint64_t *dxempty = dxfull + 2;
+  uint64_t *dwfull = dxempty + 2;
+  uint64_t *wfull = dwfull + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(wfull + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int split = blockIdx.x;
+  const int64_t t_begin = static_cast<int64_t>(split) * p.split_len;
+  int64_t t_end = t_begin + p.split_len;
+  if (t_end > p.N) t_end = p.N;
+  const int nst = t_begin < t_end ? static_cast<int>(cdiv(t_end - t_begin, kBwTB)) : 0;
+  const int nbox = p.nqd + p.nqc;
+  const int dx0 = 4 * p.CT;  // first TMEM column of the dX accumulators
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&tready[s], kBwXfWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dxfull[b], 1);
+      mbar_init(&dxempty[b], kBwEpWarps);
+    }
+    mbar_init(dwfull, 1);
+    mbar_init(wfull, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_dy);
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_dx);
+      if (nst > 0) {
+        mbar_arrive_expect_tx(wfull, p.nqd * p.chunk_bytes);
+        bulk_load(smem + L.wres, p.wt, p.nqd * p.chunk_bytes, wfull);
+      }
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ch = 0; ch < nst; ++ch) {
+        if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
+        if (ok) {
+          uint8_t *st = smem + L.stage0 + s * p.slots * kBwBox;
+          const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * kBwTB);
+          mbar_arrive_expect_tx(&full[s], nbox * kBwBox);
+          for (int q = 0; q < p.nqd; ++q)
+            tma_load_2d(st + q * kBwBox, &tm_dy, q * 16 * kT, row, &full[s]);
+          for (int q = 0; q < p.nqc; ++q)
+            tma_load_2d(st + (p.nqd + q) * kBwBox, &tm_x, q * 16 * kT, row, &full[s]);
+        }
+        if (++s == p.stages) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      // dW: planes hold -Im of bin 1 for dy and x alike (see tc_dw.cuh)
+      const uint32_t id_w = instr_desc(128, p.CT, 0, 0, 1, 1);
+      const uint32_t id_wneg = instr_desc(128, p.CT, 0, 0, 1, 1, 1);
+      // dX: M = 64 tokens, K-major operands
+      const uint32_t id_x1 = instr_desc(64, p.BD, 0, 0);
+      const uint32_t id_x2 = instr_desc(64, 2 * p.BD, 0, 0);
+      const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
+      const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
+      if (nst > 0 && ok) ok = mbar_wait(wfull, 0);
+      const uint32_t wres = smem_u32(smem + L.wres);
+      const uint32_t stage_base = smem_u32(smem + L.stage0);
+      const uint64_t dmn = smem_desc(0, kBwBox, 256, kSw32);  // planes read column-wise (dW)
+      const uint64_t dk = smem_desc(0, 16, 256, kSw32);       // K-major rows (dX, weights)
+      int s = 0;
+      uint32_t ph = 0;
+      for (int ch = 0; ch < nst; ++ch) {
+        if (ok) ok = mbar_wait(&full[s], ph);
+        if (ok) ok = mbar_wait(&tready[s], ph);
+        tc_fence_after();
+        const uint32_t st = stage_base + s * p.slots * kBwBox;
+        if (ok) {
+#pragma unroll
+          for (int k = 0; k < kBwTB / 16; ++k) {
+            const uint32_t a = st + k * 512, b = st + p.nqd * kBwBox + k * 512;  // 16 tokens
+            const uint64_t A0 = desc_at(dmn, a), A1 = desc_at(dmn, a + kBwPlane);
+            const uint64_t A2 = desc_at(dmn, a + 2 * kBwPlane), A3 = desc_at(dmn, a + 3 * kBwPlane);
+            const uint64_t B0 = desc_at(dmn, b), B1 = desc_at(dmn, b + kBwPlane);
+            const uint64_t B2 = desc_at(dmn, b + 2 * kBwPlane), B3 = desc_at(dmn, b + 3 * kBwPlane);
+            const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
+            mma_f16_ss(acc0, A0, B0, id_w, first);
+            mma_f16_ss(acc2, A1, B1, id_w, first);
+            mma_f16_ss(acc1r, A2, B2, id_w, first);
+            mma_f16_ss(acc1r, A3, B3, id_w, 1u);
+            mma_f16_ss(acc1i, A3, B2, id_wneg, first);
+            mma_f16_ss(acc1i, A2, B3, id_w, 1u);
+          }
+        }
+        const int b = ch % p.ndx;
+        if (ok) ok = mbar_wait(&dxempty[b], ((ch / p.ndx) & 1) ^ 1);
+        tc_fence_after();
+        if (ok) {
+          const uint32_t acc = tmem_base + dx0 + b * 4 * p.BD;
+          const uint32_t w1 = p.BD * 32, w2 = 2 * p.BD * 32, w4 = 4 * p.BD * 32;
+          for (int q = 0; q < p.nqd; ++q) {
+            const uint32_t box = st + q * kBwBox;
+            const uint32_t wq = wres + q * p.chunk_bytes;
+            const uint32_t in = q > 0 ? 1u : 0u;
+            mma_f16_ss(acc, desc_at(dk, box), desc_at(dk, wq), id_x1, in);
+            mma_f16_ss(acc + p.BD, desc_at(dk, box + kBwPlane), desc_at(dk, wq + w1), id_x1, in);
+            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 2 * kBwPlane), desc_at(dk, wq + w2),
+                       id_x2, in);
+            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 3 * kBwPlane), desc_at(dk, wq + w4),
+                       id_x2, 1u);
+          }
+          mma_commit(&dxfull[b]);
+          mma_commit(&empty[s]);
+        }
+        if (++s == p.stages) { s = 0; ph ^= 1; }
+      }
+      mma_commit(dwfull);
+    }
+  } else if (warp < 2 + kBwXfWarps) {
+    // ---------------------------------------------------------- transform
+    const int t = threadIdx.x - 64;
+    constexpr int kPer = kBwMaxItems / (kBwXfWarps * 32);  // items per thread (2)
+    float db_acc[kPer][16];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) db_acc[k][c] = 0.f;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int ch = 0; ch < nst; ++ch) {
+      if (ok) ok = mbar_wait(&full[s], ph);
+      uint8_t *st = smem + L.stage0 + s * p.slots * kBwBox;
+      uint32_t pl[kPer][4][8];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int e = t + k * kBwXfWarps * 32;
+        const int b = e / kBwTB, r = e % kBwTB;
+        if (b < nbox) {
+          const uint8_t *src = st + b * kBwBox + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
+            rdft4_pair(v, pl[k][0][q], pl[k][1][q], pl[k][2][q], pl[k][3][q]);
+          }
+        }
+      }
+      named_bar_sync(2, kBwXfWarps * 32);  // all rows read before the planes overwrite them
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int e = t + k * kBwXfWarps * 32;
+        const int b = e / kBwTB, r = e % kBwTB;
+        if (b < nbox) {
+#pragma unroll
+          for (int pp = 0; pp < 4; ++pp) {
+            uint8_t *row = st + b * kBwBox + pp * kBwPlane + r * 32;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              *reinterpret_cast<uint4 *>(row + (((hh ^ (r >> 2)) & 1) << 4)) =
+                  make_uint4(pl[k][pp][4 * hh + 0], pl[k][pp][4 * hh + 1], pl[k][pp][4 * hh + 2],
+                             pl[k][pp][4 * hh + 3]);
+          }
+          if (b < p.nqd) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 f = __half22float2(as_h2(pl[k][0][q]));
+              db_acc[k][2 * q] += f.x;
+              db_acc[k][2 * q + 1] += f.y;
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&tready[s]);
+      if (++s == p.stages) { s = 0; ph ^= 1; }
+    }
+
+    // ---------------------------------------------- dW partials -> workspace
+    if (ok) ok = mbar_wait(dwfull, 0);
+    tc_fence_after();
+    const int quad = warp & 3, half = (warp - 2) / 4;
+    const int d = quad * 32 + lane;
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    for (int bin = 0; bin < 4; ++bin) {
+      float *dst = p.ws + ((static_cast<int64_t>(split) * 4 + bin) * p.D + d) * p.Cs;
+      for (int g = half; g < p.CT / 16; g += 2) {
+        uint32_t v[16];
+        tmem_ld16(tl + bin * p.CT + g * 16, v);
+        tmem_ld_wait();
+        if (d < p.D && g * 16 < p.C) {
+          float4 *o = reinterpret_cast<float4 *>(dst + g * 16);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+    // db: fixed-order reduction of the per-thread partials through shared memory
+    named_bar_sync(3, kBwXfWarps * 32);  // stages are free: every chunk has been consumed
+    float *sdb = reinterpret_cast<float *>(smem + L.stage0);  // [kBwMaxItems][16]
+#pragma unroll
+    for (int k = 0; k < kPer; ++k)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) sdb[(t + k * kBwXfWarps * 32) * 16 + c] = db_acc[k][c];
+    named_bar_sync(3, kBwXfWarps * 32);
+    if (t < p.nqd * 16) {
+      const int bb = t / 16, c = t % 16;
+      float sum = 0.f;
+      for (int rr = 0; rr < kBwTB; ++rr) sum += sdb[(bb * kBwTB + rr) * 16 + c];
+      const int dd = bb * 16 + c;
+      if (dd < p.D) p.ws_db[static_cast<int64_t>(split) * p.D + dd] = sum;
+    }
+  } else {
+    // ------------------------------------------------------- dX epilogue
+    const int quad = warp & 3;
+    const int ew = warp - 2 - kBwXfWarps;
+    uint8_t *obase = smem + L.out0 + ew * kBwNumOut * kBwOutBox;
+    const int groups = p.BD / 16;
+    int oi = 0;
+    for (int ch = 0; ch < nst; ++ch) {
+      const int b = ch % p.ndx;
+      if (ok) ok = mbar_wait(&dxfull[b], (ch / p.ndx) & 1);
+      tc_fence_after();
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + dx0 + b * 4 * p.BD;
+      const int64_t tok0 = t_begin + static_cast<int64_t>(ch) * kBwTB + quad * kBwOutRows;
+      for (int g = 0; g < groups; ++g) {
+        uint32_t packed[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t y0[8], y2[8], y1r[8], y1i[8];
+          const uint32_t col = tl + g * 16 + h * 8;
+          tmem_ld8(col, y0);
+          tmem_ld8(col + p.BD, y2);
+          tmem_ld8(col + 2 * p.BD, y1r);
+          tmem_ld8(col + 3 * p.BD, y1i);
+          tmem_ld_wait();
+          if (h == 1 && g == groups - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
+            const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
+            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+          }
+        }
+        if (g * 16 >= p.C) continue;  // whole group is padding
+        uint8_t *ob = obase + (oi % kBwNumOut) * kBwOutBox;
+        if (lane == 0) bulk_wait_read<kBwNumOut - 1>();
+        __syncwarp();
+        if (lane < kBwOutRows) {  // lanes 0..15 hold this warp's 16 tokens
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4 *>(ob + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                           packed[4 * q + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_dx, g * 16 * kT, static_cast<int32_t>(tok0), ob);
+          bulk_commit();
+        }
+        ++oi;
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace feql

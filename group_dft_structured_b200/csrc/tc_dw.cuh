@@ -151,28 +151,30 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     if (lane == 0) {
       const uint32_t id = instr_desc(kDwMT, p.CT, 0, 0, 1, 1);
       const uint32_t id_neg = instr_desc(kDwMT, p.CT, 0, 0, 1, 1, 1);
-      const uint32_t lbo = chunk_plane, sbo = 256;
+      const uint64_t dmn = smem_desc(0, chunk_plane, 256, kSw32);  // MN-major planes
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
+      const uint32_t plane_base = smem_u32(smem + L.plane0);
+      const uint32_t a_bin = 8 * chunk_plane, b_bin = p.nqc_max * chunk_plane;
       for (int ch = 0; ch < nchunks; ++ch) {
         const int pb = ch & 1;
         if (ok) ok = mbar_wait(&pfull[pb], (ch >> 1) & 1);
         tc_fence_after();
         if (ok) {
-          const uint32_t pl = smem_u32(smem + L.plane0 + pb * p.plane_bytes);
+          const uint32_t pl = plane_base + pb * p.plane_bytes;
           for (int k = 0; k < p.TB / 16; ++k) {
-            const uint32_t ko = k * 512;  // 16 tokens x 32 B
-            auto A = [&](int bin) { return smem_desc(pl + bin * 8 * chunk_plane + ko, lbo, sbo, kSw32); };
-            auto B = [&](int bin) {
-              return smem_desc(pl + x_off + bin * p.nqc_max * chunk_plane + ko, lbo, sbo, kSw32);
-            };
+            const uint32_t a = pl + k * 512, b = pl + x_off + k * 512;  // 16 tokens x 32 B
+            const uint64_t A0 = desc_at(dmn, a), A1 = desc_at(dmn, a + a_bin);
+            const uint64_t A2 = desc_at(dmn, a + 2 * a_bin), A3 = desc_at(dmn, a + 3 * a_bin);
+            const uint64_t B0 = desc_at(dmn, b), B1 = desc_at(dmn, b + b_bin);
+            const uint64_t B2 = desc_at(dmn, b + 2 * b_bin), B3 = desc_at(dmn, b + 3 * b_bin);
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
-            mma_f16_ss(acc0, A(0), B(0), id, first);
-            mma_f16_ss(acc2, A(1), B(1), id, first);
-            mma_f16_ss(acc1r, A(2), B(2), id, first);
-            mma_f16_ss(acc1r, A(3), B(3), id, 1u);
-            mma_f16_ss(acc1i, A(3), B(2), id_neg, first);
-            mma_f16_ss(acc1i, A(2), B(3), id, 1u);
+            mma_f16_ss(acc0, A0, B0, id, first);
+            mma_f16_ss(acc2, A1, B1, id, first);
+            mma_f16_ss(acc1r, A2, B2, id, first);
+            mma_f16_ss(acc1r, A3, B3, id, 1u);
+            mma_f16_ss(acc1i, A3, B2, id_neg, first);
+            mma_f16_ss(acc1i, A2, B3, id, 1u);
           }
           mma_commit(&pempty[pb]);
         }

@@ -185,6 +185,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       const uint32_t id_bd = instr_desc(kBM, p.BD, 0, 0);
       const uint32_t id_2bd = instr_desc(kBM, 2 * p.BD, 0, 0);
       const uint32_t wrow = 32;  // bytes per weight row (16 fp16)
+      const uint64_t dsw32 = smem_desc(0, 16, 256, kSw32);  // K-major, 32-byte swizzle
+      const uint32_t stage_base = smem_u32(smem + L.stage0), wres_base = smem_u32(smem + L.wres);
       int m, j;
       if (p.resident && tc_unit(p, 0, m, j)) ok = mbar_wait(wfull, 0);
       int s = 0;
@@ -200,18 +202,16 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
-            const uint32_t xs = smem_u32(smem + L.stage0 + s * p.stage_bytes);
-            const uint32_t ws = p.resident ? smem_u32(smem + L.wres) + kc * p.chunk_bytes
-                                           : xs + kXChunkBytes;
+            const uint32_t xs = stage_base + s * p.stage_bytes;
+            const uint32_t ws = p.resident ? wres_base + kc * p.chunk_bytes : xs + kXChunkBytes;
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
-            mma_f16_ss(acc, smem_desc(xs + 0 * kPlaneBytes, 16, 256, kSw32),
-                       smem_desc(ws, 16, 256, kSw32), id_bd, acc_in);
-            mma_f16_ss(acc + p.BD, smem_desc(xs + 1 * kPlaneBytes, 16, 256, kSw32),
-                       smem_desc(ws + p.BD * wrow, 16, 256, kSw32), id_bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, smem_desc(xs + 2 * kPlaneBytes, 16, 256, kSw32),
-                       smem_desc(ws + 2 * p.BD * wrow, 16, 256, kSw32), id_2bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, smem_desc(xs + 3 * kPlaneBytes, 16, 256, kSw32),
-                       smem_desc(ws + 4 * p.BD * wrow, 16, 256, kSw32), id_2bd, 1u);
+            mma_f16_ss(acc, desc_at(dsw32, xs), desc_at(dsw32, ws), id_bd, acc_in);
+            mma_f16_ss(acc + p.BD, desc_at(dsw32, xs + kPlaneBytes),
+                       desc_at(dsw32, ws + p.BD * wrow), id_bd, acc_in);
+            mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 2 * kPlaneBytes),
+                       desc_at(dsw32, ws + 2 * p.BD * wrow), id_2bd, acc_in);
+            mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 3 * kPlaneBytes),
+                       desc_at(dsw32, ws + 4 * p.BD * wrow), id_2bd, 1u);
             mma_commit(&empty[s]);
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }

@@ -7,8 +7,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward_dw, feql_backward_dw_workspace_bytes,
-               feql_backward_dx, feql_forward, feql_weight_fft, feql_weight_fft_bytes)
+from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward, feql_backward_dw,
+               feql_backward_dw_workspace_bytes, feql_backward_dx, feql_forward, feql_weight_fft,
+               feql_weight_fft_bytes)
 
 
 def torch_dtype(mode: int):
@@ -44,6 +45,20 @@ def backward_dx(dy: torch.Tensor, What: torch.Tensor, C: int, mode: int, out=Non
 def dw_workspace(N: int, C: int, D: int, mode: int, device) -> torch.Tensor:
     nbytes = feql_backward_dw_workspace_bytes(N, C, D, mode)
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def backward(x: torch.Tensor, dy: torch.Tensor, What: torch.Tensor, mode: int, ws=None,
+             with_db: bool = True, stream=None):
+    """dx, dW, db from one call (fused single pass over dy where supported)."""
+    N, C, _ = x.shape
+    D = dy.shape[1]
+    if ws is None:
+        ws = dw_workspace(N, C, D, mode, x.device)
+    dx = torch.empty((N, C, 4), dtype=x.dtype, device=x.device)
+    dW = torch.empty((D, C, 4), dtype=x.dtype, device=x.device)
+    db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
+    feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode, stream)
+    return dx, dW, db
 
 
 def backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, ws=None, out=None,

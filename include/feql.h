@@ -113,6 +113,19 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db,
                      void *ws, size_t ws_bytes,
                      int64_t N, int C, int D, int dtype, feql_stream stream);
 
+/* a5 + a6 fused — both gradients from one pass over dy (technical summary
+ * "Implementazione": fused dataflow; dX and dW share the rDFT of dy):
+ * the results of feql_backward_dx followed by feql_backward_dw, reading x and
+ * dy once instead of dy twice.  Fused for FEQL_FP16 with C <= 64, D <= 128
+ * (one dW tile, one dX output tile: the bench's Swin-like layer); any other
+ * shape or mode runs the two separate passes and returns their result.
+ *   x, dy, What : as for feql_backward_dx / feql_backward_dw
+ *   dx  : device [N][C][4] (written)   dW : [D][C][4]   db : [D] or NULL
+ *   ws  : ws_bytes >= feql_backward_dw_workspace_bytes(N, C, D, dtype) */
+int feql_backward(const void *x, const void *dy, const void *What, void *dx, void *dW, void *db,
+                  void *ws, size_t ws_bytes, int64_t N, int C, int D, int dtype,
+                  feql_stream stream);
+
 /* Weight gradient for callers that cannot allocate device memory (code inside
  * a framework that owns every allocation, plug-ins that are handed only their
  * input and output tensors, runtimes that forbid allocation after start-up).

@@ -159,6 +159,51 @@ def test_fp16_tensor_core_matches_fp16_simt_closely():
         assert O.rel_err(a[k], b[k]) < 2e-3, k
 
 
+# ----------------------------------------------------------- fused backward
+
+FUSED = [(517, 24, 96), (300, 16, 16), (1000, 48, 64), (129, 6, 40), (64, 24, 96), (1, 8, 8),
+         (4097, 16, 112)]
+SEPARATE = [(257, 256, 256), (300, 96, 24), (700, 32, 112)]
+
+
+@pytest.mark.parametrize("N,C,D", FUSED + SEPARATE)
+def test_fused_backward_matches_oracle(N, C, D):
+    mode = F.FEQL_FP16
+    inp = make_inputs(12, N, C, D, "fp16")
+    x, W, dy = dev(inp["x"]), dev(inp["W"]), dev(inp["dy"])
+    What = Lyr.weight_fft(W, mode)
+    dx, dW, db = Lyr.backward(x, dy, What, mode)
+    assert F.feql_device_status() == F.FEQL_OK
+    out = {"dx": host(dx), "dW": host(dW), "db": host(db)}
+    check(out, inp, mode)
+    # same results as the two separate passes, within rounding
+    sep_dx = host(Lyr.backward_dx(dy, What, C, mode))
+    sep_dW, sep_db = (host(t) for t in Lyr.backward_dw(x, dy, mode))
+    assert O.rel_err(out["dx"], sep_dx) < 2e-3
+    assert O.rel_err(out["dW"], sep_dW) < 2e-3 and O.rel_err(out["db"], sep_db) < 2e-3
+
+
+def test_fused_backward_is_deterministic_and_stays_in_bounds():
+    mode = F.FEQL_FP16
+    N, C, D = 3000, 24, 96
+    inp = make_inputs(13, N, C, D, "fp16")
+    x, W, dy = dev(inp["x"]), dev(inp["W"]), dev(inp["dy"])
+    What = Lyr.weight_fft(W, mode)
+    guard = 4096
+    n = N * C * 4
+    buf = torch.full((n + 2 * guard,), -3.0, dtype=torch.float16, device="cuda")
+    dx = buf[guard:guard + n].view(N, C, 4)
+    dW1 = torch.empty((D, C, 4), dtype=torch.float16, device="cuda")
+    db1 = torch.empty((D,), dtype=torch.float16, device="cuda")
+    ws = Lyr.dw_workspace(N, C, D, mode, "cuda")
+    F.feql_backward(x, dy, What, dx, dW1, db1, ws, ws.numel(), N, C, D, mode)
+    dW2, db2 = torch.empty_like(dW1), torch.empty_like(db1)
+    F.feql_backward(x, dy, What, dx, dW2, db2, ws, ws.numel(), N, C, D, mode)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:guard] == -3.0) and torch.all(buf[guard + n:] == -3.0)
+    assert torch.equal(dW1, dW2) and torch.equal(db1, db2)
+
+
 # ---------------------------------------------------------------- full sizes
 
 @pytest.mark.parametrize("wid,mode", [(1, F.FEQL_FP32), (2, F.FEQL_FP16), (3, F.FEQL_FP16),
@@ -168,3 +213,15 @@ def test_workload_full_size(wid, mode):
     inp = workload_inputs(wid, dtype=NAME[mode])
     errs = check(run_all(inp, mode, passes=w.passes), inp, mode)
     print(w.name, NAME[mode], errs)
+
+
+@pytest.mark.parametrize("wid", [4, 5])
+def test_workload_full_size_fused_backward(wid):
+    mode = F.FEQL_FP16
+    inp = workload_inputs(wid, dtype="fp16")
+    x, W, dy = dev(inp["x"]), dev(inp["W"]), dev(inp["dy"])
+    What = Lyr.weight_fft(W, mode)
+    dx, dW, db = Lyr.backward(x, dy, What, mode)
+    assert F.feql_device_status() == F.FEQL_OK
+    errs = check({"dx": host(dx), "dW": host(dW), "db": host(db)}, inp, mode)
+    print(WORKLOADS[wid].name, "fused backward", errs)
