@@ -242,8 +242,9 @@ TcDwParams make_tc_dw_plan(int64_t N, int C, int D, int sms) {
   p.splits = static_cast<int>(cdiv(N > 0 ? N : 1, p.split_len));
   p.raw_bytes = nbox * p.TB * 128;
   p.plane_bytes = 4 * (8 + p.nqc_max) * p.TB * 32;
+  p.merged = 6 * p.CT <= 512 ? 1 : 0;
   int cols = 32;
-  while (cols < 4 * p.CT) cols *= 2;
+  while (cols < (p.merged ? 6 : 4) * p.CT) cols *= 2;
   p.tmem_cols = cols;
   p.stages = 0;
   p.ws = nullptr;
@@ -300,8 +301,10 @@ bool make_tc_bwd_plan(int64_t N, int C, int D, const WhatLayout &L, const Device
   p.CT = 16 * p.nqc;
   p.BD = L.dx.BD;
   p.chunk_bytes = L.dx.chunk_bytes;
+  // TMEM columns: dW (6*CT merged, else 4*CT) + dX buffers (4*BD each)
   if (4 * p.CT + 4 * p.BD > 512) return false;
-  p.ndx = (4 * p.CT + 8 * p.BD <= 512) ? 2 : 1;
+  p.merged = (6 * p.CT + 4 * p.BD <= 512) ? 1 : 0;
+  p.ndx = ((p.merged ? 6 : 4) * p.CT + 8 * p.BD <= 512) ? 2 : 1;
   p.wres_bytes = static_cast<int>(align_up(static_cast<int64_t>(p.nqd) * p.chunk_bytes, 1024));
   int64_t s = dev.sms;
   if (s > cdiv(N, kBwTB)) s = cdiv(N, kBwTB);

@@ -33,6 +33,7 @@
 #include "plan.cuh"
 #include "rdft4.cuh"
 #include "sm100.cuh"
+#include "tc_dw.cuh"
 
 namespace feql {
 
@@ -61,6 +62,7 @@ struct TcBwdParams {
   int splits;
   int64_t split_len;   // tokens per CTA, multiple of 64
   int ndx;             // dX accumulator buffers (1 or 2)
+  int merged;          // dW bin 1 as two N = 2*CT MMAs (6*CT TMEM columns), see tc_dw.cuh
   float *ws;           // [splits][4][D][Cs]
   float *ws_db;        // [splits][D]
 };
@@ -106,7 +108,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
   if (t_end > p.N) t_end = p.N;
   const int nst = t_begin < t_end ? static_cast<int>(cdiv(t_end - t_begin, kBwTB)) : 0;
   const int nbox = p.nqd + p.nqc;
-  const int dx0 = 4 * p.CT;  // first TMEM column of the dX accumulators
+  const int dx0 = (p.merged ? 6 : 4) * p.CT;  // first TMEM column of the dX accumulators
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -169,10 +171,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const uint32_t id_x2 = instr_desc(64, 2 * p.BD, 0, 0);
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
+      const uint32_t acca = tmem_base + 2 * p.CT, accb = tmem_base + 4 * p.CT;
+      const uint32_t id_w2 = instr_desc(128, 2 * p.CT, 0, 0, 1, 1);
       if (nst > 0 && ok) ok = mbar_wait(wfull, 0);
       const uint32_t wres = smem_u32(smem + L.wres);
       const uint32_t stage_base = smem_u32(smem + L.stage0);
-      const uint64_t dmn = smem_desc(0, kBwBox, 256, kSw32);  // planes read column-wise (dW)
+      const uint64_t dmn = smem_desc(0, kBwBox, 256, kSw32);    // dy planes read column-wise (dW)
+      const uint64_t dmx = smem_desc(0, kBwPlane, 256, kSw32);  // x planes read column-wise (dW)
       const uint64_t dk = smem_desc(0, 16, 256, kSw32);       // K-major rows (dX, weights)
       int s = 0;
       uint32_t ph = 0;
@@ -184,18 +189,25 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         if (ok) {
 #pragma unroll
           for (int k = 0; k < kBwTB / 16; ++k) {
+            // dy planes: d chunks 8 KB apart; x planes: plane-major, c chunks 2 KB apart
             const uint32_t a = st + k * 512, b = st + p.nqd * kBwBox + k * 512;  // 16 tokens
+            const uint32_t xb = p.nqc * kBwPlane;  // one x bin
             const uint64_t A0 = desc_at(dmn, a), A1 = desc_at(dmn, a + kBwPlane);
             const uint64_t A2 = desc_at(dmn, a + 2 * kBwPlane), A3 = desc_at(dmn, a + 3 * kBwPlane);
-            const uint64_t B0 = desc_at(dmn, b), B1 = desc_at(dmn, b + kBwPlane);
-            const uint64_t B2 = desc_at(dmn, b + 2 * kBwPlane), B3 = desc_at(dmn, b + 3 * kBwPlane);
+            const uint64_t B0 = desc_at(dmx, b), B1 = desc_at(dmx, b + xb);
+            const uint64_t B2 = desc_at(dmx, b + 2 * xb), B3 = desc_at(dmx, b + 3 * xb);
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
             mma_f16_ss(acc0, A0, B0, id_w, first);
             mma_f16_ss(acc2, A1, B1, id_w, first);
-            mma_f16_ss(acc1r, A2, B2, id_w, first);
-            mma_f16_ss(acc1r, A3, B3, id_w, 1u);
-            mma_f16_ss(acc1i, A3, B2, id_wneg, first);
-            mma_f16_ss(acc1i, A2, B3, id_w, 1u);
+            if (p.merged) {  // see tc_dw.cuh: acc_a, acc_b over [Re X1 | -Im X1]
+              mma_f16_ss(acca, A2, B2, id_w2, first);
+              mma_f16_ss(accb, A3, B2, id_w2, first);
+            } else {
+              mma_f16_ss(acc1r, A2, B2, id_w, first);
+              mma_f16_ss(acc1r, A3, B3, id_w, 1u);
+              mma_f16_ss(acc1i, A3, B2, id_wneg, first);
+              mma_f16_ss(acc1i, A2, B3, id_w, 1u);
+            }
           }
         }
         const int b = ch % p.ndx;
@@ -256,9 +268,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         const int e = t + k * kBwXfWarps * 32;
         const int b = e / kBwTB, r = e % kBwTB;
         if (b < nbox) {
+          // dy box: its four planes in place; x box q: plane pp at x + (pp * nqc + q) planes
+          uint8_t *base = b < p.nqd ? st + b * kBwBox
+                                    : st + p.nqd * kBwBox + (b - p.nqd) * kBwPlane;
+          const int pstride = b < p.nqd ? kBwPlane : p.nqc * kBwPlane;
 #pragma unroll
           for (int pp = 0; pp < 4; ++pp) {
-            uint8_t *row = st + b * kBwBox + pp * kBwPlane + r * 32;
+            uint8_t *row = base + pp * pstride + r * 32;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
               *reinterpret_cast<uint4 *>(row + (((hh ^ (r >> 2)) & 1) << 4)) =
@@ -287,18 +303,17 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     const int quad = warp & 3, half = (warp - 2) / 4;
     const int d = quad * 32 + lane;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    for (int bin = 0; bin < 4; ++bin) {
-      float *dst = p.ws + ((static_cast<int64_t>(split) * 4 + bin) * p.D + d) * p.Cs;
-      for (int g = half; g < p.CT / 16; g += 2) {
-        uint32_t v[16];
-        tmem_ld16(tl + bin * p.CT + g * 16, v);
-        tmem_ld_wait();
-        if (d < p.D && g * 16 < p.C) {
-          float4 *o = reinterpret_cast<float4 *>(dst + g * 16);
+    float *dst = p.ws + (static_cast<int64_t>(split) * 4 * p.D + d) * p.Cs;
+    const int64_t bin_stride = static_cast<int64_t>(p.D) * p.Cs;
+    for (int g = half; g < p.CT / 8; g += 2) {  // 8-column steps
+      float G[4][8];
+      dw_acc_read8(tl, p.CT, g * 8, p.merged, G);
+      if (d < p.D && g * 8 < p.C) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int bin = 0; bin < 4; ++bin) {
+          float4 *o = reinterpret_cast<float4 *>(dst + bin * bin_stride + g * 8);
+          o[0] = make_float4(G[bin][0], G[bin][1], G[bin][2], G[bin][3]);
+          o[1] = make_float4(G[bin][4], G[bin][5], G[bin][6], G[bin][7]);
         }
       }
     }

@@ -51,6 +51,7 @@ struct TcDwParams {
   int raw_bytes;         // (nqd_max + nqc_max) * TB * 128
   int plane_bytes;       // 4 * (8 + nqc_max) * TB * 32
   int tmem_cols;
+  int merged;            // 1: bin-1 products as two N = 2*CT MMAs (needs 6*CT TMEM columns)
   float *ws;             // [splits][4][D][Cs]
   float *ws_db;          // [splits][D]
 };
@@ -58,6 +59,42 @@ struct TcDwParams {
 struct DwSmem {
   int raw0, plane0, bars, total;
 };
+
+// This thread's TMEM row of the dW accumulators, 8 columns from c0, as the four
+// bins (G0, G2, Re G1, Im G1).  Column layout: [0,CT) G0, [CT,2CT) G2, then
+// either Re G1, Im G1 (CT each) or, merged, acc_a and acc_b (2*CT each) with
+// Re G1 = a[c] + b[CT+c] and Im G1 = a[CT+c] - b[c].
+__device__ __forceinline__ void dw_acc_read8(uint32_t tl, int CT, int c0, bool merged,
+                                             float (&G)[4][8]) {
+  uint32_t v0[8], v2[8], r0[8], r1[8];
+  tmem_ld8(tl + c0, v0);
+  tmem_ld8(tl + CT + c0, v2);
+  tmem_ld8(tl + 2 * CT + c0, r0);
+  tmem_ld8(tl + 3 * CT + c0, r1);
+  if (merged) {
+    uint32_t b0[8], b1[8];
+    tmem_ld8(tl + 4 * CT + c0, b0);
+    tmem_ld8(tl + 5 * CT + c0, b1);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      G[2][i] = __uint_as_float(r0[i]) + __uint_as_float(b1[i]);
+      G[3][i] = __uint_as_float(r1[i]) - __uint_as_float(b0[i]);
+    }
+  } else {
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      G[2][i] = __uint_as_float(r0[i]);
+      G[3][i] = __uint_as_float(r1[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    G[0][i] = __uint_as_float(v0[i]);
+    G[1][i] = __uint_as_float(v2[i]);
+  }
+}
 
 __host__ __device__ inline DwSmem tc_dw_smem(const TcDwParams &p) {
   DwSmem s;
@@ -148,12 +185,18 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     // The planes hold -Im of bin 1 (for dy and x alike), so
     //   Re G1 = dY1r X1r + (-dY1i)(-X1i),   Im G1 = -(-dY1i) X1r + dY1r (-X1i),
     // the first Im term through the B-negate bit.
+    // Merged form (6*CT TMEM columns): the x planes Re X1 and -Im X1 are
+    // adjacent, so one N = 2*CT MMA per dy plane gives both products:
+    //   acc_a = [dY1r X1r | -dY1r X1i],  acc_b = [-dY1i X1r | dY1i X1i]
+    // and the epilogue forms Re G1 = a0 + b1, Im G1 = a1 - b0 (4 MMAs, not 6).
     if (lane == 0) {
       const uint32_t id = instr_desc(kDwMT, p.CT, 0, 0, 1, 1);
       const uint32_t id_neg = instr_desc(kDwMT, p.CT, 0, 0, 1, 1, 1);
+      const uint32_t id2 = instr_desc(kDwMT, 2 * p.CT, 0, 0, 1, 1);
       const uint64_t dmn = smem_desc(0, chunk_plane, 256, kSw32);  // MN-major planes
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
+      const uint32_t acca = tmem_base + 2 * p.CT, accb = tmem_base + 4 * p.CT;
       const uint32_t plane_base = smem_u32(smem + L.plane0);
       const uint32_t a_bin = 8 * chunk_plane, b_bin = p.nqc_max * chunk_plane;
       for (int ch = 0; ch < nchunks; ++ch) {
@@ -171,10 +214,15 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
             mma_f16_ss(acc0, A0, B0, id, first);
             mma_f16_ss(acc2, A1, B1, id, first);
-            mma_f16_ss(acc1r, A2, B2, id, first);
-            mma_f16_ss(acc1r, A3, B3, id, 1u);
-            mma_f16_ss(acc1i, A3, B2, id_neg, first);
-            mma_f16_ss(acc1i, A2, B3, id, 1u);
+            if (p.merged) {
+              mma_f16_ss(acca, A2, B2, id2, first);
+              mma_f16_ss(accb, A3, B2, id2, first);
+            } else {
+              mma_f16_ss(acc1r, A2, B2, id, first);
+              mma_f16_ss(acc1r, A3, B3, id, 1u);
+              mma_f16_ss(acc1i, A3, B2, id_neg, first);
+              mma_f16_ss(acc1i, A2, B3, id, 1u);
+            }
           }
           mma_commit(&pempty[pb]);
         }
@@ -244,19 +292,18 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
     const int d = ti * kDwMT + quad * 32 + lane;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const int ncol = p.CT / 16;
-    for (int bin = 0; bin < 4; ++bin) {
-      float *dst = p.ws + ((static_cast<int64_t>(split) * 4 + bin) * p.D + d) * p.Cs +
-                   static_cast<int64_t>(tj) * p.CT;
-      for (int g = half; g < ncol; g += 2) {
-        uint32_t v[16];
-        tmem_ld16(tl + bin * p.CT + g * 16, v);
-        tmem_ld_wait();
-        if (d < p.D && tj * p.CT + g * 16 < p.C) {
-          float4 *o = reinterpret_cast<float4 *>(dst + g * 16);
+    float *dst = p.ws + (static_cast<int64_t>(split) * 4 * p.D + d) * p.Cs +
+                 static_cast<int64_t>(tj) * p.CT;
+    const int64_t bin_stride = static_cast<int64_t>(p.D) * p.Cs;
+    for (int g = half; g < 2 * ncol; g += 2) {  // 8-column steps
+      float G[4][8];
+      dw_acc_read8(tl, p.CT, g * 8, p.merged, G);
+      if (d < p.D && tj * p.CT + g * 8 < p.C) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            o[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                               __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int bin = 0; bin < 4; ++bin) {
+          float4 *o = reinterpret_cast<float4 *>(dst + bin * bin_stride + g * 8);
+          o[0] = make_float4(G[bin][0], G[bin][1], G[bin][2], G[bin][3]);
+          o[1] = make_float4(G[bin][4], G[bin][5], G[bin][6], G[bin][7]);
         }
       }
     }
