@@ -42,7 +42,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=WORKLOAD_ID)
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
+                    help="workload id 1-5 (group_dft_structured_b200/workloads.py)")
+    ap.add_argument("--dtype", choices=["fp16", "fp32"], default=None,
+                    help="override the workload's dtype (e.g. the fp32 run of the square layer)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -246,6 +249,9 @@ def main():
     from group_dft_structured_b200.workloads import WORKLOADS, make_inputs
 
     w = WORKLOADS[args.workload]
+    if args.dtype is not None:
+        import dataclasses
+        w = dataclasses.replace(w, dtype=args.dtype)
     torch.cuda.set_device(local_rank)
     if world > 1:
         from datetime import timedelta
@@ -405,7 +411,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16" if w.dtype == "fp16" else "f32",
         "data": "synthetic",
         "config": {"workload": w.name, "N": N, "C": C, "D": D, "T": 4,
                    "passes": passes, "accumulate": "f32", "l2": "inputs larger than L2, no flush",
