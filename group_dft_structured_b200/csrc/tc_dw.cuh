@@ -63,10 +63,12 @@ struct DwSmem {
 // This thread's TMEM row of the dW accumulators, 8 columns from c0, as the four
 // bins (G0, G2, Re G1, Im G1).  Column layout: [0,CT) G0, [CT,2CT) G2, then
 // either Re G1, Im G1 (CT each) or, merged, acc_a and acc_b (2*CT each) with
-// Re G1 = a[c] + b[CT+c] and Im G1 = a[CT+c] - b[c].
+// Re G1 = a[c] + b[CT+c] and Im G1 = a[CT+c] - b[c].  Whole warp: the TMEM
+// loads are warp-collective (.sync.aligned), so the warp reconverges first.
 __device__ __forceinline__ void dw_acc_read8(uint32_t tl, int CT, int c0, bool merged,
                                              float (&G)[4][8]) {
   uint32_t v0[8], v2[8], r0[8], r1[8];
+  __syncwarp();
   tmem_ld8(tl + c0, v0);
   tmem_ld8(tl + CT + c0, v2);
   tmem_ld8(tl + 2 * CT + c0, r0);
