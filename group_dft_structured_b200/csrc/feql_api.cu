@@ -314,6 +314,7 @@ bool make_tc_bwd_plan(int64_t N, int C, int D, const WhatLayout &L, const Device
   p.stages = 4;
   while (p.stages > 2 && tc_bwd_smem(p).total > budget) --p.stages;
   if (tc_bwd_smem(p).total > budget) return false;
+  p.dx = nullptr;
   p.ws = nullptr;
   p.ws_db = nullptr;
   return true;
@@ -323,20 +324,19 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
                   __half *dW, __half *db, float *ws, const DeviceInfo &dev, cudaStream_t stream) {
   if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
   p.wt = wt;
+  p.dx = dx;
   p.ws = ws;
   p.ws_db = ws + static_cast<int64_t>(p.splits) * 4 * p.D * p.Cs;
   const int smem = tc_bwd_smem(p).total + 1024;
-  CUtensorMap tm_dy, tm_x, tm_dx;
+  CUtensorMap tm_dy, tm_x;
   int st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, kBwTB);
   if (st != FEQL_OK) return st;
   st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB);
   if (st != FEQL_OK) return st;
-  st = make_tmap_f16(&tm_dx, dx, p.N, static_cast<int64_t>(p.C) * kT, kBwOutRows);
-  if (st != FEQL_OK) return st;
   if (cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FEQL_ERR_CUDA;
-  tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, tm_dx, p);
+  tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, p);
   const int64_t rblocks = dw_reduce_blocks(p.C, p.D);
   if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
   dw_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), kRedOut * kRedGroups, 0, stream>>>(

@@ -25,7 +25,7 @@ struct TcPlan {
   int BD;            // output channels per tile (multiple of 16, <= 128)
   int nD;            // output-channel tiles
   int nK;            // K-chunks of kCK channels
-  int chunk_bytes;   // bytes of the weight tiles for one (tile, chunk): 6*BD rows x 32 B
+  int chunk_bytes;   // bytes of the weight tiles for one (tile, chunk): 5*BD rows x 32 B
   int64_t bytes;     // nD * nK * chunk_bytes
 };
 
@@ -40,7 +40,7 @@ __host__ __device__ inline TcPlan make_tc_plan(int Ci, int Do) {
   p.nK = static_cast<int>(cdiv(Ci, kCK));
   p.nD = static_cast<int>(cdiv(Do, p.nK <= 4 ? kMaxBD / 2 : kMaxBD));
   p.BD = static_cast<int>(align_up(cdiv(Do, p.nD), 16));
-  p.chunk_bytes = 6 * p.BD * kCK * 2;
+  p.chunk_bytes = 5 * p.BD * kCK * 2;
   p.bytes = static_cast<int64_t>(p.nD) * p.nK * p.chunk_bytes;
   return p;
 }
@@ -54,9 +54,10 @@ __host__ __device__ inline int sw32_offset(int row, int k) {
 
 // Layout of the opaque What buffer.
 //   fp16 tensor-core modes: [fwd chunks][dx chunks], each direction laid out
-//       [tile j][chunk kc][rows 0..6BD) with rows
-//       [0,BD) What0 | [BD,2BD) What2 | [2BD,4BD) (Re1 ; Im1) | [4BD,6BD) (Im1 ; -Re1)
-//   (the last block multiplies the stored -Im X1 plane)
+//       [tile j][chunk kc][rows 0..5BD) with rows
+//       [0,BD) What0 | [BD,2BD) What2 | [2BD,3BD) Re1 | [3BD,4BD) Im1 | [4BD,5BD) -Re1
+//   so that rows [2BD,4BD) = (Re1 ; Im1) multiply Re X1 and the overlapping
+//   window [3BD,5BD) = (Im1 ; -Re1) multiplies the stored -Im X1 plane.
 //   SIMT modes: fp32 planes [dir][bin p][Do][Ci], p = (0, 2, Re 1, Im 1).
 struct WhatLayout {
   bool tc;

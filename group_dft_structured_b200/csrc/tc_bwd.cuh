@@ -23,7 +23,10 @@
 //                     read row-wise) into a double-buffered accumulator
 //   warps 10..13 dX epilogue: the M=64 accumulator sits in TMEM lanes
 //               (m mod 16) + 32 * (m / 16), so warp q's lanes 0..15 hold
-//               tokens 16q..16q+15; inverse rDFT, fp16, 16-row TMA stores
+//               tokens 16q..16q+15; inverse rDFT, fp16, direct 16-byte stores
+//               (each lane writes whole channels of its own token row), which
+//               leaves the shared memory to the stages (three fit for C = 24,
+//               D = 96)
 // After the last stage warps 2..9 write the dW partials and db to the
 // workspace.  Every wait is bounded.
 #pragma once
@@ -43,20 +46,18 @@ constexpr int kBwPlane = kBwTB * 32;         // 2 KB: one bin of one box
 constexpr int kBwXfWarps = 8;
 constexpr int kBwEpWarps = 4;
 constexpr int kBwThreads = 64 + (kBwXfWarps + kBwEpWarps) * 32;
-constexpr int kBwOutRows = 16;               // tokens per dX TMA store (one warp)
-constexpr int kBwOutBox = kBwOutRows * 128;  // 2 KB
-constexpr int kBwNumOut = 4;                 // staging buffers per dX epilogue warp
 constexpr int kBwMaxItems = 2 * kBwXfWarps * 32;  // (box, token) items a stage may hold
 
 struct TcBwdParams {
   const uint8_t *wt;   // conj(What)^T tiles of the dX direction (one output tile)
+  __half *dx;          // [N][C][4]
   int64_t N;
   int C, D, Cs;        // Cs: workspace row stride
   int nqd, nqc;        // 16-channel boxes of dy and of x
   int slots;           // box slots per stage: max(8, nqd + nqc) (dW operand reads 8 d boxes)
   int CT;              // dW columns: 16 * nqc
   int BD;              // dX output tile (>= C)
-  int chunk_bytes;     // one dX weight chunk: 6 * BD rows x 32 B
+  int chunk_bytes;     // one dX weight chunk: 5 * BD rows x 32 B
   int wres_bytes;      // nqd * chunk_bytes, 1 KB aligned
   int stages;
   int splits;
@@ -68,15 +69,14 @@ struct TcBwdParams {
 };
 
 struct BwSmem {
-  int wres, stage0, out0, bars, total;
+  int wres, stage0, bars, total;
 };
 
 __host__ __device__ inline BwSmem tc_bwd_smem(const TcBwdParams &p) {
   BwSmem s;
   s.wres = 0;
   s.stage0 = p.wres_bytes;
-  s.out0 = s.stage0 + p.stages * p.slots * kBwBox;
-  s.bars = s.out0 + kBwEpWarps * kBwNumOut * kBwOutBox;
+  s.bars = s.stage0 + p.stages * p.slots * kBwBox;
   // full, tready, empty per stage; dxfull, dxempty x2; dwfull; wfull; tmem slot
   s.total = s.bars + (3 * p.stages + 4 + 2) * 8 + 16;
   return s;
@@ -86,7 +86,7 @@ __host__ __device__ inline BwSmem tc_bwd_smem(const TcBwdParams &p) {
 // 4 x 32 x 128 = 16,384.
 __global__ void __maxnreg__(128)
 tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
-              const __grid_constant__ CUtensorMap tm_dx, const TcBwdParams p) {
+              const TcBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -139,7 +139,6 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     if (lane == 0) {
       tma_prefetch_desc(&tm_dy);
       tma_prefetch_desc(&tm_x);
-      tma_prefetch_desc(&tm_dx);
       if (nst > 0) {
         mbar_arrive_expect_tx(wfull, p.nqd * p.chunk_bytes);
         bulk_load(smem + L.wres, p.wt, p.nqd * p.chunk_bytes, wfull);
@@ -215,7 +214,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         tc_fence_after();
         if (ok) {
           const uint32_t acc = tmem_base + dx0 + b * 4 * p.BD;
-          const uint32_t w1 = p.BD * 32, w2 = 2 * p.BD * 32, w4 = 4 * p.BD * 32;
+          const uint32_t w1 = p.BD * 32, w2 = 2 * p.BD * 32, w3 = 3 * p.BD * 32;
           for (int q = 0; q < p.nqd; ++q) {
             const uint32_t box = st + q * kBwBox;
             const uint32_t wq = wres + q * p.chunk_bytes;
@@ -224,7 +223,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
             mma_f16_ss(acc + p.BD, desc_at(dk, box + kBwPlane), desc_at(dk, wq + w1), id_x1, in);
             mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 2 * kBwPlane), desc_at(dk, wq + w2),
                        id_x2, in);
-            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 3 * kBwPlane), desc_at(dk, wq + w4),
+            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 3 * kBwPlane), desc_at(dk, wq + w3),
                        id_x2, 1u);
           }
           mma_commit(&dxfull[b]);
@@ -336,22 +335,25 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
   } else {
     // ------------------------------------------------------- dX epilogue
     const int quad = warp & 3;
-    const int ew = warp - 2 - kBwXfWarps;
-    uint8_t *obase = smem + L.out0 + ew * kBwNumOut * kBwOutBox;
     const int groups = p.BD / 16;
-    int oi = 0;
+    const int64_t row_elems = static_cast<int64_t>(p.C) * kT;
     for (int ch = 0; ch < nst; ++ch) {
       const int b = ch % p.ndx;
       if (ok) ok = mbar_wait(&dxfull[b], (ch / p.ndx) & 1);
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + dx0 + b * 4 * p.BD;
-      const int64_t tok0 = t_begin + static_cast<int64_t>(ch) * kBwTB + quad * kBwOutRows;
+      // lanes 0..15 hold this warp's 16 tokens
+      const int64_t n = t_begin + static_cast<int64_t>(ch) * kBwTB + quad * 16 + lane;
+      const bool row_ok = lane < 16 && n < t_end;
+      __half *drow = p.dx + n * row_elems;
       for (int g = 0; g < groups; ++g) {
-        uint32_t packed[32];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t y0[8], y2[8], y1r[8], y1i[8];
           const uint32_t col = tl + g * 16 + h * 8;
+          // the TMEM loads are warp-collective: reconverge after the wait and the
+          // per-lane stores of the previous step
+          __syncwarp();
           tmem_ld8(col, y0);
           tmem_ld8(col + p.BD, y2);
           tmem_ld8(col + 2 * p.BD, y1r);
@@ -362,36 +364,27 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
           }
+          uint32_t packed[16];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
             const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
             const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
-            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+            packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+            packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+          }
+          // C is even, so channels go out in 16-byte pairs
+          const int c0 = g * 16 + h * 8;
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (c0 + 2 * j + 2 <= p.C)
+                *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
+                    packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
           }
         }
-        if (g * 16 >= p.C) continue;  // whole group is padding
-        uint8_t *ob = obase + (oi % kBwNumOut) * kBwOutBox;
-        if (lane == 0) bulk_wait_read<kBwNumOut - 1>();
-        __syncwarp();
-        if (lane < kBwOutRows) {  // lanes 0..15 hold this warp's 16 tokens
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<uint4 *>(ob + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
-                           packed[4 * q + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_dx, g * 16 * kT, static_cast<int32_t>(tok0), ob);
-          bulk_commit();
-        }
-        ++oi;
       }
     }
-    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();

@@ -24,6 +24,8 @@
 //   acc[0, BD)    += X0  * What0^T                (N = BD)
 //   acc[BD, 2BD)  += X2  * What2^T                (N = BD)
 //   acc[2BD, 4BD) += ReX1 * (Re1 ; Im1)^T + (-ImX1) * (Im1 ; -Re1)^T   (N = 2 BD)
+// (the weight chunk stores What0, What2, Re1, Im1, -Re1; the two N = 2 BD
+// operands are overlapping windows of its last three planes)
 // so columns [2BD, 3BD) hold Re Y1 and [3BD, 4BD) hold Im Y1.  When 4*BD <= 256
 // the accumulators are double-buffered in TMEM so the epilogue of one tile
 // overlaps the MMAs of the next.
@@ -211,7 +213,7 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
             mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 2 * kPlaneBytes),
                        desc_at(dsw32, ws + 2 * p.BD * wrow), id_2bd, acc_in);
             mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 3 * kPlaneBytes),
-                       desc_at(dsw32, ws + 4 * p.BD * wrow), id_2bd, 1u);
+                       desc_at(dsw32, ws + 3 * p.BD * wrow), id_2bd, 1u);
             mma_commit(&empty[s]);
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }

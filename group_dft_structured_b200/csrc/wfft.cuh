@@ -45,19 +45,14 @@ __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict
     const int dir = e < n_fwd ? 0 : 1;
     const TcPlan &P = dir == 0 ? L.fwd : L.dx;
     const int64_t le = dir == 0 ? e : e - n_fwd;
-    const int rows = 6 * P.BD;
+    const int rows = 5 * P.BD;
     const int64_t chunk = le / (rows * kCK);
     const int rem = static_cast<int>(le % (rows * kCK));
     const int row = rem / kCK, k = rem % kCK;
     const int j = static_cast<int>(chunk / P.nK), kc = static_cast<int>(chunk % P.nK);
-    // which bin, which output channel
-    int sub, r;
-    if (row < P.BD) { sub = 0; r = row; }
-    else if (row < 2 * P.BD) { sub = 1; r = row - P.BD; }
-    else if (row < 4 * P.BD) { sub = 2; r = row - 2 * P.BD; }
-    else { sub = 3; r = row - 4 * P.BD; }
-    const bool hi = r >= P.BD;
-    const int o = j * P.BD + (hi ? r - P.BD : r);
+    // which plane (What0, What2, Re1, Im1, -Re1), which output channel
+    const int sub = row / P.BD;
+    const int o = j * P.BD + row % P.BD;
     const int i = kc * kCK + k;
     float v = 0.f;
     if (o < P.Do && i < P.Ci) {
@@ -65,8 +60,9 @@ __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict
       weight_bins(W, C, dir, o, i, b0, b2, b1r, b1i);
       if (sub == 0) v = b0;
       else if (sub == 1) v = b2;
-      else if (sub == 2) v = hi ? b1i : b1r;    // rows (Re1 ; Im1): multiply Re X1
-      else v = hi ? -b1r : b1i;                 // rows (Im1 ; -Re1): multiply -Im X1
+      else if (sub == 2) v = b1r;
+      else if (sub == 3) v = b1i;
+      else v = -b1r;
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);

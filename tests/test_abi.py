@@ -66,7 +66,7 @@ def _tc_plan(Ci, Do):
     nK = -(-Ci // 16)
     nD = -(-Do // (64 if nK <= 4 else 128))
     BD = -(-(-(-Do // nD)) // 16) * 16
-    return nD, BD, nK, nD * nK * 6 * BD * 16 * 2
+    return nD, BD, nK, nD * nK * 5 * BD * 16 * 2
 
 
 @pytest.mark.parametrize("C,D", [(16, 16), (48, 192), (192, 192), (256, 256), (24, 96), (6, 40)])
