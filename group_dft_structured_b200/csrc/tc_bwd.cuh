@@ -185,16 +185,19 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         if (ok) ok = mbar_wait(&tready[s], ph);
         tc_fence_after();
         const uint32_t st = stage_base + s * p.slots * kBwBox;
+        // every operand below is one of these bases plus a 16-byte-unit offset
+        const uint64_t bmn = desc_at(dmn, st), bmx = desc_at(dmx, st + p.nqd * kBwBox);
+        const uint64_t bk = desc_at(dk, st);
         if (ok) {
+          const uint64_t xb16 = (p.nqc * kBwPlane) >> 4;  // one x bin
 #pragma unroll
           for (int k = 0; k < kBwTB / 16; ++k) {
-            // dy planes: d chunks 8 KB apart; x planes: plane-major, c chunks 2 KB apart
-            const uint32_t a = st + k * 512, b = st + p.nqd * kBwBox + k * 512;  // 16 tokens
-            const uint32_t xb = p.nqc * kBwPlane;  // one x bin
-            const uint64_t A0 = desc_at(dmn, a), A1 = desc_at(dmn, a + kBwPlane);
-            const uint64_t A2 = desc_at(dmn, a + 2 * kBwPlane), A3 = desc_at(dmn, a + 3 * kBwPlane);
-            const uint64_t B0 = desc_at(dmx, b), B1 = desc_at(dmx, b + xb);
-            const uint64_t B2 = desc_at(dmx, b + 2 * xb), B3 = desc_at(dmx, b + 3 * xb);
+            // dy planes: d chunks 8 KB apart; x planes: plane-major, c chunks 2 KB apart;
+            // 16 tokens = 512 B
+            const uint64_t A0 = bmn + k * 32, A1 = A0 + (kBwPlane >> 4);
+            const uint64_t A2 = A0 + 2 * (kBwPlane >> 4), A3 = A0 + 3 * (kBwPlane >> 4);
+            const uint64_t B0 = bmx + k * 32, B1 = B0 + xb16;
+            const uint64_t B2 = B1 + xb16, B3 = B2 + xb16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
             mma_f16_ss(acc0, A0, B0, id_w, first);
             mma_f16_ss(acc2, A1, B1, id_w, first);
@@ -214,17 +217,14 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         tc_fence_after();
         if (ok) {
           const uint32_t acc = tmem_base + dx0 + b * 4 * p.BD;
-          const uint32_t w1 = p.BD * 32, w2 = 2 * p.BD * 32, w3 = 3 * p.BD * 32;
-          for (int q = 0; q < p.nqd; ++q) {
-            const uint32_t box = st + q * kBwBox;
-            const uint32_t wq = wres + q * p.chunk_bytes;
+          const uint64_t w1 = (p.BD * 32) >> 4, chunk16 = p.chunk_bytes >> 4;
+          uint64_t ab = bk, wb = desc_at(dk, wres);  // running box and weight-chunk descriptors
+          for (int q = 0; q < p.nqd; ++q, ab += kBwBox >> 4, wb += chunk16) {
             const uint32_t in = q > 0 ? 1u : 0u;
-            mma_f16_ss(acc, desc_at(dk, box), desc_at(dk, wq), id_x1, in);
-            mma_f16_ss(acc + p.BD, desc_at(dk, box + kBwPlane), desc_at(dk, wq + w1), id_x1, in);
-            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 2 * kBwPlane), desc_at(dk, wq + w2),
-                       id_x2, in);
-            mma_f16_ss(acc + 2 * p.BD, desc_at(dk, box + 3 * kBwPlane), desc_at(dk, wq + w3),
-                       id_x2, 1u);
+            mma_f16_ss(acc, ab, wb, id_x1, in);
+            mma_f16_ss(acc + p.BD, ab + (kBwPlane >> 4), wb + w1, id_x1, in);
+            mma_f16_ss(acc + 2 * p.BD, ab + 2 * (kBwPlane >> 4), wb + 2 * w1, id_x2, in);
+            mma_f16_ss(acc + 2 * p.BD, ab + 3 * (kBwPlane >> 4), wb + 3 * w1, id_x2, 1u);
           }
           mma_commit(&dxfull[b]);
           mma_commit(&empty[s]);

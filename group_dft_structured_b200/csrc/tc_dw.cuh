@@ -207,12 +207,14 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
         tc_fence_after();
         if (ok) {
           const uint32_t pl = plane_base + pb * p.plane_bytes;
+          // every operand is one of two base descriptors plus a 16-byte-unit offset
+          const uint64_t ba = desc_at(dmn, pl), bb = desc_at(dmn, pl + x_off);
+          const uint64_t a16 = a_bin >> 4, b16 = b_bin >> 4;
           for (int k = 0; k < p.TB / 16; ++k) {
-            const uint32_t a = pl + k * 512, b = pl + x_off + k * 512;  // 16 tokens x 32 B
-            const uint64_t A0 = desc_at(dmn, a), A1 = desc_at(dmn, a + a_bin);
-            const uint64_t A2 = desc_at(dmn, a + 2 * a_bin), A3 = desc_at(dmn, a + 3 * a_bin);
-            const uint64_t B0 = desc_at(dmn, b), B1 = desc_at(dmn, b + b_bin);
-            const uint64_t B2 = desc_at(dmn, b + 2 * b_bin), B3 = desc_at(dmn, b + 3 * b_bin);
+            const uint64_t A0 = ba + k * 32, A1 = A0 + a16;  // 16 tokens x 32 B = 512 B
+            const uint64_t A2 = A1 + a16, A3 = A2 + a16;
+            const uint64_t B0 = bb + k * 32, B1 = B0 + b16;
+            const uint64_t B2 = B1 + b16, B3 = B2 + b16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
             mma_f16_ss(acc0, A0, B0, id, first);
             mma_f16_ss(acc2, A1, B1, id, first);

@@ -193,32 +193,35 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       if (p.resident && tc_unit(p, 0, m, j)) ok = mbar_wait(wfull, 0);
       int s = 0;
       uint32_t ph = 0;
+      // every operand is a chunk's base descriptor plus a 16-byte-unit offset
+      const uint64_t pl16 = kPlaneBytes >> 4, w16 = (p.BD * wrow) >> 4;
+      const uint64_t stage16 = p.stage_bytes >> 4, chunk16 = p.chunk_bytes >> 4;
+      const uint64_t x0 = desc_at(dsw32, stage_base), wr0 = desc_at(dsw32, wres_base);
+      int a = 0;        // accumulator buffer of this unit
+      uint32_t aph = 0;  // its phase
       for (int it = 0; tc_unit(p, it, m, j); ++it) {
-        const int a = it % p.nacc;
-        const uint32_t aph = (it / p.nacc) & 1;
         if (ok) ok = mbar_wait(&acc_empty[a], aph ^ 1);
         tc_fence_after();
         const uint32_t acc = tmem_base + a * p.acc_stride;
-        for (int kc = 0; kc < p.nK; ++kc) {
+        uint64_t wr = wr0;
+        for (int kc = 0; kc < p.nK; ++kc, wr += chunk16) {
           if (ok) ok = mbar_wait(&full[s], ph);
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
-            const uint32_t xs = stage_base + s * p.stage_bytes;
-            const uint32_t ws = p.resident ? wres_base + kc * p.chunk_bytes : xs + kXChunkBytes;
+            const uint64_t xd = x0 + s * stage16;
+            const uint64_t wd = p.resident ? wr : xd + (kXChunkBytes >> 4);
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
-            mma_f16_ss(acc, desc_at(dsw32, xs), desc_at(dsw32, ws), id_bd, acc_in);
-            mma_f16_ss(acc + p.BD, desc_at(dsw32, xs + kPlaneBytes),
-                       desc_at(dsw32, ws + p.BD * wrow), id_bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 2 * kPlaneBytes),
-                       desc_at(dsw32, ws + 2 * p.BD * wrow), id_2bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, desc_at(dsw32, xs + 3 * kPlaneBytes),
-                       desc_at(dsw32, ws + 3 * p.BD * wrow), id_2bd, 1u);
+            mma_f16_ss(acc, xd, wd, id_bd, acc_in);
+            mma_f16_ss(acc + p.BD, xd + pl16, wd + w16, id_bd, acc_in);
+            mma_f16_ss(acc + 2 * p.BD, xd + 2 * pl16, wd + 2 * w16, id_2bd, acc_in);
+            mma_f16_ss(acc + 2 * p.BD, xd + 3 * pl16, wd + 3 * w16, id_2bd, 1u);
             mma_commit(&empty[s]);
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }
         }
         if (ok) mma_commit(&acc_full[a]);
+        if (++a == p.nacc) { a = 0; aph ^= 1; }
       }
       // all MMAs (and hence all loads they consumed) complete before exit
       mma_commit(final_bar);
