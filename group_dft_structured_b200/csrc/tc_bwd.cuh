@@ -178,6 +178,10 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const uint64_t dmn = smem_desc(0, kBwBox, 256, kSw32);    // dy planes read column-wise (dW)
       const uint64_t dmx = smem_desc(0, kBwPlane, 256, kSw32);  // x planes read column-wise (dW)
       const uint64_t dk = smem_desc(0, 16, 256, kSw32);       // K-major rows (dX, weights)
+      const uint32_t dhi = desc_hi(dk);  // same for dmn and dmx: only the low words differ
+      const uint32_t xb16 = (p.nqc * kBwPlane) >> 4;  // one x bin
+      const uint32_t wl = desc_lo(desc_at(dk, wres)), chunk16 = p.chunk_bytes >> 4;
+      const uint32_t w1 = (p.BD * 32) >> 4;
       int s = 0;
       uint32_t ph = 0;
       for (int ch = 0; ch < nst; ++ch) {
@@ -185,30 +189,30 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         if (ok) ok = mbar_wait(&tready[s], ph);
         tc_fence_after();
         const uint32_t st = stage_base + s * p.slots * kBwBox;
-        // every operand below is one of these bases plus a 16-byte-unit offset
-        const uint64_t bmn = desc_at(dmn, st), bmx = desc_at(dmx, st + p.nqd * kBwBox);
-        const uint64_t bk = desc_at(dk, st);
+        // every operand below is the low descriptor word of one of these bases plus a
+        // 16-byte-unit offset (the high words are all dhi)
+        const uint32_t mn = desc_lo(desc_at(dmn, st)), mx = desc_lo(desc_at(dmx, st + p.nqd * kBwBox));
+        const uint32_t kl = desc_lo(desc_at(dk, st));
         if (ok) {
-          const uint64_t xb16 = (p.nqc * kBwPlane) >> 4;  // one x bin
 #pragma unroll
           for (int k = 0; k < kBwTB / 16; ++k) {
             // dy planes: d chunks 8 KB apart; x planes: plane-major, c chunks 2 KB apart;
             // 16 tokens = 512 B
-            const uint64_t A0 = bmn + k * 32, A1 = A0 + (kBwPlane >> 4);
-            const uint64_t A2 = A0 + 2 * (kBwPlane >> 4), A3 = A0 + 3 * (kBwPlane >> 4);
-            const uint64_t B0 = bmx + k * 32, B1 = B0 + xb16;
-            const uint64_t B2 = B1 + xb16, B3 = B2 + xb16;
+            const uint32_t A0 = mn + k * 32, A1 = A0 + (kBwPlane >> 4);
+            const uint32_t A2 = A0 + 2 * (kBwPlane >> 4), A3 = A0 + 3 * (kBwPlane >> 4);
+            const uint32_t B0 = mx + k * 32, B1 = B0 + xb16;
+            const uint32_t B2 = B1 + xb16, B3 = B2 + xb16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
-            mma_f16_ss(acc0, A0, B0, id_w, first);
-            mma_f16_ss(acc2, A1, B1, id_w, first);
+            mma_f16_lo(acc0, A0, B0, dhi, id_w, first);
+            mma_f16_lo(acc2, A1, B1, dhi, id_w, first);
             if (p.merged) {  // see tc_dw.cuh: acc_a, acc_b over [Re X1 | -Im X1]
-              mma_f16_ss(acca, A2, B2, id_w2, first);
-              mma_f16_ss(accb, A3, B2, id_w2, first);
+              mma_f16_lo(acca, A2, B2, dhi, id_w2, first);
+              mma_f16_lo(accb, A3, B2, dhi, id_w2, first);
             } else {
-              mma_f16_ss(acc1r, A2, B2, id_w, first);
-              mma_f16_ss(acc1r, A3, B3, id_w, 1u);
-              mma_f16_ss(acc1i, A3, B2, id_wneg, first);
-              mma_f16_ss(acc1i, A2, B3, id_w, 1u);
+              mma_f16_lo(acc1r, A2, B2, dhi, id_w, first);
+              mma_f16_lo(acc1r, A3, B3, dhi, id_w, 1u);
+              mma_f16_lo(acc1i, A3, B2, dhi, id_wneg, first);
+              mma_f16_lo(acc1i, A2, B3, dhi, id_w, 1u);
             }
           }
         }
@@ -217,14 +221,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         tc_fence_after();
         if (ok) {
           const uint32_t acc = tmem_base + dx0 + b * 4 * p.BD;
-          const uint64_t w1 = (p.BD * 32) >> 4, chunk16 = p.chunk_bytes >> 4;
-          uint64_t ab = bk, wb = desc_at(dk, wres);  // running box and weight-chunk descriptors
+          uint32_t ab = kl, wb = wl;  // running box and weight-chunk descriptor words
           for (int q = 0; q < p.nqd; ++q, ab += kBwBox >> 4, wb += chunk16) {
             const uint32_t in = q > 0 ? 1u : 0u;
-            mma_f16_ss(acc, ab, wb, id_x1, in);
-            mma_f16_ss(acc + p.BD, ab + (kBwPlane >> 4), wb + w1, id_x1, in);
-            mma_f16_ss(acc + 2 * p.BD, ab + 2 * (kBwPlane >> 4), wb + 2 * w1, id_x2, in);
-            mma_f16_ss(acc + 2 * p.BD, ab + 3 * (kBwPlane >> 4), wb + 3 * w1, id_x2, 1u);
+            mma_f16_lo(acc, ab, wb, dhi, id_x1, in);
+            mma_f16_lo(acc + p.BD, ab + (kBwPlane >> 4), wb + w1, dhi, id_x1, in);
+            mma_f16_lo(acc + 2 * p.BD, ab + 2 * (kBwPlane >> 4), wb + 2 * w1, dhi, id_x2, in);
+            mma_f16_lo(acc + 2 * p.BD, ab + 3 * (kBwPlane >> 4), wb + 3 * w1, dhi, id_x2, 1u);
           }
           mma_commit(&dxfull[b]);
           mma_commit(&empty[s]);

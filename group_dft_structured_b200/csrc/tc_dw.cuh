@@ -196,6 +196,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
       const uint32_t id_neg = instr_desc(kDwMT, p.CT, 0, 0, 1, 1, 1);
       const uint32_t id2 = instr_desc(kDwMT, 2 * p.CT, 0, 0, 1, 1);
       const uint64_t dmn = smem_desc(0, chunk_plane, 256, kSw32);  // MN-major planes
+      const uint32_t dhi = desc_hi(dmn);
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
       const uint32_t acca = tmem_base + 2 * p.CT, accb = tmem_base + 4 * p.CT;
@@ -207,25 +208,26 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
         tc_fence_after();
         if (ok) {
           const uint32_t pl = plane_base + pb * p.plane_bytes;
-          // every operand is one of two base descriptors plus a 16-byte-unit offset
-          const uint64_t ba = desc_at(dmn, pl), bb = desc_at(dmn, pl + x_off);
-          const uint64_t a16 = a_bin >> 4, b16 = b_bin >> 4;
+          // every operand is the low descriptor word of one of two bases plus a
+          // 16-byte-unit offset; the high word is common
+          const uint32_t ba = desc_lo(desc_at(dmn, pl)), bb = desc_lo(desc_at(dmn, pl + x_off));
+          const uint32_t a16 = a_bin >> 4, b16 = b_bin >> 4;
           for (int k = 0; k < p.TB / 16; ++k) {
-            const uint64_t A0 = ba + k * 32, A1 = A0 + a16;  // 16 tokens x 32 B = 512 B
-            const uint64_t A2 = A1 + a16, A3 = A2 + a16;
-            const uint64_t B0 = bb + k * 32, B1 = B0 + b16;
-            const uint64_t B2 = B1 + b16, B3 = B2 + b16;
+            const uint32_t A0 = ba + k * 32, A1 = A0 + a16;  // 16 tokens x 32 B = 512 B
+            const uint32_t A2 = A1 + a16, A3 = A2 + a16;
+            const uint32_t B0 = bb + k * 32, B1 = B0 + b16;
+            const uint32_t B2 = B1 + b16, B3 = B2 + b16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
-            mma_f16_ss(acc0, A0, B0, id, first);
-            mma_f16_ss(acc2, A1, B1, id, first);
+            mma_f16_lo(acc0, A0, B0, dhi, id, first);
+            mma_f16_lo(acc2, A1, B1, dhi, id, first);
             if (p.merged) {
-              mma_f16_ss(acca, A2, B2, id2, first);
-              mma_f16_ss(accb, A3, B2, id2, first);
+              mma_f16_lo(acca, A2, B2, dhi, id2, first);
+              mma_f16_lo(accb, A3, B2, dhi, id2, first);
             } else {
-              mma_f16_ss(acc1r, A2, B2, id, first);
-              mma_f16_ss(acc1r, A3, B3, id, 1u);
-              mma_f16_ss(acc1i, A3, B2, id_neg, first);
-              mma_f16_ss(acc1i, A2, B3, id, 1u);
+              mma_f16_lo(acc1r, A2, B2, dhi, id, first);
+              mma_f16_lo(acc1r, A3, B3, dhi, id, 1u);
+              mma_f16_lo(acc1i, A3, B2, dhi, id_neg, first);
+              mma_f16_lo(acc1i, A2, B3, dhi, id, 1u);
             }
           }
           mma_commit(&pempty[pb]);

@@ -193,29 +193,32 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       if (p.resident && tc_unit(p, 0, m, j)) ok = mbar_wait(wfull, 0);
       int s = 0;
       uint32_t ph = 0;
-      // every operand is a chunk's base descriptor plus a 16-byte-unit offset
-      const uint64_t pl16 = kPlaneBytes >> 4, w16 = (p.BD * wrow) >> 4;
-      const uint64_t stage16 = p.stage_bytes >> 4, chunk16 = p.chunk_bytes >> 4;
-      const uint64_t x0 = desc_at(dsw32, stage_base), wr0 = desc_at(dsw32, wres_base);
+      // every operand is the low descriptor word of a chunk's base plus a 16-byte-unit
+      // offset; the high word is common
+      const uint32_t dhi = desc_hi(dsw32);
+      const uint32_t pl16 = kPlaneBytes >> 4, w16 = (p.BD * wrow) >> 4;
+      const uint32_t stage16 = p.stage_bytes >> 4, chunk16 = p.chunk_bytes >> 4;
+      const uint32_t x0 = desc_lo(desc_at(dsw32, stage_base));
+      const uint32_t wr0 = desc_lo(desc_at(dsw32, wres_base));
       int a = 0;        // accumulator buffer of this unit
       uint32_t aph = 0;  // its phase
       for (int it = 0; tc_unit(p, it, m, j); ++it) {
         if (ok) ok = mbar_wait(&acc_empty[a], aph ^ 1);
         tc_fence_after();
         const uint32_t acc = tmem_base + a * p.acc_stride;
-        uint64_t wr = wr0;
+        uint32_t wr = wr0;
         for (int kc = 0; kc < p.nK; ++kc, wr += chunk16) {
           if (ok) ok = mbar_wait(&full[s], ph);
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
-            const uint64_t xd = x0 + s * stage16;
-            const uint64_t wd = p.resident ? wr : xd + (kXChunkBytes >> 4);
+            const uint32_t xd = x0 + s * stage16;
+            const uint32_t wd = p.resident ? wr : xd + (kXChunkBytes >> 4);
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
-            mma_f16_ss(acc, xd, wd, id_bd, acc_in);
-            mma_f16_ss(acc + p.BD, xd + pl16, wd + w16, id_bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, xd + 2 * pl16, wd + 2 * w16, id_2bd, acc_in);
-            mma_f16_ss(acc + 2 * p.BD, xd + 3 * pl16, wd + 3 * w16, id_2bd, 1u);
+            mma_f16_lo(acc, xd, wd, dhi, id_bd, acc_in);
+            mma_f16_lo(acc + p.BD, xd + pl16, wd + w16, dhi, id_bd, acc_in);
+            mma_f16_lo(acc + 2 * p.BD, xd + 2 * pl16, wd + 2 * w16, dhi, id_2bd, acc_in);
+            mma_f16_lo(acc + 2 * p.BD, xd + 3 * pl16, wd + 3 * w16, dhi, id_2bd, 1u);
             mma_commit(&empty[s]);
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }
