@@ -56,6 +56,12 @@ _SIGNATURES = {
     "feql_backward_dw": (_I, [_VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
     "feql_backward": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
     "feql_backward_dw_noalloc": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
+    "feql_ct_weight_fft_bytes": (_SZ, [_I, _I, _I, _I]),
+    "feql_ct_weight_fft": (_I, [_I, _VP, _VP, _I, _I, _I, _VP]),
+    "feql_ct_forward": (_I, [_I, _VP, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
+    "feql_ct_backward_dx": (_I, [_I, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
+    "feql_ct_backward_dw_workspace_bytes": (_SZ, [_I, _I64, _I, _I, _I]),
+    "feql_ct_backward_dw": (_I, [_I, _VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
     "feql_device_status": (_I, [_VP]),
     "feql_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -146,6 +152,38 @@ def feql_backward_dw_noalloc(x, dy, dW, db, N: int, C: int, D: int, dtype: int,
     (see include/feql.h for the size limit and the no-overlap rule)."""
     _check(load().feql_backward_dw_noalloc(_ptr(x), _ptr(dy), _ptr(dW), _ptr(db), N, C, D,
                                            dtype, _stream(stream)), "feql_backward_dw_noalloc")
+
+
+def feql_ct_weight_fft_bytes(T: int, C: int, D: int, dtype: int) -> int:
+    return int(load().feql_ct_weight_fft_bytes(T, C, D, dtype))
+
+
+def feql_ct_weight_fft(T: int, W, What, C: int, D: int, dtype: int, stream=None) -> None:
+    _check(load().feql_ct_weight_fft(T, _ptr(W), _ptr(What), C, D, dtype, _stream(stream)),
+           "feql_ct_weight_fft")
+
+
+def feql_ct_forward(T: int, x, What, b, y, N: int, C: int, D: int, dtype: int,
+                    stream=None) -> None:
+    _check(load().feql_ct_forward(T, _ptr(x), _ptr(What), _ptr(b), _ptr(y), N, C, D, dtype,
+                                  _stream(stream)), "feql_ct_forward")
+
+
+def feql_ct_backward_dx(T: int, dy, What, dx, N: int, C: int, D: int, dtype: int,
+                        stream=None) -> None:
+    _check(load().feql_ct_backward_dx(T, _ptr(dy), _ptr(What), _ptr(dx), N, C, D, dtype,
+                                      _stream(stream)), "feql_ct_backward_dx")
+
+
+def feql_ct_backward_dw_workspace_bytes(T: int, N: int, C: int, D: int, dtype: int) -> int:
+    return int(load().feql_ct_backward_dw_workspace_bytes(T, N, C, D, dtype))
+
+
+def feql_ct_backward_dw(T: int, x, dy, dW, db, ws, ws_bytes: int, N: int, C: int, D: int,
+                        dtype: int, stream=None) -> None:
+    _check(load().feql_ct_backward_dw(T, _ptr(x), _ptr(dy), _ptr(dW), _ptr(db), _ptr(ws),
+                                      ws_bytes, N, C, D, dtype, _stream(stream)),
+           "feql_ct_backward_dw")
 
 
 def feql_device_status(stream=None) -> int:

@@ -8,7 +8,9 @@ from __future__ import annotations
 import torch
 
 from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward, feql_backward_dw,
-               feql_backward_dw_workspace_bytes, feql_backward_dx, feql_forward, feql_weight_fft,
+               feql_backward_dw_workspace_bytes, feql_backward_dx, feql_ct_backward_dw,
+               feql_ct_backward_dw_workspace_bytes, feql_ct_backward_dx, feql_ct_forward,
+               feql_ct_weight_fft, feql_ct_weight_fft_bytes, feql_forward, feql_weight_fft,
                feql_weight_fft_bytes)
 
 
@@ -73,4 +75,43 @@ def backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, ws=None, out=None,
     else:
         dW, db = out
     feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
+    return dW, db
+
+
+# --------------------------------------------------------- cyclic group C_T
+# The group order T is the length of the last axis (T = 4 goes to the p4 path).
+
+def ct_weight_fft(W: torch.Tensor, mode: int, stream=None) -> torch.Tensor:
+    D, C, T = W.shape
+    nbytes = feql_ct_weight_fft_bytes(T, C, D, mode)
+    if nbytes == 0:
+        raise ValueError("unsupported (T, C, D, mode)")
+    What = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    feql_ct_weight_fft(T, W, What, C, D, mode, stream)
+    return What
+
+
+def ct_forward(x: torch.Tensor, What: torch.Tensor, b, D: int, mode: int, stream=None):
+    N, C, T = x.shape
+    y = torch.empty((N, D, T), dtype=x.dtype, device=x.device)
+    feql_ct_forward(T, x, What, b, y, N, C, D, mode, stream)
+    return y
+
+
+def ct_backward_dx(dy: torch.Tensor, What: torch.Tensor, C: int, mode: int, stream=None):
+    N, D, T = dy.shape
+    dx = torch.empty((N, C, T), dtype=dy.dtype, device=dy.device)
+    feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, stream)
+    return dx
+
+
+def ct_backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, with_db: bool = True,
+                   stream=None):
+    N, C, T = x.shape
+    D = dy.shape[1]
+    nbytes = feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    dW = torch.empty((D, C, T), dtype=x.dtype, device=x.device)
+    db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
+    feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
     return dW, db

@@ -1,17 +1,17 @@
-"""Workload shapes and seeded synthetic inputs for the p4 EQ-Linear layer.
+"""Workload shapes and seeded synthetic inputs for the EQ-Linear layer (p4 and C_8).
 
 This module holds no arithmetic of the method: it only draws random numbers
 and rounds them to the compute dtype.  Both the CUDA path (through the tests
 and the benchmark) and the float64 oracle consume exactly the rounded arrays
 produced here.
 
-Recipe.  Layout x[N,C,4], W[D,C,4], b[D], dy[N,D,4] (group index innermost).
-Values are drawn in float64 with numpy's PCG64 generator and rounded
-(round-to-nearest-even) to the mode dtype:
+Recipe.  Layout x[N,C,T], W[D,C,T], b[D], dy[N,D,T] (group index innermost,
+T = 4 for p4, 8 for the cyclic group C_8).  Values are drawn in float64 with
+numpy's PCG64 generator and rounded (round-to-nearest-even) to the mode dtype:
 
 * x, dy ~ N(0, 1)
-* W ~ N(0, variance 1/(4C)), i.e. std 1/(2 sqrt C): the fan-in of the
-  unrolled 4C-wide layer, so that Var(y) is about 1
+* W ~ N(0, variance 1/(T C)), i.e. std 1/sqrt(T C): the fan-in of the
+  unrolled TC-wide layer, so that Var(y) is about 1 (1/(2 sqrt C) for p4)
 * b ~ N(0, std 0.02)
 
 Seeds: 20260000 + 100 * workload_id + {x: 0, W: 1, b: 2, dy: 3}.
@@ -19,7 +19,8 @@ Seeds: 20260000 + 100 * workload_id + {x: 0, W: 1, b: 2, dy: 3}.
 The shapes stand in for the token streams of the networks the paper
 evaluates (Flash EQ-ViT and Flash EQ-Swin, technical summary "Livello di
 Rete"): a ViT MLP fc1 at 64 x 197 tokens and a Swin stage-1 stream at
-128 x 3136 tokens; no dataset is involved.
+128 x 3136 tokens; no dataset is involved.  The C_8 workload keeps the Swin
+stream's token count and unrolled widths (96 -> 384) with T = 8.
 """
 
 from __future__ import annotations
@@ -27,8 +28,6 @@ from __future__ import annotations
 from dataclasses import dataclass
 
 import numpy as np
-
-T = 4
 
 
 @dataclass(frozen=True)
@@ -41,6 +40,7 @@ class Workload:
     dtype: str          # "fp16" or "fp32"
     passes: tuple       # subset of ("fwd", "dx", "dw")
     note: str
+    T: int = 4          # group order
 
 
 WORKLOADS = {
@@ -55,6 +55,9 @@ WORKLOADS = {
     5: Workload(5, "p4_fwdbwd_fp16_swin_N401408_C24_D96", 401408, 24, 96, "fp16",
                 ("fwd", "dx", "dw"),
                 "Swin stage-1-like forward+backward, 128x3136 tokens (96->384 unrolled)"),
+    6: Workload(6, "c8_fwdbwd_fp16_swin_N401408_C12_D48", 401408, 12, 48, "fp16",
+                ("fwd", "dx", "dw"),
+                "cyclic group C_8, Swin stage-1-like stream (96->384 unrolled)", T=8),
 }
 
 
@@ -71,7 +74,7 @@ def _normal(seed: int, shape, std: float, dtype: str) -> np.ndarray:
 
 
 def make_inputs(wid: int, N: int, C: int, D: int, dtype: str,
-                which=("x", "W", "b", "dy")) -> dict:
+                which=("x", "W", "b", "dy"), T: int = 4) -> dict:
     """Seeded, dtype-rounded inputs for a layer of the given shape.
 
     ``wid`` selects the seed block; any shape may be drawn with it (small
@@ -82,7 +85,7 @@ def make_inputs(wid: int, N: int, C: int, D: int, dtype: str,
     if "x" in which:
         out["x"] = _normal(base + 0, (N, C, T), 1.0, dtype)
     if "W" in which:
-        out["W"] = _normal(base + 1, (D, C, T), 1.0 / (2.0 * np.sqrt(C)), dtype)
+        out["W"] = _normal(base + 1, (D, C, T), 1.0 / np.sqrt(T * C), dtype)
     if "b" in which:
         out["b"] = _normal(base + 2, (D,), 0.02, dtype)
     if "dy" in which:
@@ -93,4 +96,4 @@ def make_inputs(wid: int, N: int, C: int, D: int, dtype: str,
 def workload_inputs(wid: int, dtype: str | None = None, N: int | None = None,
                     which=("x", "W", "b", "dy")) -> dict:
     w = WORKLOADS[wid]
-    return make_inputs(wid, w.N if N is None else N, w.C, w.D, dtype or w.dtype, which)
+    return make_inputs(wid, w.N if N is None else N, w.C, w.D, dtype or w.dtype, which, T=w.T)

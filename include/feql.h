@@ -147,6 +147,31 @@ int feql_backward(const void *x, const void *dy, const void *What, void *dx, voi
 int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW, void *db,
                              int64_t N, int C, int D, int dtype, feql_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * Cyclic group C_T of order T (Flash EQ-Linear, arXiv abstract: the method for
+ * a group of size T costs 2(T-1)/T^2 of the dense layer; the paper's kernels
+ * are for p4).  Tensors as above with the group axis of length T:
+ * x[N][C][T], y[N][D][T], W[D][C][T], dW[D][C][T]; b, db [D].
+ *   y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod T] x[n,c,s]
+ * T = 4 is the p4 layer: every call forwards to the function above with the
+ * same arguments (all modes).  T = 8: FEQL_FP16 only (kernels on the tensor
+ * cores: bins 0 and 4 real, 1..3 complex, 14 real products instead of 64);
+ * FEQL_FP32 modes return FEQL_ERR_UNSUPPORTED, and so does every other T.
+ * Any C, D >= 1 for T = 8 (the row of 8C or 8D fp16 values is always a
+ * multiple of 16 bytes).  Argument checks, N == 0, ownership, streams and
+ * errors are as for the p4 functions; the Fourier buffer of T = 8 has its own
+ * layout and size (feql_ct_weight_fft_bytes). */
+size_t feql_ct_weight_fft_bytes(int T, int C, int D, int dtype);
+int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype,
+                       feql_stream stream);
+int feql_ct_forward(int T, const void *x, const void *What, const void *b, void *y, int64_t N,
+                    int C, int D, int dtype, feql_stream stream);
+int feql_ct_backward_dx(int T, const void *dy, const void *What, void *dx, int64_t N, int C,
+                        int D, int dtype, feql_stream stream);
+size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int dtype);
+int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db, void *ws,
+                        size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word
  * of the current device: FEQL_OK, or FEQL_ERR_TIMEOUT when some kernel gave up
  * on a bounded wait since the last call (its outputs are then undefined). */
