@@ -11,6 +11,9 @@ no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+--workload selects another shape (workloads.py); workload 6 is the same stream
+for the cyclic group C_8 (feql_ct_* entry points, dX and dW as two passes).
+
 Multi-GPU (torchrun, one rank per GPU): every rank runs the full workload on
 its own tokens (weak scaling); the data-parallel weight gradient is summed
 with one NCCL all-reduce per step.  --impl reference times the float64 CPU
@@ -43,7 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
-                    help="workload id 1-5 (group_dft_structured_b200/workloads.py)")
+                    help="workload id 1-6 (group_dft_structured_b200/workloads.py; 6 is the "
+                         "cyclic group C_8)")
     ap.add_argument("--dtype", choices=["fp16", "fp32"], default=None,
                     help="override the workload's dtype (e.g. the fp32 run of the square layer)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -84,16 +88,23 @@ def max_over_ranks(value: float, device) -> float:
 
 def workload_bytes(w, elt):
     """Algorithmic HBM bytes per launch of each pass (inputs read once, outputs
-    written once; Fourier weights counted as their 4*D*C values)."""
-    N, C, D = w.N, w.C, w.D
-    x, y, what, b = 4 * N * C * elt, 4 * N * D * elt, 4 * D * C * elt, D * elt
+    written once; Fourier weights counted as their T*D*C real values)."""
+    N, C, D, T = w.N, w.C, w.D, w.T
+    x, y, what, b = T * N * C * elt, T * N * D * elt, T * D * C * elt, D * elt
     return {
-        "wfft": 4 * D * C * elt + what,
+        "wfft": T * D * C * elt + what,
         "fwd": x + what + b + y,
         "dx": y + what + x,
-        "dw": x + y + 4 * D * C * elt + b,
-        "bwd": x + y + what + x + 4 * D * C * elt + b,  # x, dy, What in; dx, dW, db out
+        "dw": x + y + T * D * C * elt + b,
+        "bwd": x + y + what + x + T * D * C * elt + b,  # x, dy, What in; dx, dW, db out
     }
+
+
+def layer_macs(w):
+    """Real MACs of one contraction pass with the Fourier method: (2T-2) NCD for
+    even T (bins 0 and T/2 real, the others complex), and of the unrolled
+    dense method: T^2 NCD."""
+    return (2 * w.T - 2) * w.N * w.C * w.D, w.T * w.T * w.N * w.C * w.D
 
 
 def kernel_source_hash():
@@ -175,8 +186,11 @@ def time_oracle(w, n_sample):
     import numpy as np
 
     from group_dft_structured_b200.workloads import make_inputs
-    from oracle import feql_oracle as O
-    inp = make_inputs(w.wid, n_sample, w.C, w.D, w.dtype)
+    if w.T == 4:
+        from oracle import feql_oracle as O
+    else:
+        from oracle import feql_ct_oracle as O
+    inp = make_inputs(w.wid, n_sample, w.C, w.D, w.dtype, T=w.T)
     f = {k: v.astype(np.float64) for k, v in inp.items()}
     t0 = time.perf_counter()
     if "fwd" in w.passes:
@@ -245,7 +259,6 @@ def main():
     import torch.distributed as dist
 
     import group_dft_structured_b200 as F
-    from group_dft_structured_b200 import layer as L
     from group_dft_structured_b200.workloads import WORKLOADS, make_inputs
 
     w = WORKLOADS[args.workload]
@@ -259,30 +272,32 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     F.load()
     mode = F.FEQL_FP16 if w.dtype == "fp16" else F.FEQL_FP32
-    N, C, D = w.N, w.C, w.D
+    N, C, D, T = w.N, w.C, w.D, w.T
     elt = 2 if w.dtype == "fp16" else 4
-    inp = make_inputs(rank_seed_id(w.wid, rank), N, C, D, w.dtype)
+    inp = make_inputs(rank_seed_id(w.wid, rank), N, C, D, w.dtype, T=T)
     dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
     x, W, b, dy = dev["x"], dev["W"], dev["b"], dev["dy"]
-    What = torch.empty(F.feql_weight_fft_bytes(C, D, mode), dtype=torch.uint8, device="cuda")
-    y = torch.empty((N, D, 4), dtype=x.dtype, device="cuda")
-    dx = torch.empty((N, C, 4), dtype=x.dtype, device="cuda")
-    dW = torch.empty((D, C, 4), dtype=x.dtype, device="cuda")
+    What = torch.empty(F.feql_ct_weight_fft_bytes(T, C, D, mode), dtype=torch.uint8,
+                       device="cuda")
+    y = torch.empty((N, D, T), dtype=x.dtype, device="cuda")
+    dx = torch.empty((N, C, T), dtype=x.dtype, device="cuda")
+    dW = torch.empty((D, C, T), dtype=x.dtype, device="cuda")
     db = torch.empty((D,), dtype=x.dtype, device="cuda")
-    ws = L.dw_workspace(N, C, D, mode, "cuda")
+    ws = torch.empty(max(F.feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode), 16),
+                     dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     s = stream.cuda_stream
     # One step = every row of the path: weight rDFT, forward, and the backward
-    # (dX and dW/db, fused into one pass over dy unless --separate-backward).
+    # (dX and dW/db, fused into one pass over dy for p4 unless --separate-backward).
     calls = {
-        "wfft": lambda: F.feql_weight_fft(W, What, C, D, mode, s),
-        "fwd": lambda: F.feql_forward(x, What, b, y, N, C, D, mode, s),
-        "dx": lambda: F.feql_backward_dx(dy, What, dx, N, C, D, mode, s),
-        "dw": lambda: F.feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
+        "wfft": lambda: F.feql_ct_weight_fft(T, W, What, C, D, mode, s),
+        "fwd": lambda: F.feql_ct_forward(T, x, What, b, y, N, C, D, mode, s),
+        "dx": lambda: F.feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, s),
+        "dw": lambda: F.feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
         "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode, s),
     }
     passes = ["wfft"] + (["fwd"] if "fwd" in w.passes else [])
-    if "dx" in w.passes and "dw" in w.passes and not args.separate_backward:
+    if "dx" in w.passes and "dw" in w.passes and not args.separate_backward and T == 4:
         passes.append("bwd")
     else:
         passes += [p for p in ("dx", "dw") if p in w.passes]
@@ -384,7 +399,7 @@ def main():
     value = N * world * args.steps / (ms * 1e-3)
     peak, peak_src = measured_peaks()
     nbytes = workload_bytes(w, elt)
-    macs = 6 * N * C * D
+    macs, dense_macs = layer_macs(w)
     mean_ms = {p: float(np.mean(v)) for p, v in per_pass.items()}
     gemm_passes = {"wfft": 0, "fwd": 1, "dx": 1, "dw": 1, "bwd": 2}  # layer contractions per pass
     pass_report = {}
@@ -396,7 +411,7 @@ def main():
             g = gemm_passes[p]
             pass_report[p]["alg_TFLOP_s"] = round(2 * macs * g / (mean_ms[p] * 1e-3) / 1e12, 2)
             pass_report[p]["dense_equiv_TFLOP_s"] = round(
-                2 * 16 * N * C * D * g / (mean_ms[p] * 1e-3) / 1e12, 2)
+                2 * dense_macs * g / (mean_ms[p] * 1e-3) / 1e12, 2)
     dom = max((p for p in passes if p != "wfft"), key=lambda p: mean_ms[p])
     achieved = nbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
     traffic = None
@@ -414,11 +429,11 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16" if w.dtype == "fp16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "N": N, "C": C, "D": D, "T": 4,
+        "config": {"workload": w.name, "N": N, "C": C, "D": D, "T": T,
                    "passes": passes, "accumulate": "f32", "l2": "inputs larger than L2, no flush",
                    "global_tokens": N * world,
                    "parallelism": f"dp{world}" if world > 1 else "single"},
-        "effective_TFLOP_s": round(2 * 16 * N * C * D * sum(gemm_passes[p] for p in passes)
+        "effective_TFLOP_s": round(2 * dense_macs * sum(gemm_passes[p] for p in passes)
                                    * world / (step_ms * 1e-3) / 1e12, 2),
         "roofline_pct_step": round(100 * sum(nbytes[p] for p in passes) / (step_ms * 1e-3) / 1e9
                                    / peak, 2),

@@ -87,6 +87,32 @@ __device__ __forceinline__ void rdft8(const float (&v)[8], float (&o)[8]) {
   o[7] = g - b2;
 }
 
+// The same transform for two channels at once on packed fp16 pairs (like the
+// p4 butterflies): w0, w1 are the 16-byte rows (8 group elements) of channels
+// q and q+1; o[p] packs plane p of (q, q+1), low half first.  Each add or
+// multiply rounds to fp16 (three to four roundings per output).
+__device__ __forceinline__ void rdft8_pair(const uint4 &w0, const uint4 &w1, uint32_t (&o)[8]) {
+  const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w}, b[4] = {w1.x, w1.y, w1.z, w1.w};
+  __half2 v[8];  // v[t] = (channel q, channel q+1) at group element t
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = __byte_perm(a[e], b[e], 0x5410), hi = __byte_perm(a[e], b[e], 0x7632);
+    v[2 * e] = *reinterpret_cast<const __half2 *>(&lo);
+    v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
+  }
+  const __half2 c = __float2half2_rn(kC8);
+  const __half2 a0 = __hadd2(v[0], v[4]), a1 = __hadd2(v[1], v[5]);
+  const __half2 a2 = __hadd2(v[2], v[6]), a3 = __hadd2(v[3], v[7]);
+  const __half2 b0 = __hsub2(v[0], v[4]), b1 = __hsub2(v[1], v[5]);
+  const __half2 b2 = __hsub2(v[2], v[6]), b3 = __hsub2(v[3], v[7]);
+  const __half2 e02 = __hadd2(a0, a2), e13 = __hadd2(a1, a3);
+  const __half2 h = __hmul2(c, __hsub2(b1, b3)), g = __hmul2(c, __hadd2(b1, b3));
+  const __half2 r[8] = {__hadd2(e02, e13), __hsub2(e02, e13), __hadd2(b0, h), __hadd2(b2, g),
+                        __hsub2(a0, a2),   __hsub2(a1, a3),   __hsub2(b0, h), __hsub2(g, b2)};
+#pragma unroll
+  for (int p = 0; p < 8; ++p) o[p] = *reinterpret_cast<const uint32_t *>(&r[p]);
+}
+
 // Inverse: y[0..7] from Y0, Y4 and (Re, Im) of bins 1..3.
 __device__ __forceinline__ void irdft8(float Y0, float Y4, float r1, float i1, float r2, float i2,
                                        float r3, float i3, float (&y)[8]) {
@@ -170,15 +196,18 @@ __global__ void wfft_ct8_kernel(const __half *__restrict__ W, uint8_t *__restric
 //                N = BD for bins 0 and 4, two N = 2 BD for each complex bin,
 //                into 8 BD accumulator columns (double-buffered when BD <= 32)
 //   warps 2..9   transform: thread = (token row, box); the 8-point rDFT of its
-//                8 channel fibres in fp32, then, after a team barrier, the
+//                8 channel fibres on packed fp16 pairs, then, after a team barrier, the
 //                chunk rewritten in place as eight K-major planes of 4 KB
 //   warps 10..13 epilogue: warp q reads TMEM lane quadrant q (32 token rows);
-//                inverse rDFT + bias in fp32; each lane writes its row's
-//                8 output channels (8 x 16 B contiguous) directly
+//                inverse rDFT + bias in fp32; per 8 output channels each lane
+//                writes its row (128 B) into a 128-byte-swizzled staging box
+//                and the warp issues one 4 KB TMA store (two boxes per warp)
 constexpr int kCt8Threads = 64 + 12 * 32;
 constexpr int kCt8XChunk = kBM * kCK * kT8 * 2;  // 32 KB: 128 tokens x 16 channels x 8
 constexpr int kCt8Box = kCt8XChunk / 2;          // 16 KB: 8 channels
 constexpr int kCt8Plane = kBM * kCK * 2;         // 4 KB: 128 tokens x 32 B
+constexpr int kCt8OutBox = 32 * 128;             // 4 KB: 32 rows x 8 channels x 8
+constexpr int kCt8NumOut = 2;                    // staging boxes per epilogue warp
 
 struct Ct8FwdParams {
   const uint8_t *wt;   // weight chunks of this direction, [j][kc]
@@ -192,13 +221,14 @@ struct Ct8FwdParams {
 };
 
 struct Ct8Smem {
-  int stage0, bias, bars, total;
+  int stage0, out0, bias, bars, total;
 };
 
 __host__ __device__ inline Ct8Smem ct8_fwd_smem(const Ct8FwdParams &p) {
   Ct8Smem s;
   s.stage0 = 0;
-  s.bias = p.stages * p.stage_bytes;
+  s.out0 = p.stages * p.stage_bytes;
+  s.bias = s.out0 + 4 * kCt8NumOut * kCt8OutBox;
   s.bars = s.bias + static_cast<int>(align_up(p.bias_floats * 4, 16));
   // full, tready, empty per stage; acc_full, acc_empty x2; final; tmem slot
   s.total = s.bars + (3 * p.stages + 4 + 1) * 8 + 16;
@@ -215,7 +245,8 @@ __device__ __forceinline__ bool ct8_unit(const Ct8FwdParams &p, int k, int &m, i
 
 // 14 warps over the 4 SM sub-partitions put 4 warps on one 16K-register slice.
 __global__ void __maxnreg__(128)
-tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const Ct8FwdParams p) {
+tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
+                  const Ct8FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -260,6 +291,7 @@ tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const Ct8FwdParams 
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
+      tma_prefetch_desc(&tm_out);
       int s = 0, m, j;
       uint32_t ph = 0;
       for (int k = 0; ct8_unit(p, k, m, j); ++k) {
@@ -333,23 +365,13 @@ tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const Ct8FwdParams 
         const uint8_t *src = st + bx * kCt8Box + r * 128;
         uint32_t pw[8][4];  // [plane][channel pair], packed fp16
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {  // 16-byte chunk q = channel 8 bx + q, its 8 group elements
-          const uint4 raw = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-          float v[8], o[8];
+        for (int q = 0; q < 8; q += 2) {  // 16-byte chunk q = channel 8 bx + q, its 8 group elements
+          const uint4 r0 = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
+          const uint4 r1 = *reinterpret_cast<const uint4 *>(src + (((q + 1) ^ (r & 7)) << 4));
+          uint32_t o[8];
+          rdft8_pair(r0, r1, o);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wv[e]));
-            v[2 * e] = f.x;
-            v[2 * e + 1] = f.y;
-          }
-          rdft8(v, o);
-#pragma unroll
-          for (int pp = 0; pp < 8; ++pp) {
-            const uint32_t hv = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(o[pp])));
-            if (q % 2 == 0) pw[pp][q / 2] = hv;
-            else pw[pp][q / 2] |= hv << 16;
-          }
+          for (int pp = 0; pp < 8; ++pp) pw[pp][q / 2] = o[pp];
         }
         named_bar_sync(2, 256);  // every row read before the planes overwrite it
 #pragma unroll
@@ -366,13 +388,13 @@ tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const Ct8FwdParams 
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;
     const int groups = p.BD / 8;
-    int a = 0, m, j;
+    uint8_t *obase = smem + L.out0 + (warp - 10) * kCt8NumOut * kCt8OutBox;
+    int a = 0, oi = 0, m, j;
     uint32_t aph = 0;
     for (int it = 0; ct8_unit(p, it, m, j); ++it) {
       if (ok) ok = mbar_wait(&acc_full[a], aph);
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
-      const int64_t n = static_cast<int64_t>(m) * kBM + quad * 32 + lane;
       for (int g = 0; g < groups; ++g) {
         uint32_t Y[8][8];  // [accumulator block][column]: Y0, Y4, Re1, Im1, Re2, Im2, Re3, Im3
         __syncwarp();      // the TMEM loads are warp-collective
@@ -385,24 +407,32 @@ tc_ct8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const Ct8FwdParams 
           if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
         }
         const int d0 = j * p.BD + g * 8;
-        if (n < p.N) {
+        if (d0 >= p.Do) continue;  // whole group is padding
+        uint8_t *ob = obase + (oi % kCt8NumOut) * kCt8OutBox;
+        if (lane == 0) bulk_wait_read<kCt8NumOut - 1>();  // this box's last store has read it
+        __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (d0 + i < p.Do) {
-              float y[8];
-              irdft8(__uint_as_float(Y[0][i]), __uint_as_float(Y[1][i]), __uint_as_float(Y[2][i]),
-                     __uint_as_float(Y[3][i]), __uint_as_float(Y[4][i]), __uint_as_float(Y[5][i]),
-                     __uint_as_float(Y[6][i]), __uint_as_float(Y[7][i]), y);
-              const float bv = sbias[d0 + i];
-              *reinterpret_cast<uint4 *>(p.out + (n * p.Do + d0 + i) * kT8) =
-                  make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
-                             pack_half2(y[4] + bv, y[5] + bv), pack_half2(y[6] + bv, y[7] + bv));
-            }
-          }
+        for (int i = 0; i < 8; ++i) {  // 16-byte chunk i of the row = output channel d0 + i
+          float y[8];
+          irdft8(__uint_as_float(Y[0][i]), __uint_as_float(Y[1][i]), __uint_as_float(Y[2][i]),
+                 __uint_as_float(Y[3][i]), __uint_as_float(Y[4][i]), __uint_as_float(Y[5][i]),
+                 __uint_as_float(Y[6][i]), __uint_as_float(Y[7][i]), y);
+          const float bv = sbias[d0 + i];
+          *reinterpret_cast<uint4 *>(ob + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+              make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
+                         pack_half2(y[4] + bv, y[5] + bv), pack_half2(y[6] + bv, y[7] + bv));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {  // the store clips rows past N and channels past Do
+          tma_store_2d(&tm_out, d0 * kT8, m * kBM + quad * 32, ob);
+          bulk_commit();
+        }
+        ++oi;
       }
       if (++a == p.nacc) { a = 0; aph ^= 1; }
     }
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -595,24 +625,18 @@ tc_ct8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
           const uint8_t *src = st + (bi < nqd ? bi * kCt8DwBox : xoff + (bi - nqd) * kCt8DwBox) +
                                r * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-            float v[8], o[8];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wv[u]));
-              v[2 * u] = f.x;
-              v[2 * u + 1] = f.y;
+          for (int q = 0; q < 8; q += 2) {
+            const uint4 r0 = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
+            const uint4 r1 = *reinterpret_cast<const uint4 *>(src + (((q + 1) ^ (r & 7)) << 4));
+            uint32_t o[8];
+            rdft8_pair(r0, r1, o);
+            if (bi < nqd) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&o[0]));
+              db_acc[k][q] += f.x;
+              db_acc[k][q + 1] += f.y;
             }
-            rdft8(v, o);
-            if (bi < nqd) db_acc[k][q] += o[0];
 #pragma unroll
-            for (int pp = 0; pp < 8; ++pp) {
-              const uint32_t hv = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(o[pp])));
-              if (q % 2 == 0) pw[k][pp][q / 2] = hv;
-              else pw[k][pp][q / 2] |= hv << 16;
-            }
+            for (int pp = 0; pp < 8; ++pp) pw[k][pp][q / 2] = o[pp];
           }
         }
       }

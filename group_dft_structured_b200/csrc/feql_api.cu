@@ -375,15 +375,17 @@ int launch_ct8_fwd(const void *in, const uint8_t *wt, const Ct8Plan &P, const __
   p.stages = 6;
   while (p.stages > 2 && ct8_fwd_smem(p).total > budget) --p.stages;
   if (ct8_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
-  CUtensorMap tm;
+  CUtensorMap tm, tm_out;
   st = make_tmap_f16(&tm, in, N, static_cast<int64_t>(P.Ci) * kT8, kBM);
+  if (st != FEQL_OK) return st;
+  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT8, 32);
   if (st != FEQL_OK) return st;
   const int smem = ct8_fwd_smem(p).total + 1024;
   if (cudaFuncSetAttribute(tc_ct8_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FEQL_ERR_CUDA;
   const int grid = p.n_units < dev.sms ? p.n_units : dev.sms;
-  tc_ct8_fwd_kernel<<<grid, kCt8Threads, smem, stream>>>(tm, p);
+  tc_ct8_fwd_kernel<<<grid, kCt8Threads, smem, stream>>>(tm, tm_out, p);
   return launch_status();
 }
 
