@@ -734,33 +734,62 @@ tc_ct8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
   }
 }
 
-// Fixed-order sum of the split partials, then dW[d][c][0..7] = irDFT_8 of the
-// eight bin planes and db[d].  One thread per (d, c) output fibre, then per d.
-__global__ void ct8_dw_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
-                                     __half *__restrict__ dW, __half *__restrict__ db, int splits,
-                                     int C, int D, int Cs) {
+// Sum of the split partials in a fixed order, then dW[d][c][0..7] = irDFT_8 of
+// the eight bin planes, and db[d].  A block takes 16 consecutive (d, c) outputs
+// (the last blocks take db); its 32 warps each sum every 32nd split (the loads
+// of a warp's splits are independent, so they overlap), then warp 0 adds the
+// 32 partial sums in warp order: the same grouping on every run.
+constexpr int kRed8Out = 16, kRed8Groups = 32;
+
+__host__ __device__ inline int64_t ct8_reduce_blocks(int C, int D) {
+  return cdiv(static_cast<int64_t>(D) * C, kRed8Out) + cdiv(D, kRed8Out);
+}
+
+__global__ void __launch_bounds__(kRed8Out * kRed8Groups)
+ct8_dw_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
+                     __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
+                     int Cs) {
+  __shared__ float part[kRed8Groups][kT8][kRed8Out];
   const int64_t n = static_cast<int64_t>(D) * C;
   const int64_t plane = static_cast<int64_t>(D) * Cs;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n + D;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  const int64_t nblk_w = cdiv(n, kRed8Out);
+  const int lo = threadIdx.x % kRed8Out, grp = threadIdx.x / kRed8Out;
+  if (blockIdx.x < nblk_w) {
+    const int64_t e = blockIdx.x * static_cast<int64_t>(kRed8Out) + lo;
+    float G[kT8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (e < n) {
-      const int64_t d = e / C, c = e % C;
-      float G[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int s = 0; s < splits; ++s) {
-        const float *q = ws + static_cast<int64_t>(s) * 8 * plane + d * Cs + c;
+      const float *src = ws + (e / C) * Cs + (e % C);
+      for (int s = grp; s < splits; s += kRed8Groups) {
+        const float *q = src + static_cast<int64_t>(s) * kT8 * plane;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) G[k] += q[k * plane];
+        for (int k = 0; k < kT8; ++k) G[k] += q[k * plane];
       }
-      float y[8];
-      irdft8(G[0], G[1], G[2], G[3], G[4], G[5], G[6], G[7], y);
+    }
+#pragma unroll
+    for (int k = 0; k < kT8; ++k) part[grp][k][lo] = G[k];
+    __syncthreads();
+    if (grp == 0 && e < n) {
+      float t[kT8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < kRed8Groups; ++q)
+#pragma unroll
+        for (int k = 0; k < kT8; ++k) t[k] += part[q][k][lo];
+      float y[kT8];
+      irdft8(t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7], y);
       *reinterpret_cast<uint4 *>(dW + e * kT8) =
           make_uint4(pack_half2(y[0], y[1]), pack_half2(y[2], y[3]), pack_half2(y[4], y[5]),
                      pack_half2(y[6], y[7]));
-    } else if (db != nullptr) {
-      const int64_t d = e - n;
-      float sum = 0.f;
-      for (int s = 0; s < splits; ++s) sum += ws_db[static_cast<int64_t>(s) * D + d];
-      db[d] = __float2half_rn(sum);
+    }
+  } else if (db != nullptr) {
+    const int64_t d = (blockIdx.x - nblk_w) * kRed8Out + lo;
+    float sdb = 0.f;
+    if (d < D)
+      for (int s = grp; s < splits; s += kRed8Groups) sdb += ws_db[static_cast<int64_t>(s) * D + d];
+    part[grp][0][lo] = sdb;
+    __syncthreads();
+    if (grp == 0 && d < D) {
+      float t = 0.f;
+      for (int q = 0; q < kRed8Groups; ++q) t += part[q][0][lo];
+      db[d] = __float2half_rn(t);
     }
   }
 }

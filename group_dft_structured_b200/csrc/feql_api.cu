@@ -443,9 +443,10 @@ int launch_ct8_dw(const void *x, const void *dy, __half *dW, __half *db, float *
     if (grid > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
     tc_ct8_dw_kernel<<<static_cast<unsigned>(grid), kCt8DwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  const int64_t outs = static_cast<int64_t>(D) * C + D;
-  ct8_dw_reduce_kernel<<<grid_for(outs, 256, dev.sms), 256, 0, stream>>>(p.ws, p.ws_db, dW, db,
-                                                                        p.splits, C, D, p.Cs);
+  const int64_t rblocks = ct8_reduce_blocks(C, D);
+  if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  ct8_dw_reduce_kernel<<<static_cast<unsigned>(rblocks), kRed8Out * kRed8Groups, 0, stream>>>(
+      p.ws, p.ws_db, dW, db, p.splits, C, D, p.Cs);
   return launch_status();
 }
 
