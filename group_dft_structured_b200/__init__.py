@@ -62,6 +62,9 @@ _SIGNATURES = {
     "feql_ct_backward_dx": (_I, [_I, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
     "feql_ct_backward_dw_workspace_bytes": (_SZ, [_I, _I64, _I, _I, _I]),
     "feql_ct_backward_dw": (_I, [_I, _VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
+    "feql_mlp_weight_fft_bytes": (_SZ, [_I, _I, _I, _I]),
+    "feql_mlp_weight_fft": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP]),
+    "feql_mlp_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP]),
     "feql_device_status": (_I, [_VP]),
     "feql_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -184,6 +187,21 @@ def feql_ct_backward_dw(T: int, x, dy, dW, db, ws, ws_bytes: int, N: int, C: int
     _check(load().feql_ct_backward_dw(T, _ptr(x), _ptr(dy), _ptr(dW), _ptr(db), _ptr(ws),
                                       ws_bytes, N, C, D, dtype, _stream(stream)),
            "feql_ct_backward_dw")
+
+
+def feql_mlp_weight_fft_bytes(C: int, H: int, Co: int, dtype: int) -> int:
+    return int(load().feql_mlp_weight_fft_bytes(C, H, Co, dtype))
+
+
+def feql_mlp_weight_fft(W1, W2, What, C: int, H: int, Co: int, dtype: int, stream=None) -> None:
+    _check(load().feql_mlp_weight_fft(_ptr(W1), _ptr(W2), _ptr(What), C, H, Co, dtype,
+                                      _stream(stream)), "feql_mlp_weight_fft")
+
+
+def feql_mlp_forward(x, What, b1, b2, y, N: int, C: int, H: int, Co: int, dtype: int,
+                     stream=None) -> None:
+    _check(load().feql_mlp_forward(_ptr(x), _ptr(What), _ptr(b1), _ptr(b2), _ptr(y), N, C, H, Co,
+                                   dtype, _stream(stream)), "feql_mlp_forward")
 
 
 def feql_device_status(stream=None) -> int:

@@ -18,6 +18,7 @@
 #include "tc_dw.cuh"
 #include "tc_fwd.cuh"
 #include "ct8.cuh"
+#include "tc_mlp.cuh"
 #include "wfft.cuh"
 
 using namespace feql;
@@ -450,6 +451,66 @@ int launch_ct8_dw(const void *x, const void *dy, __half *dW, __half *db, float *
   return launch_status();
 }
 
+// ---------------------------------------------------------------- MLP block
+// Shared memory a block may use on sm_100 (227 KB), less the base alignment.
+constexpr int kMlpSmemBudget = 227 * 1024 - 1024;
+
+// The plan depends only on (C, H, Co), so the weight buffer's layout does too:
+// the widest hidden slice whose two fc1 accumulators and the fc2 accumulator
+// fit 512 TMEM columns, with two x tile buffers if they fit, else one.
+int plan_mlp(int C, int H, int Co, TcMlpParams *out) {
+  if (align_up(Co, 16) > 64) return FEQL_ERR_UNSUPPORTED;
+  const int hs_opts[4] = {64, 48, 32, 16};
+  for (int nx = 2; nx >= 1; --nx) {
+    for (int hs_max : hs_opts) {
+      TcMlpParams p;
+      p.P = make_mlp_plan(C, H, Co, hs_max);
+      p.nx = nx;
+      if (mlp_tmem_cols(p.P) > 512 || mlp_smem(p).total > kMlpSmemBudget) continue;
+      *out = p;
+      return FEQL_OK;
+    }
+  }
+  return FEQL_ERR_UNSUPPORTED;
+}
+
+int mlp_check(int C, int H, int Co, int dtype) {
+  if (!valid_dtype(dtype) || check_shape(C, H) != FEQL_OK || check_shape(H, Co) != FEQL_OK)
+    return FEQL_ERR_INVALID_ARG;
+  if (resolve(dtype) != FEQL_FP16) return FEQL_ERR_UNSUPPORTED;
+  if ((C | Co) & 1) return FEQL_ERR_UNSUPPORTED;  // TMA rows of 8C and 8Co bytes
+  return FEQL_OK;
+}
+
+int launch_mlp(const void *x, const uint8_t *wt, const __half *b1, const __half *b2, void *y,
+               int64_t N, const TcMlpParams &plan, cudaStream_t stream) {
+  DeviceInfo dev;
+  int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
+  TcMlpParams p = plan;
+  p.wt = wt;
+  p.b1 = b1;
+  p.b2 = b2;
+  p.N = N;
+  const int64_t nM = cdiv(N, kBM);
+  if (nM > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  p.nM = static_cast<int>(nM);
+  const int smem = mlp_smem(p).total + 1024;
+  if (smem > dev.smem_optin) return FEQL_ERR_UNSUPPORTED;
+  CUtensorMap tm_in, tm_out;
+  st = make_tmap_f16(&tm_in, x, N, static_cast<int64_t>(p.P.C) * kT, kBM);
+  if (st != FEQL_OK) return st;
+  st = make_tmap_f16(&tm_out, y, N, static_cast<int64_t>(p.P.Co) * kT, 32);
+  if (st != FEQL_OK) return st;
+  if (cudaFuncSetAttribute(tc_mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FEQL_ERR_CUDA;
+  const int grid = p.nM < dev.sms ? p.nM : dev.sms;
+  tc_mlp_kernel<<<grid, kMlpThreads, smem, stream>>>(tm_in, tm_out, p);
+  return launch_status();
+}
+
 // Checks shared by the C_T entry points: a supported group order and mode.
 // Returns FEQL_OK for T = 8 in FEQL_FP16 (T = 4 is forwarded before this).
 int ct_check(int T, int dtype) {
@@ -694,6 +755,49 @@ int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db
   return launch_ct8_dw(x, dy, static_cast<__half *>(dW), static_cast<__half *>(db),
                        static_cast<float *>(ws), ws_bytes, N, C, D,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t feql_mlp_weight_fft_bytes(int C, int H, int Co, int dtype) {
+  TcMlpParams p;
+  if (mlp_check(C, H, Co, dtype) != FEQL_OK || plan_mlp(C, H, Co, &p) != FEQL_OK) return 0;
+  return static_cast<size_t>(p.P.bytes);
+}
+
+int feql_mlp_weight_fft(const void *W1, const void *W2, void *What, int C, int H, int Co,
+                        int dtype, feql_stream stream) {
+  int st = mlp_check(C, H, Co, dtype);
+  if (st != FEQL_OK) return st;
+  if (W1 == nullptr || W2 == nullptr || What == nullptr) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(W1) || !aligned16(W2) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
+  TcMlpParams p;
+  st = plan_mlp(C, H, Co, &p);
+  if (st != FEQL_OK) return st;
+  DeviceInfo dev;
+  st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  wfft_mlp_kernel<<<grid_for((p.P.w1_bytes + p.P.w2_bytes) / 2, 256, dev.sms), 256, 0,
+                    reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half *>(W1), static_cast<const __half *>(W2),
+      static_cast<uint8_t *>(What), p.P);
+  return launch_status();
+}
+
+int feql_mlp_forward(const void *x, const void *What, const void *b1, const void *b2, void *y,
+                     int64_t N, int C, int H, int Co, int dtype, feql_stream stream) {
+  int st = mlp_check(C, H, Co, dtype);
+  if (st != FEQL_OK) return st;
+  if (N < 0 || N > kMaxTokens) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || What == nullptr || y == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(What) || !aligned16(y) || (b1 != nullptr && !aligned16(b1)) ||
+      (b2 != nullptr && !aligned16(b2)))
+    return FEQL_ERR_INVALID_ARG;
+  TcMlpParams p;
+  st = plan_mlp(C, H, Co, &p);
+  if (st != FEQL_OK) return st;
+  if (N == 0) return FEQL_OK;
+  return launch_mlp(x, static_cast<const uint8_t *>(What), static_cast<const __half *>(b1),
+                    static_cast<const __half *>(b2), y, N, p,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 int feql_device_status(feql_stream stream) {

@@ -1,0 +1,487 @@
+// tc_mlp.cuh — the p4-equivariant MLP block (fc1 -> GELU -> fc2) as one
+// kernel on the sm_100a tensor cores, fp16 data with fp32 accumulation.
+//
+// Flash EQ-Linear builds its networks (technical summary "Livello di Rete":
+// Flash EQ-ViT, Flash EQ-Swin) from EQ-Linear layers; a transformer MLP is two
+// of them with a pointwise GELU between.  Both layers run the Fourier method
+// (rDFT along the group axis, six real products per 16 channels, inverse),
+// and the hidden activation never leaves the SM: fc1's accumulators are read
+// from TMEM, inverse-transformed, biased, passed through GELU, transformed
+// again and written to shared memory as fc2's A operand.
+//
+//   h[n,j,t] = b1[j] + sum_c sum_s W1[j,c,(t-s) mod 4] x[n,c,s]
+//   y[n,o,t] = b2[o] + sum_j sum_s W2[o,j,(t-s) mod 4] GELU(h[n,j,s])
+//
+// GELU is evaluated in its tanh form, 0.5 z (1 + tanh(sqrt(2/pi)(z + 0.044715 z^3)))
+// (Hendrycks and Gimpel), on packed fp16 pairs with the hardware tanh; it is
+// within 5e-4 of the exact z*Phi(z) for every z.
+//
+// One persistent CTA per SM, 128-token tiles, 18 warps:
+//   warp 0        TMA: the resident Fourier weights of both layers (once), then
+//                 each tile's x chunks [128 tokens x 16 channels x 4] into one
+//                 of `nx` tile buffers
+//   warp 1        TMEM allocator + single-thread MMA issuer
+//   warps 2..5    transform: rDFT of the x tile in place into four K-major
+//                 planes per chunk (V0, V2, Re V1, -Im V1)
+//   warps 6..13   two GELU teams, one per fc1 accumulator buffer: hidden slice
+//                 of HS channels -> inverse rDFT + b1 -> GELU -> rDFT -> fp16
+//                 planes in one of two hidden buffers
+//   warps 14..17  fc2 epilogue: inverse rDFT + b2, TMA stores of y
+// TMEM: fc1 accumulators 2 x 4*HS columns (Y0 | Y2 | Re Y1 | Im Y1 of a
+// slice), fc2 accumulator 4*BD2 columns at 8*HS.
+// Issue order per tile: fc1(0), fc1(1), fc2(0), fc1(2), fc2(1), ..., fc2(nS-1),
+// so the GELU of one slice overlaps the MMAs of the next.
+// Every wait is bounded (mbar_wait); a timed-out thread stops issuing work but
+// keeps the loop structure so named barriers stay matched.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "plan.cuh"
+#include "rdft4.cuh"
+#include "sm100.cuh"
+#include "wfft.cuh"
+
+namespace feql {
+
+constexpr int kMlpThreads = 18 * 32;
+constexpr int kMlpYBoxes = 2;                    // output staging boxes per epilogue warp
+constexpr int kMlpChunkBytes = kBM * kCK * kT * 2;  // 16 KB: 128 tokens x 16 channels x 4
+constexpr int kMlpPlaneBytes = kBM * kCK * 2;       // 4 KB: one plane of a chunk
+
+// Plan of the block: shapes, hidden slicing and the Fourier-weight layout.
+//   fc1 weights: [slice j][x chunk kc] blocks of 5*HS rows x 32 B
+//   fc2 weights: [hidden chunk kh] blocks of 5*BD2 rows x 32 B
+// each block laid out like the single layer's (planes What0, What2, Re1, Im1,
+// -Re1 of BD rows, K-major, 32-byte swizzle).
+struct MlpPlan {
+  int C, H, Co;
+  int nK1;             // x chunks of 16 channels
+  int HS, nS;          // hidden slice width (multiple of 16) and count
+  int nKh;             // hidden chunks of 16 channels: nS * HS / 16
+  int BD2;             // fc2 output channels, padded to 16 (<= 64)
+  int w1_chunk, w2_chunk;
+  int64_t w1_bytes, w2_bytes, off_w2, bytes;
+};
+
+__host__ __device__ inline MlpPlan make_mlp_plan(int C, int H, int Co, int hs_max) {
+  MlpPlan p;
+  p.C = C;
+  p.H = H;
+  p.Co = Co;
+  p.nK1 = static_cast<int>(cdiv(C, kCK));
+  p.BD2 = static_cast<int>(align_up(Co, 16));
+  p.nS = static_cast<int>(cdiv(H, hs_max));
+  p.HS = static_cast<int>(align_up(cdiv(H, p.nS), 16));
+  p.nKh = p.nS * p.HS / kCK;
+  p.w1_chunk = 5 * p.HS * kCK * 2;
+  p.w2_chunk = 5 * p.BD2 * kCK * 2;
+  p.w1_bytes = static_cast<int64_t>(p.nS) * p.nK1 * p.w1_chunk;
+  p.w2_bytes = static_cast<int64_t>(p.nKh) * p.w2_chunk;
+  p.off_w2 = align_up(p.w1_bytes, 1024);
+  p.bytes = p.off_w2 + align_up(p.w2_bytes, 1024);
+  return p;
+}
+
+// Weight transform of both layers: one thread per fp16 element of the buffer.
+__global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__restrict__ W2,
+                                uint8_t *__restrict__ What, MlpPlan P) {
+  const int64_t n1 = P.w1_bytes / 2, n2 = P.w2_bytes / 2;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n1 + n2;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool first = e < n1;
+    const int64_t le = first ? e : e - n1;
+    const int BD = first ? P.HS : P.BD2;
+    const int rows = 5 * BD;
+    const int64_t chunk = le / (rows * kCK);
+    const int rem = static_cast<int>(le % (rows * kCK));
+    const int row = rem / kCK, k = rem % kCK;
+    const int sub = row / BD;
+    int o, i, Do, Ci;
+    if (first) {  // chunk = slice j * nK1 + kc
+      o = static_cast<int>(chunk / P.nK1) * BD + row % BD;
+      i = static_cast<int>(chunk % P.nK1) * kCK + k;
+      Do = P.H;
+      Ci = P.C;
+    } else {  // chunk = hidden chunk kh
+      o = row % BD;
+      i = static_cast<int>(chunk) * kCK + k;
+      Do = P.Co;
+      Ci = P.H;
+    }
+    float v = 0.f;
+    if (o < Do && i < Ci) {
+      float b0, b2, b1r, b1i;
+      weight_bins(first ? W1 : W2, Ci, 0, o, i, b0, b2, b1r, b1i);
+      v = sub == 0 ? b0 : sub == 1 ? b2 : sub == 2 ? b1r : sub == 3 ? b1i : -b1r;
+    }
+    const int64_t base = first ? chunk * P.w1_chunk : P.off_w2 + chunk * P.w2_chunk;
+    *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);
+  }
+}
+
+struct TcMlpParams {
+  MlpPlan P;
+  const uint8_t *wt;   // Fourier weights (MlpPlan layout)
+  const __half *b1;    // [H] or nullptr
+  const __half *b2;    // [Co] or nullptr
+  int64_t N;
+  int nM;              // token tiles
+  int nx;              // x tile buffers (1 or 2)
+};
+
+struct MlpSmem {
+  int w1, w2, x0, h0, y0, b1, b2, bars, total;
+  int xtile, htile;    // bytes of one x tile buffer / one hidden buffer
+};
+
+__host__ __device__ inline MlpSmem mlp_smem(const TcMlpParams &p) {
+  MlpSmem s;
+  s.xtile = p.P.nK1 * kMlpChunkBytes;
+  s.htile = (p.P.HS / kCK) * kMlpChunkBytes;
+  s.w1 = 0;
+  s.w2 = static_cast<int>(align_up(p.P.w1_bytes, 1024));
+  s.x0 = s.w2 + static_cast<int>(align_up(p.P.w2_bytes, 1024));
+  s.h0 = s.x0 + p.nx * s.xtile;
+  s.y0 = s.h0 + 2 * s.htile;
+  s.b1 = s.y0 + 4 * kMlpYBoxes * 4096;
+  s.b2 = s.b1 + p.P.nS * p.P.HS * 4;
+  s.bars = s.b2 + static_cast<int>(align_up(p.P.BD2 * 4, 16));
+  s.total = s.bars + 24 * 8 + 16;
+  return s;
+}
+
+// TMEM columns the block needs: two fc1 accumulators and the fc2 accumulator.
+__host__ __device__ inline int mlp_tmem_cols(const MlpPlan &P) { return 8 * P.HS + 4 * P.BD2; }
+
+__device__ __forceinline__ uint32_t tanh_h2(uint32_t x) {
+  uint32_t y;
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// GELU (tanh form) of a packed fp16 pair.
+__device__ __forceinline__ uint32_t gelu_h2(uint32_t zu) {
+  const __half2 z = as_h2(zu);
+  const __half2 k0 = __float2half2_rn(0.7978845608028654f);   // sqrt(2/pi)
+  const __half2 k1 = __float2half2_rn(0.0356774081363001f);   // 0.044715 sqrt(2/pi)
+  const __half2 hf = __float2half2_rn(0.5f);
+  const __half2 u = __hmul2(z, __hfma2(k1, __hmul2(z, z), k0));
+  const __half2 t = as_h2(tanh_h2(as_u32(u)));
+  const __half2 hz = __hmul2(hf, z);
+  return as_u32(__hfma2(hz, t, hz));
+}
+
+// 18 warps: 5 on one register slice of an SM sub-partition, 96 registers each.
+__global__ void __maxnreg__(96)
+tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
+              const TcMlpParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const MlpPlan &P = p.P;
+  const MlpSmem L = mlp_smem(p);
+  float *sb1 = reinterpret_cast<float *>(smem + L.b1);
+  float *sb2 = reinterpret_cast<float *>(smem + L.b2);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint64_t *wfull = bars;
+  uint64_t *xfull = bars + 1, *xready = bars + 3, *xempty = bars + 5;
+  uint64_t *a1full = bars + 7, *a1empty = bars + 9;
+  uint64_t *hready = bars + 11, *hempty = bars + 13;
+  uint64_t *a2full = bars + 15, *a2empty = bars + 16, *final_bar = bars + 17;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int hs = P.HS, nS = P.nS;
+
+  if (threadIdx.x == 0) {
+    mbar_init(wfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xfull[b], 1);
+      mbar_init(&xready[b], 4);
+      mbar_init(&xempty[b], 1);
+      mbar_init(&a1full[b], 1);
+      mbar_init(&a1empty[b], 4);
+      mbar_init(&hready[b], 4);
+      mbar_init(&hempty[b], 1);
+    }
+    mbar_init(a2full, 1);
+    mbar_init(a2empty, 4);
+    mbar_init(final_bar, 1);
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < nS * hs; i += blockDim.x)
+    sb1[i] = (p.b1 != nullptr && i < P.H) ? __half2float(p.b1[i]) : 0.f;
+  for (int i = threadIdx.x; i < P.BD2; i += blockDim.x)
+    sb2[i] = (p.b2 != nullptr && i < P.Co) ? __half2float(p.b2[i]) : 0.f;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t acc2_col = 8 * hs;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_in);
+      tma_prefetch_desc(&tm_out);
+      if (static_cast<int>(blockIdx.x) < p.nM) {
+        mbar_arrive_expect_tx(wfull, static_cast<uint32_t>(P.w1_bytes + P.w2_bytes));
+        bulk_load(smem + L.w1, p.wt, static_cast<uint32_t>(P.w1_bytes), wfull);
+        bulk_load(smem + L.w2, p.wt + P.off_w2, static_cast<uint32_t>(P.w2_bytes), wfull);
+      }
+      int xb = 0;
+      uint32_t xph = 0;
+      for (int m = blockIdx.x; m < p.nM; m += gridDim.x) {
+        if (ok) ok = mbar_wait(&xempty[xb], xph ^ 1);
+        if (ok) {
+          uint8_t *xt = smem + L.x0 + xb * L.xtile;
+          mbar_arrive_expect_tx(&xfull[xb], L.xtile);
+          for (int kc = 0; kc < P.nK1; ++kc)
+            tma_load_2d(xt + kc * kMlpChunkBytes, &tm_in, kc * (kCK * kT), m * kBM, &xfull[xb]);
+        }
+        if (++xb == p.nx) { xb = 0; xph ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t id1a = instr_desc(kBM, hs, 0, 0), id1b = instr_desc(kBM, 2 * hs, 0, 0);
+      const uint32_t id2a = instr_desc(kBM, P.BD2, 0, 0);
+      const uint32_t id2b = instr_desc(kBM, 2 * P.BD2, 0, 0);
+      const uint64_t dsw32 = smem_desc(0, 16, 256, kSw32);  // K-major, 32-byte swizzle
+      const uint32_t dhi = desc_hi(dsw32);
+      const uint32_t x0 = desc_lo(desc_at(dsw32, smem_u32(smem + L.x0)));
+      const uint32_t h0 = desc_lo(desc_at(dsw32, smem_u32(smem + L.h0)));
+      const uint32_t w1_0 = desc_lo(desc_at(dsw32, smem_u32(smem + L.w1)));
+      const uint32_t w2_0 = desc_lo(desc_at(dsw32, smem_u32(smem + L.w2)));
+      const uint32_t pl16 = kMlpPlaneBytes >> 4, ch16 = kMlpChunkBytes >> 4;
+      const uint32_t xt16 = L.xtile >> 4, ht16 = L.htile >> 4;
+      const uint32_t w1r16 = (hs * 32) >> 4, w1c16 = P.w1_chunk >> 4;
+      const uint32_t w2r16 = (P.BD2 * 32) >> 4, w2c16 = P.w2_chunk >> 4;
+      const uint32_t acc2 = tmem_base + acc2_col;
+      const int kh_per = hs / kCK;
+      if (static_cast<int>(blockIdx.x) < p.nM) ok = mbar_wait(wfull, 0);
+      int xb = 0;
+      uint32_t xph = 0;
+      int g = 0;  // hidden slices issued so far (selects the fc1/hidden buffer)
+      int it = 0;
+      // fc2 over hidden slice s of this tile, slice gs overall
+      auto fc2 = [&](int gs, int s) {
+        const int b = gs & 1;
+        const uint32_t bph = (gs >> 1) & 1;
+        if (s == 0 && ok) ok = mbar_wait(a2empty, (it & 1) ^ 1);
+        if (ok) ok = mbar_wait(&hready[b], bph);
+        tc_fence_after();
+        if (ok) {
+          uint32_t hd = h0 + b * ht16, wd = w2_0 + s * kh_per * w2c16;
+          for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
+            const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
+            mma_f16_lo(acc2, hd, wd, dhi, id2a, acc_in);
+            mma_f16_lo(acc2 + P.BD2, hd + pl16, wd + w2r16, dhi, id2a, acc_in);
+            mma_f16_lo(acc2 + 2 * P.BD2, hd + 2 * pl16, wd + 2 * w2r16, dhi, id2b, acc_in);
+            mma_f16_lo(acc2 + 2 * P.BD2, hd + 3 * pl16, wd + 3 * w2r16, dhi, id2b, 1u);
+          }
+          mma_commit(&hempty[b]);
+        }
+      };
+      for (int m = blockIdx.x; m < p.nM; m += gridDim.x, ++it) {
+        if (ok) ok = mbar_wait(&xready[xb], xph);
+        tc_fence_after();
+        for (int s = 0; s < nS; ++s) {
+          const int gs = g + s, b = gs & 1;
+          const uint32_t bph = (gs >> 1) & 1;
+          if (ok) ok = mbar_wait(&a1empty[b], bph ^ 1);
+          tc_fence_after();
+          if (ok) {
+            const uint32_t acc = tmem_base + b * 4 * hs;
+            uint32_t xd = x0 + xb * xt16, wd = w1_0 + s * P.nK1 * w1c16;
+            for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
+              const uint32_t acc_in = kc > 0 ? 1u : 0u;
+              mma_f16_lo(acc, xd, wd, dhi, id1a, acc_in);
+              mma_f16_lo(acc + hs, xd + pl16, wd + w1r16, dhi, id1a, acc_in);
+              mma_f16_lo(acc + 2 * hs, xd + 2 * pl16, wd + 2 * w1r16, dhi, id1b, acc_in);
+              mma_f16_lo(acc + 2 * hs, xd + 3 * pl16, wd + 3 * w1r16, dhi, id1b, 1u);
+            }
+            mma_commit(&a1full[b]);
+            if (s == nS - 1) mma_commit(&xempty[xb]);
+          }
+          if (s >= 1) fc2(gs - 1, s - 1);
+        }
+        fc2(g + nS - 1, nS - 1);
+        if (ok) mma_commit(a2full);
+        g += nS;
+        if (++xb == p.nx) { xb = 0; xph ^= 1; }
+      }
+      // all MMAs (and hence all loads they consumed) complete before exit
+      mma_commit(final_bar);
+      mbar_wait(final_bar, 0);
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------- transform
+    const int r = threadIdx.x - 64;  // token row of the tile
+    int xb = 0;
+    uint32_t xph = 0;
+    for (int m = blockIdx.x; m < p.nM; m += gridDim.x) {
+      if (ok) ok = mbar_wait(&xfull[xb], xph);
+      uint8_t *xt = smem + L.x0 + xb * L.xtile;
+      for (int kc = 0; kc < P.nK1; ++kc) {
+        uint8_t *st = xt + kc * kMlpChunkBytes;
+        uint4 raw[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          raw[q] = *reinterpret_cast<const uint4 *>(st + r * 128 + ((q ^ (r & 7)) << 4));
+        uint32_t pl[4][8];  // [plane][channel pair]: V0, V2, Re V1, -Im V1
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rdft4_pair(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+        named_bar_sync(2, 128);  // every row read before the planes overwrite it
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          uint8_t *plane = st + pp * kMlpPlaneBytes + r * 32;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            *reinterpret_cast<uint4 *>(plane + (((h ^ (r >> 2)) & 1) << 4)) =
+                make_uint4(pl[pp][4 * h + 0], pl[pp][4 * h + 1], pl[pp][4 * h + 2],
+                           pl[pp][4 * h + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(&xready[xb]);
+      if (++xb == p.nx) { xb = 0; xph ^= 1; }
+    }
+  } else if (warp < 14) {
+    // --------------------------------------------------------------- GELU
+    // Team t takes the hidden slices gs with gs % 2 == t (fc1 accumulator and
+    // hidden buffer t).  Warp quadrant q = warp % 4 reads TMEM lanes 32q..32q+31,
+    // i.e. token rows row = 32q + lane.
+    const int team = (warp - 6) / 4;
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int groups = hs / 8;  // 8 hidden channels per step
+    int g = 0;
+    for (int m = blockIdx.x; m < p.nM; m += gridDim.x, g += nS) {
+      for (int s = 0; s < nS; ++s) {
+        const int gs = g + s;
+        if ((gs & 1) != team) continue;
+        const uint32_t bph = (gs >> 1) & 1;
+        if (ok) ok = mbar_wait(&a1full[team], bph);
+        if (ok) ok = mbar_wait(&hempty[team], bph ^ 1);
+        tc_fence_after();
+        const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + team * 4 * hs;
+        uint8_t *hb = smem + L.h0 + team * L.htile + row * 32;
+        const float *bias = sb1 + s * hs;
+        for (int c8 = 0; c8 < groups; ++c8) {
+          uint32_t y0[8], y2[8], yr[8], yi[8];
+          __syncwarp();
+          tmem_ld8(tl + c8 * 8, y0);
+          tmem_ld8(tl + hs + c8 * 8, y2);
+          tmem_ld8(tl + 2 * hs + c8 * 8, yr);
+          tmem_ld8(tl + 3 * hs + c8 * 8, yi);
+          tmem_ld_wait();
+          if (c8 == groups - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(&a1empty[team]);
+          }
+          // group values of the 8 channels (inverse rDFT + b1), GELU, as fp16 pairs
+          uint32_t ga[8], gb[8];  // (g0, g1), (g2, g3) of channel i
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+            const float Yr = __uint_as_float(yr[i]), Yi = __uint_as_float(yi[i]);
+            const float bv = bias[c8 * 8 + i];
+            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
+            ga[i] = gelu_h2(pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o)));
+            gb[i] = gelu_h2(pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o)));
+          }
+          // rDFT of the activations, channel pairs packed: fc2's four planes
+          uint32_t pl[4][4];
+#pragma unroll
+          for (int i2 = 0; i2 < 4; ++i2)
+            rdft4_pair(make_uint4(ga[2 * i2], gb[2 * i2], ga[2 * i2 + 1], gb[2 * i2 + 1]),
+                       pl[0][i2], pl[1][i2], pl[2][i2], pl[3][i2]);
+          uint8_t *dst = hb + (c8 >> 1) * kMlpChunkBytes + ((((c8 & 1) ^ (row >> 2)) & 1) << 4);
+#pragma unroll
+          for (int pp = 0; pp < 4; ++pp)
+            *reinterpret_cast<uint4 *>(dst + pp * kMlpPlaneBytes) =
+                make_uint4(pl[pp][0], pl[pp][1], pl[pp][2], pl[pp][3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(&hready[team]);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int ew = warp - 14;
+    uint8_t *obase = smem + L.y0 + ew * kMlpYBoxes * 4096;
+    const int groups = P.BD2 / 16;
+    int oi = 0, it = 0;
+    for (int m = blockIdx.x; m < p.nM; m += gridDim.x, ++it) {
+      if (ok) ok = mbar_wait(a2full, it & 1);
+      tc_fence_after();
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc2_col;
+      for (int grp = 0; grp < groups; ++grp) {
+        const int d0 = grp * 16;
+        uint32_t packed[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t y0[8], y2[8], yr[8], yi[8];
+          const uint32_t col = tl + d0 + h * 8;
+          __syncwarp();
+          tmem_ld8(col, y0);
+          tmem_ld8(col + P.BD2, y2);
+          tmem_ld8(col + 2 * P.BD2, yr);
+          tmem_ld8(col + 3 * P.BD2, yi);
+          tmem_ld_wait();
+          if (h == 1 && grp == groups - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(a2empty);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+            const float Yr = __uint_as_float(yr[i]), Yi = __uint_as_float(yi[i]);
+            const float bv = sb2[d0 + h * 8 + i];
+            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
+            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+          }
+        }
+        if (d0 >= P.Co) continue;  // whole group is padding
+        uint8_t *ob = obase + (oi % kMlpYBoxes) * 4096;
+        if (lane == 0) bulk_wait_read<kMlpYBoxes - 1>();  // this box's last store has read it
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4 *>(ob + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+              make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_out, d0 * kT, m * kBM + q * 32, ob);
+          bulk_commit();
+        }
+        ++oi;
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace feql

@@ -10,7 +10,8 @@ import torch
 from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward, feql_backward_dw,
                feql_backward_dw_workspace_bytes, feql_backward_dx, feql_ct_backward_dw,
                feql_ct_backward_dw_workspace_bytes, feql_ct_backward_dx, feql_ct_forward,
-               feql_ct_weight_fft, feql_ct_weight_fft_bytes, feql_forward, feql_weight_fft,
+               feql_ct_weight_fft, feql_ct_weight_fft_bytes, feql_forward, feql_mlp_forward,
+               feql_mlp_weight_fft, feql_mlp_weight_fft_bytes, feql_weight_fft,
                feql_weight_fft_bytes)
 
 
@@ -115,3 +116,24 @@ def ct_backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, with_db: bool =
     db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
     feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
     return dW, db
+
+
+# ------------------------------------------------------------ MLP block (p4)
+
+def mlp_weight_fft(W1: torch.Tensor, W2: torch.Tensor, mode: int, stream=None) -> torch.Tensor:
+    H, C, _ = W1.shape
+    Co = W2.shape[0]
+    nbytes = feql_mlp_weight_fft_bytes(C, H, Co, mode)
+    if nbytes == 0:
+        raise ValueError("unsupported (C, H, Co, mode) for the fused MLP block")
+    What = torch.empty(nbytes, dtype=torch.uint8, device=W1.device)
+    feql_mlp_weight_fft(W1, W2, What, C, H, Co, mode, stream)
+    return What
+
+
+def mlp_forward(x: torch.Tensor, What: torch.Tensor, b1, b2, H: int, Co: int, mode: int,
+                stream=None) -> torch.Tensor:
+    N, C, _ = x.shape
+    y = torch.empty((N, Co, 4), dtype=x.dtype, device=x.device)
+    feql_mlp_forward(x, What, b1, b2, y, N, C, H, Co, mode, stream)
+    return y

@@ -16,11 +16,17 @@ numpy's PCG64 generator and rounded (round-to-nearest-even) to the mode dtype:
 
 Seeds: 20260000 + 100 * workload_id + {x: 0, W: 1, b: 2, dy: 3}.
 
+MLP block (fc1: C -> H, GELU, fc2: H -> Co; p4): x ~ N(0, 1); W1 std
+1/(2 sqrt C), W2 std 1/(2 sqrt H) (the fan-ins 4C and 4H); b1, b2 std 0.02.
+Seeds: 20260000 + 100 * workload_id + {x: 0, W1: 1, b1: 2, W2: 4, b2: 5}.
+
 The shapes stand in for the token streams of the networks the paper
 evaluates (Flash EQ-ViT and Flash EQ-Swin, technical summary "Livello di
 Rete"): a ViT MLP fc1 at 64 x 197 tokens and a Swin stage-1 stream at
 128 x 3136 tokens; no dataset is involved.  The C_8 workload keeps the Swin
-stream's token count and unrolled widths (96 -> 384) with T = 8.
+stream's token count and unrolled widths (96 -> 384) with T = 8.  The MLP
+workload is the Swin-T stage-1 block (96 -> 384 -> 96 unrolled) on the same
+token stream.
 """
 
 from __future__ import annotations
@@ -58,6 +64,9 @@ WORKLOADS = {
     6: Workload(6, "c8_fwdbwd_fp16_swin_N401408_C12_D48", 401408, 12, 48, "fp16",
                 ("fwd", "dx", "dw"),
                 "cyclic group C_8, Swin stage-1-like stream (96->384 unrolled)", T=8),
+    7: Workload(7, "p4_mlp_fp16_swin_N401408_C24_H96", 401408, 24, 96, "fp16", ("mlp",),
+                "Swin stage-1-like MLP block fc1 -> GELU -> fc2 (96->384->96 unrolled); "
+                "D is the hidden width, the output has C channels"),
 }
 
 
@@ -97,3 +106,13 @@ def workload_inputs(wid: int, dtype: str | None = None, N: int | None = None,
                     which=("x", "W", "b", "dy")) -> dict:
     w = WORKLOADS[wid]
     return make_inputs(wid, w.N if N is None else N, w.C, w.D, dtype or w.dtype, which, T=w.T)
+
+
+def make_mlp_inputs(wid: int, N: int, C: int, H: int, Co: int, dtype: str) -> dict:
+    """Seeded, dtype-rounded inputs of the MLP block (x, W1, b1, W2, b2)."""
+    base = 20260000 + 100 * wid
+    return {"x": _normal(base + 0, (N, C, 4), 1.0, dtype),
+            "W1": _normal(base + 1, (H, C, 4), 1.0 / np.sqrt(4 * C), dtype),
+            "b1": _normal(base + 2, (H,), 0.02, dtype),
+            "W2": _normal(base + 4, (Co, H, 4), 1.0 / np.sqrt(4 * H), dtype),
+            "b2": _normal(base + 5, (Co,), 0.02, dtype)}

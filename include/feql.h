@@ -172,6 +172,31 @@ size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int d
 int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db, void *ws,
                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * p4-equivariant MLP block, forward (Flash EQ-Linear, technical summary
+ * "Livello di Rete": the EQ-ViT / EQ-Swin networks built from the layer; their
+ * MLP is two EQ-Linear layers around a pointwise GELU):
+ *   h[n,j,t] = b1[j] + sum_c sum_s W1[j,c,(t-s) mod 4] x[n,c,s]        fc1: C -> H
+ *   y[n,o,t] = b2[o] + sum_j sum_s W2[o,j,(t-s) mod 4] GELU(h[n,j,s])   fc2: H -> Co
+ * in one kernel: the hidden activation h never goes to device memory.  GELU is
+ * evaluated in its tanh form (within 5e-4 of the exact z*Phi(z)) on fp16 values.
+ *   x  : device [N][C][4]     y : device [N][Co][4] (written)
+ *   W1 : device [H][C][4]     b1: device [H] or NULL
+ *   W2 : device [Co][H][4]    b2: device [Co] or NULL
+ * FEQL_FP16 only (other modes FEQL_ERR_UNSUPPORTED).  C and Co even; Co <= 64;
+ * the Fourier weights of both layers must fit in shared memory beside the
+ * tile buffers (e.g. C = 24, H = 96, Co = 24, the Swin stage-1 block): shapes
+ * that do not fit return FEQL_ERR_UNSUPPORTED (feql_mlp_weight_fft_bytes
+ * returns 0 for them).  Conventions otherwise as above (device pointers,
+ * 16-byte alignment, stream-ordered, N == 0 is a no-op). */
+size_t feql_mlp_weight_fft_bytes(int C, int H, int Co, int dtype);
+/* Fourier weights of both layers in the kernel's tile layout (opaque; depends
+ * only on C, H, Co): What must hold feql_mlp_weight_fft_bytes(C, H, Co, dtype) bytes. */
+int feql_mlp_weight_fft(const void *W1, const void *W2, void *What, int C, int H, int Co,
+                        int dtype, feql_stream stream);
+int feql_mlp_forward(const void *x, const void *What, const void *b1, const void *b2, void *y,
+                     int64_t N, int C, int H, int Co, int dtype, feql_stream stream);
+
 /* Synchronises `stream`, then returns and clears the device-side status word
  * of the current device: FEQL_OK, or FEQL_ERR_TIMEOUT when some kernel gave up
  * on a bounded wait since the last call (its outputs are then undefined). */
