@@ -12,7 +12,10 @@ no flush is needed between steps.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 --workload selects another shape (workloads.py); workload 6 is the same stream
-for the cyclic group C_8 (feql_ct_* entry points, dX and dW as two passes).
+for the cyclic group C_8 (feql_ct_* entry points, dX and dW as two passes), and
+workload 7 the Swin stage-1 MLP block (fc1 -> GELU -> fc2, one fused kernel,
+feql_mlp_forward; its "unfused" line times the same block as fc1 forward, a
+torch GELU and fc2 forward, for context).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the full workload on
 its own tokens (weak scaling); the data-parallel weight gradient is summed
@@ -46,8 +49,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
-                    help="workload id 1-6 (group_dft_structured_b200/workloads.py; 6 is the "
-                         "cyclic group C_8)")
+                    help="workload id 1-7 (group_dft_structured_b200/workloads.py; 6 is the "
+                         "cyclic group C_8, 7 the MLP block)")
     ap.add_argument("--dtype", choices=["fp16", "fp32"], default=None,
                     help="override the workload's dtype (e.g. the fp32 run of the square layer)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -98,6 +101,14 @@ def workload_bytes(w, elt):
         "dw": x + y + T * D * C * elt + b,
         "bwd": x + y + what + x + T * D * C * elt + b,  # x, dy, What in; dx, dW, db out
     }
+
+
+def mlp_bytes(w, elt):
+    """Algorithmic HBM bytes of the fused MLP block: x in, y out, both layers'
+    weights (as real values) and biases; the hidden activation stays on chip."""
+    N, C, H = w.N, w.C, w.D
+    wts = 4 * H * C * elt * 2 + (H + C) * elt
+    return {"wfft": 2 * wts, "mlp": 4 * N * C * elt * 2 + wts}
 
 
 def layer_macs(w):
@@ -185,7 +196,14 @@ def time_oracle(w, n_sample):
     """Float64 oracle (unrolled dense method) for all passes on n_sample tokens."""
     import numpy as np
 
-    from group_dft_structured_b200.workloads import make_inputs
+    from group_dft_structured_b200.workloads import make_inputs, make_mlp_inputs
+    if "mlp" in w.passes:
+        from oracle import feql_mlp_oracle as M
+        inp = make_mlp_inputs(w.wid, n_sample, w.C, w.D, w.C, w.dtype)
+        f = {k: v.astype(np.float64) for k, v in inp.items()}
+        t0 = time.perf_counter()
+        M.forward(f["x"], f["W1"], f["b1"], f["W2"], f["b2"])
+        return time.perf_counter() - t0
     if w.T == 4:
         from oracle import feql_oracle as O
     else:
@@ -210,7 +228,8 @@ def cpu_baseline(w, target_s=3.0):
         t = time_oracle(w, n)
     return {"value": n / t, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
             "sample": f"{n} of {w.N} tokens, passes {'+'.join(w.passes)}, float64 numpy "
-                      f"(unrolled circulant), one timed run of {t:.2f} s"}
+                      f"(unrolled circulant{', exact GELU' if 'mlp' in w.passes else ''}), "
+                      f"one timed run of {t:.2f} s"}
 
 
 def run_reference(args, rank, world):
@@ -248,29 +267,9 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------- ours
-def main():
-    args = parse()
-    rank, world, local_rank = dist_env()
-    if args.impl == "reference":
-        return run_reference(args, rank, world)
-
-    import numpy as np
-    import torch
-    import torch.distributed as dist
-
-    import group_dft_structured_b200 as F
-    from group_dft_structured_b200.workloads import WORKLOADS, make_inputs
-
-    w = WORKLOADS[args.workload]
-    if args.dtype is not None:
-        import dataclasses
-        w = dataclasses.replace(w, dtype=args.dtype)
-    torch.cuda.set_device(local_rank)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-    F.load()
+def setup_layer(args, w, rank, s, F, torch):
+    """Buffers and calls of the EQ-Linear layer workloads (p4 and C_8)."""
+    from group_dft_structured_b200.workloads import make_inputs
     mode = F.FEQL_FP16 if w.dtype == "fp16" else F.FEQL_FP32
     N, C, D, T = w.N, w.C, w.D, w.T
     elt = 2 if w.dtype == "fp16" else 4
@@ -285,8 +284,6 @@ def main():
     db = torch.empty((D,), dtype=x.dtype, device="cuda")
     ws = torch.empty(max(F.feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode), 16),
                      dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
-    s = stream.cuda_stream
     # One step = every row of the path: weight rDFT, forward, and the backward
     # (dX and dW/db, fused into one pass over dy for p4 unless --separate-backward).
     calls = {
@@ -301,7 +298,112 @@ def main():
         passes.append("bwd")
     else:
         passes += [p for p in ("dx", "dw") if p in w.passes]
-    launches_per_step = {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2, "bwd": 2}
+    macs, dense_macs = layer_macs(w)
+    gemms = {"wfft": 0, "fwd": 1, "dx": 1, "dw": 1, "bwd": 2}  # layer contractions per pass
+    has_bwd = any(p in passes for p in ("dx", "dw", "bwd"))
+    ins = ["x", "W", "b"] + (["dy"] if has_bwd else [])
+    src = {"y": y, "dx": dx, "dW": dW, "db": db}
+    outs = [k for k in ("y", "dx", "dW", "db")
+            if (k == "y" and "fwd" in passes)
+            or (k == "dx" and ("dx" in passes or "bwd" in passes))
+            or (k in ("dW", "db") and ("dw" in passes or "bwd" in passes))]
+    return {
+        "calls": calls, "passes": passes, "tokens": N, "elt": elt,
+        "launches": {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2, "bwd": 2},
+        "bytes": workload_bytes(w, elt),
+        "flops": {p: (2 * macs * gemms[p], 2 * dense_macs * gemms[p]) for p in passes},
+        "host": {k: inp[k] for k in ins}, "dev": {k: dev[k] for k in ins},
+        "outs": {k: src[k] for k in outs},
+        "allreduce": (lambda: dp_allreduce_grads(dW, db)) if has_bwd else None,
+        "config": {"N": N, "C": C, "D": D, "T": T},
+        "extra": {},
+    }
+
+
+def setup_mlp(args, w, rank, s, F, torch):
+    """Buffers and calls of the fused MLP block (fc1 C -> H, GELU, fc2 H -> C)."""
+    import torch.nn.functional as TF
+
+    from group_dft_structured_b200.workloads import make_mlp_inputs
+    mode = F.FEQL_FP16
+    N, C, H, Co = w.N, w.C, w.D, w.C
+    inp = make_mlp_inputs(rank_seed_id(w.wid, rank), N, C, H, Co, w.dtype)
+    dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+    x, W1, b1, W2, b2 = (dev[k] for k in ("x", "W1", "b1", "W2", "b2"))
+    What = torch.empty(F.feql_mlp_weight_fft_bytes(C, H, Co, mode), dtype=torch.uint8,
+                       device="cuda")
+    y = torch.empty((N, Co, 4), dtype=x.dtype, device="cuda")
+    calls = {
+        "wfft": lambda: F.feql_mlp_weight_fft(W1, W2, What, C, H, Co, mode, s),
+        "mlp": lambda: F.feql_mlp_forward(x, What, b1, b2, y, N, C, H, Co, mode, s),
+    }
+    macs = 6 * N * H * (C + Co)
+    # context: the same block as three launches with the hidden activation in HBM
+    W1hat = torch.empty(F.feql_weight_fft_bytes(C, H, mode), dtype=torch.uint8, device="cuda")
+    W2hat = torch.empty(F.feql_weight_fft_bytes(H, Co, mode), dtype=torch.uint8, device="cuda")
+    F.feql_weight_fft(W1, W1hat, C, H, mode, s)
+    F.feql_weight_fft(W2, W2hat, H, Co, mode, s)
+    h = torch.empty((N, H, 4), dtype=x.dtype, device="cuda")
+    y2 = torch.empty_like(y)
+    stream = torch.cuda.current_stream()
+
+    def unfused():
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            F.feql_forward(x, W1hat, b1, h, N, C, H, mode, s)
+            g = TF.gelu(h)
+            F.feql_forward(g, W2hat, b2, y2, N, H, Co, mode, s)
+        a.record(stream)
+        reps = 20
+        for _ in range(reps):
+            F.feql_forward(x, W1hat, b1, h, N, C, H, mode, s)
+            g = TF.gelu(h)
+            F.feql_forward(g, W2hat, b2, y2, N, H, Co, mode, s)
+        z.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(z) / reps
+
+    return {
+        "calls": calls, "passes": ["wfft", "mlp"], "tokens": N, "elt": 2,
+        "launches": {"wfft": 1, "mlp": 1},
+        "bytes": mlp_bytes(w, 2),
+        "flops": {"wfft": (0, 0), "mlp": (2 * macs, 2 * 16 * N * H * (C + Co))},
+        "host": {k: inp[k] for k in ("x", "W1", "b1", "W2", "b2")},
+        "dev": {k: dev[k] for k in ("x", "W1", "b1", "W2", "b2")},
+        "outs": {"y": y},
+        "allreduce": None,
+        "config": {"N": N, "C": C, "H": H, "Co": Co, "T": 4, "gelu": "tanh form, fp16"},
+        "extra": {"unfused": unfused},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import group_dft_structured_b200 as F
+    from group_dft_structured_b200.workloads import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.dtype is not None:
+        import dataclasses
+        w = dataclasses.replace(w, dtype=args.dtype)
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    F.load()
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    job = (setup_mlp if "mlp" in w.passes else setup_layer)(args, w, rank, s, F, torch)
+    calls, passes, N = job["calls"], job["passes"], job["tokens"]
 
     def step(ev=None):
         if ev is not None:
@@ -310,8 +412,8 @@ def main():
             calls[p]()
             if ev is not None:
                 ev[i + 1].record(stream)
-        if world > 1:
-            dp_allreduce_grads(dW, db)
+        if world > 1 and job["allreduce"] is not None:
+            job["allreduce"]()
 
     def barrier():
         if world > 1:
@@ -349,30 +451,17 @@ def main():
     # ---------------------------------------------------------- e2e (host buffers)
     e2e = None
     if not args.no_e2e:
-        hin = {k: torch.from_numpy(v).pin_memory() for k, v in inp.items()}
-        hout = {"y": torch.empty_like(y, device="cpu").pin_memory(),
-                "dx": torch.empty_like(dx, device="cpu").pin_memory(),
-                "dW": torch.empty_like(dW, device="cpu").pin_memory(),
-                "db": torch.empty_like(db, device="cpu").pin_memory()}
-        has_bwd = any(p in passes for p in ("dx", "dw", "bwd"))
-        h2d = sum(hin[k].numel() * hin[k].element_size() for k in ("x", "W", "b")) + \
-            (hin["dy"].numel() * hin["dy"].element_size() if has_bwd else 0)
-        outs = [k for k in ("y", "dx", "dW", "db")
-                if (k == "y" and "fwd" in passes)
-                or (k == "dx" and ("dx" in passes or "bwd" in passes))
-                or (k in ("dW", "db") and ("dw" in passes or "bwd" in passes))]
-        d2h = sum(hout[k].numel() * hout[k].element_size() for k in outs)
-        src = {"y": y, "dx": dx, "dW": dW, "db": db}
+        hin = {k: torch.from_numpy(v).pin_memory() for k, v in job["host"].items()}
+        hout = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in job["outs"].items()}
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
 
         def e2e_step():
-            x.copy_(hin["x"], non_blocking=True)
-            W.copy_(hin["W"], non_blocking=True)
-            b.copy_(hin["b"], non_blocking=True)
-            if has_bwd:
-                dy.copy_(hin["dy"], non_blocking=True)
+            for k, t in hin.items():
+                job["dev"][k].copy_(t, non_blocking=True)
             step()
-            for k in outs:
-                hout[k].copy_(src[k], non_blocking=True)
+            for k, t in hout.items():
+                t.copy_(job["outs"][k], non_blocking=True)
 
         e2e_step()
         barrier()
@@ -388,6 +477,9 @@ def main():
         e2e = {"value": N * world * args.e2e_steps / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps}
+    extra = {}
+    if rank == 0 and "unfused" in job["extra"]:
+        extra["unfused_ms"] = round(job["extra"]["unfused"](), 5)
 
     if world > 1:
         dist.barrier()
@@ -398,20 +490,17 @@ def main():
     # ------------------------------------------------------------- report
     value = N * world * args.steps / (ms * 1e-3)
     peak, peak_src = measured_peaks()
-    nbytes = workload_bytes(w, elt)
-    macs, dense_macs = layer_macs(w)
+    nbytes = job["bytes"]
     mean_ms = {p: float(np.mean(v)) for p, v in per_pass.items()}
-    gemm_passes = {"wfft": 0, "fwd": 1, "dx": 1, "dw": 1, "bwd": 2}  # layer contractions per pass
     pass_report = {}
     for p in passes:
         gbs = nbytes[p] / (mean_ms[p] * 1e-3) / 1e9
         pass_report[p] = {"ms": round(mean_ms[p], 5), "GB_s": round(gbs, 1),
                           "frac_hbm": round(gbs / peak, 4), "algorithmic_bytes": nbytes[p]}
-        if p != "wfft":
-            g = gemm_passes[p]
-            pass_report[p]["alg_TFLOP_s"] = round(2 * macs * g / (mean_ms[p] * 1e-3) / 1e12, 2)
-            pass_report[p]["dense_equiv_TFLOP_s"] = round(
-                2 * dense_macs * g / (mean_ms[p] * 1e-3) / 1e12, 2)
+        alg, dense = job["flops"][p]
+        if alg:
+            pass_report[p]["alg_TFLOP_s"] = round(alg / (mean_ms[p] * 1e-3) / 1e12, 2)
+            pass_report[p]["dense_equiv_TFLOP_s"] = round(dense / (mean_ms[p] * 1e-3) / 1e12, 2)
     dom = max((p for p in passes if p != "wfft"), key=lambda p: mean_ms[p])
     achieved = nbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
     traffic = None
@@ -421,7 +510,7 @@ def main():
             tj = json.load(f)
         if tj.get("source_hash") == kernel_source_hash():
             traffic = tj.get(w.name, {}).get(dom)
-    nkern = sum(launches_per_step[p] for p in passes)
+    nkern = sum(job["launches"][p] for p in passes)
     step_ms = ms / args.steps
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -429,12 +518,12 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16" if w.dtype == "fp16" else "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "N": N, "C": C, "D": D, "T": T,
-                   "passes": passes, "accumulate": "f32", "l2": "inputs larger than L2, no flush",
-                   "global_tokens": N * world,
-                   "parallelism": f"dp{world}" if world > 1 else "single"},
-        "effective_TFLOP_s": round(2 * dense_macs * sum(gemm_passes[p] for p in passes)
-                                   * world / (step_ms * 1e-3) / 1e12, 2),
+        "config": dict({"workload": w.name}, **job["config"],
+                       passes=passes, accumulate="f32", l2="inputs larger than L2, no flush",
+                       global_tokens=N * world,
+                       parallelism=f"dp{world}" if world > 1 else "single"),
+        "effective_TFLOP_s": round(sum(job["flops"][p][1] for p in passes) * world
+                                   / (step_ms * 1e-3) / 1e12, 2),
         "roofline_pct_step": round(100 * sum(nbytes[p] for p in passes) / (step_ms * 1e-3) / 1e9
                                    / peak, 2),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
@@ -445,11 +534,11 @@ def main():
         "clocks": clk,
         "e2e": e2e,
     }
+    line.update(extra)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))
     return 0
-
 
 if __name__ == "__main__":
     sys.exit(main())
