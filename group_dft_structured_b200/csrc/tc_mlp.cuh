@@ -28,9 +28,10 @@
 //                 planes in one of two hidden buffers
 //   warps 14..17  fc2 epilogue: inverse rDFT + b2, TMA stores of y
 // TMEM: fc1 accumulators 2 x 4*HS columns (Y0 | Y2 | Re Y1 | Im Y1 of a
-// slice), fc2 accumulator 4*BD2 columns at 8*HS.
-// Issue order per tile: fc1(0), fc1(1), fc2(0), fc1(2), fc2(1), ..., fc2(nS-1),
-// so the GELU of one slice overlaps the MMAs of the next.
+// slice), fc2 accumulators (one or two, by tile) of 4*BD2 columns from 8*HS.
+// Issue order over the CTA's hidden slices gs (tile-major, across tiles):
+// fc1(0), fc1(1), fc2(0), fc1(2), fc2(1), ..., so the GELU of one slice
+// overlaps the fc1 MMAs of the next, also at tile boundaries.
 // Every wait is bounded (mbar_wait); a timed-out thread stops issuing work but
 // keeps the loop structure so named barriers stay matched.
 #pragma once
@@ -84,6 +85,9 @@ __host__ __device__ inline MlpPlan make_mlp_plan(int C, int H, int Co, int hs_ma
 }
 
 // Weight transform of both layers: one thread per fp16 element of the buffer.
+// fc1's bins carry the inverse transform's scales and the 1/2 of GELU: bins 0
+// and 2 are stored times 1/8, bin 1 times 1/4 (powers of two: exact), so its
+// accumulators give u_t = h_t / 2 with sums and differences alone.
 __global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__restrict__ W2,
                                 uint8_t *__restrict__ What, MlpPlan P) {
   const int64_t n1 = P.w1_bytes / 2, n2 = P.w2_bytes / 2;
@@ -114,6 +118,7 @@ __global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__r
       float b0, b2, b1r, b1i;
       weight_bins(first ? W1 : W2, Ci, 0, o, i, b0, b2, b1r, b1i);
       v = sub == 0 ? b0 : sub == 1 ? b2 : sub == 2 ? b1r : sub == 3 ? b1i : -b1r;
+      if (first) v *= sub < 2 ? 0.125f : 0.25f;
     }
     const int64_t base = first ? chunk * P.w1_chunk : P.off_w2 + chunk * P.w2_chunk;
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);
@@ -151,8 +156,12 @@ __host__ __device__ inline MlpSmem mlp_smem(const TcMlpParams &p) {
   return s;
 }
 
-// TMEM columns the block needs: two fc1 accumulators and the fc2 accumulator.
+// TMEM columns the block needs: two fc1 accumulators and one fc2 accumulator;
+// a second fc2 accumulator is used when it fits.
 __host__ __device__ inline int mlp_tmem_cols(const MlpPlan &P) { return 8 * P.HS + 4 * P.BD2; }
+__host__ __device__ inline int mlp_acc2_buffers(const MlpPlan &P) {
+  return 8 * P.HS + 8 * P.BD2 <= 512 ? 2 : 1;
+}
 
 __device__ __forceinline__ uint32_t tanh_h2(uint32_t x) {
   uint32_t y;
@@ -160,16 +169,14 @@ __device__ __forceinline__ uint32_t tanh_h2(uint32_t x) {
   return y;
 }
 
-// GELU (tanh form) of a packed fp16 pair.
-__device__ __forceinline__ uint32_t gelu_h2(uint32_t zu) {
-  const __half2 z = as_h2(zu);
-  const __half2 k0 = __float2half2_rn(0.7978845608028654f);   // sqrt(2/pi)
-  const __half2 k1 = __float2half2_rn(0.0356774081363001f);   // 0.044715 sqrt(2/pi)
-  const __half2 hf = __float2half2_rn(0.5f);
-  const __half2 u = __hmul2(z, __hfma2(k1, __hmul2(z, z), k0));
-  const __half2 t = as_h2(tanh_h2(as_u32(u)));
-  const __half2 hz = __hmul2(hf, z);
-  return as_u32(__hfma2(hz, t, hz));
+// GELU (tanh form) of z = 2u for a packed fp16 pair u:
+//   GELU(2u) = u (1 + tanh(2 k0 u + 8 k1 u^3)),  k0 = sqrt(2/pi), k1 = 0.044715 k0.
+__device__ __forceinline__ uint32_t gelu_half_arg_h2(uint32_t uu) {
+  const __half2 u = as_h2(uu);
+  const __half2 c0 = __float2half2_rn(1.5957691216057308f);  // 2 sqrt(2/pi)
+  const __half2 c1 = __float2half2_rn(0.2854192650904008f);  // 8 * 0.044715 sqrt(2/pi)
+  const __half2 t = as_h2(tanh_h2(as_u32(__hmul2(u, __hfma2(c1, __hmul2(u, u), c0)))));
+  return as_u32(__hfma2(u, t, u));
 }
 
 // 18 warps: 5 on one register slice of an SM sub-partition, 96 registers each.
@@ -188,7 +195,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
   uint64_t *xfull = bars + 1, *xready = bars + 3, *xempty = bars + 5;
   uint64_t *a1full = bars + 7, *a1empty = bars + 9;
   uint64_t *hready = bars + 11, *hempty = bars + 13;
-  uint64_t *a2full = bars + 15, *a2empty = bars + 16, *final_bar = bars + 17;
+  uint64_t *a2full = bars + 15, *a2empty = bars + 17, *final_bar = bars + 19;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -205,13 +212,15 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       mbar_init(&hready[b], 4);
       mbar_init(&hempty[b], 1);
     }
-    mbar_init(a2full, 1);
-    mbar_init(a2empty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&a2full[b], 1);
+      mbar_init(&a2empty[b], 4);
+    }
     mbar_init(final_bar, 1);
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < nS * hs; i += blockDim.x)
-    sb1[i] = (p.b1 != nullptr && i < P.H) ? __half2float(p.b1[i]) : 0.f;
+  for (int i = threadIdx.x; i < nS * hs; i += blockDim.x)  // b1 / 2, like fc1's accumulators
+    sb1[i] = (p.b1 != nullptr && i < P.H) ? 0.5f * __half2float(p.b1[i]) : 0.f;
   for (int i = threadIdx.x; i < P.BD2; i += blockDim.x)
     sb2[i] = (p.b2 != nullptr && i < P.Co) ? __half2float(p.b2[i]) : 0.f;
   if (warp == 1) {
@@ -222,7 +231,12 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t acc2_col = 8 * hs;
+  const uint32_t acc2_col = 8 * hs;  // fc2 accumulator buffer a at acc2_col + a * 4 * BD2
+  const int nacc2 = mlp_acc2_buffers(P);
+  // this CTA's tiles m = blockIdx.x + i * gridDim.x, i < n_my; hidden slices gs = i * nS + s
+  const int n_my = static_cast<int>(blockIdx.x) < p.nM
+                       ? (p.nM - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                       : 0;
   bool ok = true;
 
   if (warp == 0) {
@@ -264,59 +278,53 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       const uint32_t xt16 = L.xtile >> 4, ht16 = L.htile >> 4;
       const uint32_t w1r16 = (hs * 32) >> 4, w1c16 = P.w1_chunk >> 4;
       const uint32_t w2r16 = (P.BD2 * 32) >> 4, w2c16 = P.w2_chunk >> 4;
-      const uint32_t acc2 = tmem_base + acc2_col;
       const int kh_per = hs / kCK;
       if (static_cast<int>(blockIdx.x) < p.nM) ok = mbar_wait(wfull, 0);
-      int xb = 0;
-      uint32_t xph = 0;
-      int g = 0;  // hidden slices issued so far (selects the fc1/hidden buffer)
-      int it = 0;
-      // fc2 over hidden slice s of this tile, slice gs overall
-      auto fc2 = [&](int gs, int s) {
-        const int b = gs & 1;
-        const uint32_t bph = (gs >> 1) & 1;
-        if (s == 0 && ok) ok = mbar_wait(a2empty, (it & 1) ^ 1);
-        if (ok) ok = mbar_wait(&hready[b], bph);
+      // fc1 of hidden slice gs: its x tile (ready once per tile), fc1 accumulator gs % 2
+      auto fc1 = [&](int gs) {
+        const int i = gs / nS, s = gs % nS, b = gs & 1, xb = i % p.nx;
+        if (s == 0 && ok) ok = mbar_wait(&xready[xb], (i / p.nx) & 1);
+        if (ok) ok = mbar_wait(&a1empty[b], ((gs >> 1) & 1) ^ 1);
         tc_fence_after();
-        if (ok) {
-          uint32_t hd = h0 + b * ht16, wd = w2_0 + s * kh_per * w2c16;
-          for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
-            const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
-            mma_f16_lo(acc2, hd, wd, dhi, id2a, acc_in);
-            mma_f16_lo(acc2 + P.BD2, hd + pl16, wd + w2r16, dhi, id2a, acc_in);
-            mma_f16_lo(acc2 + 2 * P.BD2, hd + 2 * pl16, wd + 2 * w2r16, dhi, id2b, acc_in);
-            mma_f16_lo(acc2 + 2 * P.BD2, hd + 3 * pl16, wd + 3 * w2r16, dhi, id2b, 1u);
-          }
-          mma_commit(&hempty[b]);
+        if (!ok) return;
+        const uint32_t acc = tmem_base + b * 4 * hs;
+        uint32_t xd = x0 + xb * xt16, wd = w1_0 + s * P.nK1 * w1c16;
+        for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
+          const uint32_t acc_in = kc > 0 ? 1u : 0u;
+          mma_f16_lo(acc, xd, wd, dhi, id1a, acc_in);
+          mma_f16_lo(acc + hs, xd + pl16, wd + w1r16, dhi, id1a, acc_in);
+          mma_f16_lo(acc + 2 * hs, xd + 2 * pl16, wd + 2 * w1r16, dhi, id1b, acc_in);
+          mma_f16_lo(acc + 2 * hs, xd + 3 * pl16, wd + 3 * w1r16, dhi, id1b, 1u);
         }
+        mma_commit(&a1full[b]);
+        if (s == nS - 1) mma_commit(&xempty[xb]);
       };
-      for (int m = blockIdx.x; m < p.nM; m += gridDim.x, ++it) {
-        if (ok) ok = mbar_wait(&xready[xb], xph);
+      // fc2 over the activations of slice gs into fc2 accumulator (tile % nacc2)
+      auto fc2 = [&](int gs) {
+        const int i = gs / nS, s = gs % nS, b = gs & 1, a = i % nacc2;
+        if (s == 0 && ok) ok = mbar_wait(&a2empty[a], ((i / nacc2) & 1) ^ 1);
+        if (ok) ok = mbar_wait(&hready[b], (gs >> 1) & 1);
         tc_fence_after();
-        for (int s = 0; s < nS; ++s) {
-          const int gs = g + s, b = gs & 1;
-          const uint32_t bph = (gs >> 1) & 1;
-          if (ok) ok = mbar_wait(&a1empty[b], bph ^ 1);
-          tc_fence_after();
-          if (ok) {
-            const uint32_t acc = tmem_base + b * 4 * hs;
-            uint32_t xd = x0 + xb * xt16, wd = w1_0 + s * P.nK1 * w1c16;
-            for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
-              const uint32_t acc_in = kc > 0 ? 1u : 0u;
-              mma_f16_lo(acc, xd, wd, dhi, id1a, acc_in);
-              mma_f16_lo(acc + hs, xd + pl16, wd + w1r16, dhi, id1a, acc_in);
-              mma_f16_lo(acc + 2 * hs, xd + 2 * pl16, wd + 2 * w1r16, dhi, id1b, acc_in);
-              mma_f16_lo(acc + 2 * hs, xd + 3 * pl16, wd + 3 * w1r16, dhi, id1b, 1u);
-            }
-            mma_commit(&a1full[b]);
-            if (s == nS - 1) mma_commit(&xempty[xb]);
-          }
-          if (s >= 1) fc2(gs - 1, s - 1);
+        if (!ok) return;
+        const uint32_t acc2 = tmem_base + acc2_col + a * 4 * P.BD2;
+        uint32_t hd = h0 + b * ht16, wd = w2_0 + s * kh_per * w2c16;
+        for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
+          const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
+          mma_f16_lo(acc2, hd, wd, dhi, id2a, acc_in);
+          mma_f16_lo(acc2 + P.BD2, hd + pl16, wd + w2r16, dhi, id2a, acc_in);
+          mma_f16_lo(acc2 + 2 * P.BD2, hd + 2 * pl16, wd + 2 * w2r16, dhi, id2b, acc_in);
+          mma_f16_lo(acc2 + 2 * P.BD2, hd + 3 * pl16, wd + 3 * w2r16, dhi, id2b, 1u);
         }
-        fc2(g + nS - 1, nS - 1);
-        if (ok) mma_commit(a2full);
-        g += nS;
-        if (++xb == p.nx) { xb = 0; xph ^= 1; }
+        mma_commit(&hempty[b]);
+        if (s == nS - 1) mma_commit(&a2full[a]);
+      };
+      // fc1 runs one slice ahead of fc2, across tile boundaries, so the GELU of
+      // slice gs overlaps the fc1 MMAs of slice gs + 1
+      const int total = n_my * nS;
+      if (total > 0) fc1(0);
+      for (int gs = 0; gs < total; ++gs) {
+        if (gs + 1 < total) fc1(gs + 1);
+        fc2(gs);
       }
       // all MMAs (and hence all loads they consumed) complete before exit
       mma_commit(final_bar);
@@ -389,16 +397,17 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&a1empty[team]);
           }
-          // group values of the 8 channels (inverse rDFT + b1), GELU, as fp16 pairs
+          // half the group values of the 8 channels (inverse rDFT + b1, scales
+          // folded into the weights), then GELU, as fp16 pairs
           uint32_t ga[8], gb[8];  // (g0, g1), (g2, g3) of channel i
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-            const float Yr = __uint_as_float(yr[i]), Yi = __uint_as_float(yi[i]);
-            const float bv = bias[c8 * 8 + i];
-            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
-            ga[i] = gelu_h2(pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o)));
-            gb[i] = gelu_h2(pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o)));
+            const float A0 = __uint_as_float(y0[i]), A2 = __uint_as_float(y2[i]);
+            const float Ar = __uint_as_float(yr[i]), Ai = __uint_as_float(yi[i]);
+            const float pb = A0 + bias[c8 * 8 + i];
+            const float e = pb + A2, o = pb - A2;
+            ga[i] = gelu_half_arg_h2(pack_half2(e + Ar, o - Ai));
+            gb[i] = gelu_half_arg_h2(pack_half2(e - Ar, o + Ai));
           }
           // rDFT of the activations, channel pairs packed: fc2's four planes
           uint32_t pl[4][4];
@@ -425,9 +434,11 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     const int groups = P.BD2 / 16;
     int oi = 0, it = 0;
     for (int m = blockIdx.x; m < p.nM; m += gridDim.x, ++it) {
-      if (ok) ok = mbar_wait(a2full, it & 1);
+      const int a = it % nacc2;
+      if (ok) ok = mbar_wait(&a2full[a], (it / nacc2) & 1);
       tc_fence_after();
-      const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc2_col;
+      const uint32_t tl =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc2_col + a * 4 * P.BD2;
       for (int grp = 0; grp < groups; ++grp) {
         const int d0 = grp * 16;
         uint32_t packed[32];
@@ -444,7 +455,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           if (h == 1 && grp == groups - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(a2empty);
+            if (lane == 0 && ok) mbar_arrive(&a2empty[a]);
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
