@@ -199,6 +199,16 @@ __device__ __forceinline__ void mma_f16_lo(uint32_t d_tmem, uint32_t a_lo, uint3
 }
 
 // Low / high 32-bit words of a shared-memory descriptor.
+// One lane of a converged warp (elect.sync).  An issue loop run by the whole
+// warp keeps its descriptors warp-uniform; only the elected lane issues.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .b32 r;\n\t.reg .pred p;\n\telect.sync r|p, 0xffffffff;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ uint32_t desc_lo(uint64_t d) { return static_cast<uint32_t>(d); }
 __device__ __forceinline__ uint32_t desc_hi(uint64_t d) { return static_cast<uint32_t>(d >> 32); }
 

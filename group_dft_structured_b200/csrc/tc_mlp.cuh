@@ -264,7 +264,9 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the issue loop (its descriptors stay warp-uniform);
+    // one elected lane issues each MMA and commit.
+    {
       const uint32_t id1a = instr_desc(kBM, hs, 0, 0), id1b = instr_desc(kBM, 2 * hs, 0, 0);
       const uint32_t id2a = instr_desc(kBM, P.BD2, 0, 0);
       const uint32_t id2b = instr_desc(kBM, 2 * P.BD2, 0, 0);
@@ -279,44 +281,66 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       const uint32_t w1r16 = (hs * 32) >> 4, w1c16 = P.w1_chunk >> 4;
       const uint32_t w2r16 = (P.BD2 * 32) >> 4, w2c16 = P.w2_chunk >> 4;
       const int kh_per = hs / kCK;
-      if (static_cast<int>(blockIdx.x) < p.nM) ok = mbar_wait(wfull, 0);
+      if (static_cast<int>(blockIdx.x) < p.nM) ok = __all_sync(0xffffffffu, mbar_wait(wfull, 0));
+      // The issuing thread's scalar work adds to every MMA, so the two cursors
+      // below advance by increments (no divisions).
+      int s1 = 0, xb = 0;      // fc1 cursor: slice s1 of the tile in x buffer xb
+      uint32_t xph = 0;
+      int s2 = 0, ab = 0;      // fc2 cursor: slice s2 of the tile in fc2 accumulator ab
+      uint32_t abph = 0;
       // fc1 of hidden slice gs: its x tile (ready once per tile), fc1 accumulator gs % 2
       auto fc1 = [&](int gs) {
-        const int i = gs / nS, s = gs % nS, b = gs & 1, xb = i % p.nx;
-        if (s == 0 && ok) ok = mbar_wait(&xready[xb], (i / p.nx) & 1);
+        const int b = gs & 1, s = s1, x = xb;
+        if (s == 0 && ok) ok = mbar_wait(&xready[x], xph);
         if (ok) ok = mbar_wait(&a1empty[b], ((gs >> 1) & 1) ^ 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (++s1 == nS) {
+          s1 = 0;
+          if (++xb == p.nx) { xb = 0; xph ^= 1; }
+        }
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc = tmem_base + b * 4 * hs;
-        uint32_t xd = x0 + xb * xt16, wd = w1_0 + s * P.nK1 * w1c16;
-        for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
-          const uint32_t acc_in = kc > 0 ? 1u : 0u;
-          mma_f16_lo(acc, xd, wd, dhi, id1a, acc_in);
-          mma_f16_lo(acc + hs, xd + pl16, wd + w1r16, dhi, id1a, acc_in);
-          mma_f16_lo(acc + 2 * hs, xd + 2 * pl16, wd + 2 * w1r16, dhi, id1b, acc_in);
-          mma_f16_lo(acc + 2 * hs, xd + 3 * pl16, wd + 3 * w1r16, dhi, id1b, 1u);
+        uint32_t xd = x0 + x * xt16, wd = w1_0 + s * P.nK1 * w1c16;
+        if (elect_one()) {
+          for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
+            const uint32_t acc_in = kc > 0 ? 1u : 0u;
+            mma_f16_lo(acc, xd, wd, dhi, id1a, acc_in);
+            mma_f16_lo(acc + hs, xd + pl16, wd + w1r16, dhi, id1a, acc_in);
+            mma_f16_lo(acc + 2 * hs, xd + 2 * pl16, wd + 2 * w1r16, dhi, id1b, acc_in);
+            mma_f16_lo(acc + 2 * hs, xd + 3 * pl16, wd + 3 * w1r16, dhi, id1b, 1u);
+          }
+          mma_commit(&a1full[b]);
+          if (s == nS - 1) mma_commit(&xempty[x]);
         }
-        mma_commit(&a1full[b]);
-        if (s == nS - 1) mma_commit(&xempty[xb]);
+        __syncwarp();
       };
       // fc2 over the activations of slice gs into fc2 accumulator (tile % nacc2)
       auto fc2 = [&](int gs) {
-        const int i = gs / nS, s = gs % nS, b = gs & 1, a = i % nacc2;
-        if (s == 0 && ok) ok = mbar_wait(&a2empty[a], ((i / nacc2) & 1) ^ 1);
+        const int b = gs & 1, s = s2, a = ab;
+        if (s == 0 && ok) ok = mbar_wait(&a2empty[a], abph ^ 1);
         if (ok) ok = mbar_wait(&hready[b], (gs >> 1) & 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (++s2 == nS) {
+          s2 = 0;
+          if (++ab == nacc2) { ab = 0; abph ^= 1; }
+        }
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc2 = tmem_base + acc2_col + a * 4 * P.BD2;
         uint32_t hd = h0 + b * ht16, wd = w2_0 + s * kh_per * w2c16;
-        for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
-          const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
-          mma_f16_lo(acc2, hd, wd, dhi, id2a, acc_in);
-          mma_f16_lo(acc2 + P.BD2, hd + pl16, wd + w2r16, dhi, id2a, acc_in);
-          mma_f16_lo(acc2 + 2 * P.BD2, hd + 2 * pl16, wd + 2 * w2r16, dhi, id2b, acc_in);
-          mma_f16_lo(acc2 + 2 * P.BD2, hd + 3 * pl16, wd + 3 * w2r16, dhi, id2b, 1u);
+        if (elect_one()) {
+          for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
+            const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
+            mma_f16_lo(acc2, hd, wd, dhi, id2a, acc_in);
+            mma_f16_lo(acc2 + P.BD2, hd + pl16, wd + w2r16, dhi, id2a, acc_in);
+            mma_f16_lo(acc2 + 2 * P.BD2, hd + 2 * pl16, wd + 2 * w2r16, dhi, id2b, acc_in);
+            mma_f16_lo(acc2 + 2 * P.BD2, hd + 3 * pl16, wd + 3 * w2r16, dhi, id2b, 1u);
+          }
+          mma_commit(&hempty[b]);
+          if (s == nS - 1) mma_commit(&a2full[a]);
         }
-        mma_commit(&hempty[b]);
-        if (s == nS - 1) mma_commit(&a2full[a]);
+        __syncwarp();
       };
       // fc1 runs one slice ahead of fc2, across tile boundaries, so the GELU of
       // slice gs overlaps the fc1 MMAs of slice gs + 1
@@ -327,7 +351,8 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
         fc2(gs);
       }
       // all MMAs (and hence all loads they consumed) complete before exit
-      mma_commit(final_bar);
+      if (elect_one()) mma_commit(final_bar);
+      __syncwarp();
       mbar_wait(final_bar, 0);
     }
   } else if (warp < 6) {
