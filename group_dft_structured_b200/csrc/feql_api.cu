@@ -456,13 +456,14 @@ int launch_ct8_dw(const void *x, const void *dy, __half *dW, __half *db, float *
 constexpr int kMlpSmemBudget = 227 * 1024 - 1024;
 
 // The plan depends only on (C, H, Co), so the weight buffer's layout does too:
-// the widest hidden slice whose two fc1 accumulators and the fc2 accumulator
-// fit 512 TMEM columns, with two x tile buffers if they fit, else one.
+// the widest hidden slice (fewest fc1 MMAs: the kernel is bound by its MMA
+// issue) whose two fc1 accumulators and the fc2 accumulator fit 512 TMEM
+// columns, with two x tile buffers if they fit, else one.
 int plan_mlp(int C, int H, int Co, TcMlpParams *out) {
   if (align_up(Co, 16) > 64) return FEQL_ERR_UNSUPPORTED;
   const int hs_opts[4] = {64, 48, 32, 16};
-  for (int nx = 2; nx >= 1; --nx) {
-    for (int hs_max : hs_opts) {
+  for (int hs_max : hs_opts) {
+    for (int nx = 2; nx >= 1; --nx) {
       TcMlpParams p;
       p.P = make_mlp_plan(C, H, Co, hs_max);
       p.nx = nx;

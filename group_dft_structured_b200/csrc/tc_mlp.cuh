@@ -23,9 +23,9 @@
 //   warp 1        TMEM allocator + single-thread MMA issuer
 //   warps 2..5    transform: rDFT of the x tile in place into four K-major
 //                 planes per chunk (V0, V2, Re V1, -Im V1)
-//   warps 6..13   two GELU teams, one per fc1 accumulator buffer: hidden slice
-//                 of HS channels -> inverse rDFT + b1 -> GELU -> rDFT -> fp16
-//                 planes in one of two hidden buffers
+//   warps 6..13   GELU: per hidden slice of HS channels (two warps per TMEM
+//                 lane quadrant, half the channels each) inverse rDFT + b1 ->
+//                 GELU -> rDFT -> fp16 planes in one of two hidden buffers
 //   warps 14..17  fc2 epilogue: inverse rDFT + b2, TMA stores of y
 // TMEM: fc1 accumulators 2 x 4*HS columns (Y0 | Y2 | Re Y1 | Im Y1 of a
 // slice), fc2 accumulators (one or two, by tile) of 4*BD2 columns from 8*HS.
@@ -208,8 +208,8 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       mbar_init(&xready[b], 4);
       mbar_init(&xempty[b], 1);
       mbar_init(&a1full[b], 1);
-      mbar_init(&a1empty[b], 4);
-      mbar_init(&hready[b], 4);
+      mbar_init(&a1empty[b], 8);
+      mbar_init(&hready[b], 8);
       mbar_init(&hempty[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -390,26 +390,27 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     }
   } else if (warp < 14) {
     // --------------------------------------------------------------- GELU
-    // Team t takes the hidden slices gs with gs % 2 == t (fc1 accumulator and
-    // hidden buffer t).  Warp quadrant q = warp % 4 reads TMEM lanes 32q..32q+31,
-    // i.e. token rows row = 32q + lane.
-    const int team = (warp - 6) / 4;
+    // All eight warps take every hidden slice gs (fc1 accumulator and hidden
+    // buffer gs % 2): warp quadrant q = warp % 4 reads TMEM lanes 32q..32q+31,
+    // i.e. token rows row = 32q + lane, and each of the two warps of a
+    // quadrant takes half of the slice's 8-channel groups.
+    const int half = (warp - 6) / 4;
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const int groups = hs / 8;  // 8 hidden channels per step
+    const int c8_0 = half * (groups / 2), c8_1 = c8_0 + groups / 2;
     int g = 0;
     for (int m = blockIdx.x; m < p.nM; m += gridDim.x, g += nS) {
       for (int s = 0; s < nS; ++s) {
-        const int gs = g + s;
-        if ((gs & 1) != team) continue;
+        const int gs = g + s, b = gs & 1;
         const uint32_t bph = (gs >> 1) & 1;
-        if (ok) ok = mbar_wait(&a1full[team], bph);
-        if (ok) ok = mbar_wait(&hempty[team], bph ^ 1);
+        if (ok) ok = mbar_wait(&a1full[b], bph);
+        if (ok) ok = mbar_wait(&hempty[b], bph ^ 1);
         tc_fence_after();
-        const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + team * 4 * hs;
-        uint8_t *hb = smem + L.h0 + team * L.htile + row * 32;
+        const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * 4 * hs;
+        uint8_t *hb = smem + L.h0 + b * L.htile + row * 32;
         const float *bias = sb1 + s * hs;
-        for (int c8 = 0; c8 < groups; ++c8) {
+        for (int c8 = c8_0; c8 < c8_1; ++c8) {
           uint32_t y0[8], y2[8], yr[8], yi[8];
           __syncwarp();
           tmem_ld8(tl + c8 * 8, y0);
@@ -417,10 +418,10 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           tmem_ld8(tl + 2 * hs + c8 * 8, yr);
           tmem_ld8(tl + 3 * hs + c8 * 8, yi);
           tmem_ld_wait();
-          if (c8 == groups - 1) {
+          if (c8 == c8_1 - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&a1empty[team]);
+            if (lane == 0 && ok) mbar_arrive(&a1empty[b]);
           }
           // half the group values of the 8 channels (inverse rDFT + b1, scales
           // folded into the weights), then GELU, as fp16 pairs
@@ -448,7 +449,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&hready[team]);
+        if (lane == 0 && ok) mbar_arrive(&hready[b]);
       }
     }
   } else {
