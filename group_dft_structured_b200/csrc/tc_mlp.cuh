@@ -188,7 +188,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
                                               ~static_cast<uintptr_t>(1023));
   const MlpPlan &P = p.P;
   const MlpSmem L = mlp_smem(p);
-  float *sb1 = reinterpret_cast<float *>(smem + L.b1);
+  uint32_t *sb1 = reinterpret_cast<uint32_t *>(smem + L.b1);  // b1 / 2, fp16 channel pairs
   float *sb2 = reinterpret_cast<float *>(smem + L.b2);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *wfull = bars;
@@ -219,8 +219,12 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     mbar_init(final_bar, 1);
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < nS * hs; i += blockDim.x)  // b1 / 2, like fc1's accumulators
-    sb1[i] = (p.b1 != nullptr && i < P.H) ? 0.5f * __half2float(p.b1[i]) : 0.f;
+  for (int i = threadIdx.x; i < nS * hs / 2; i += blockDim.x) {  // b1 / 2, like fc1's accumulators
+    const int j = 2 * i;
+    const float v0 = (p.b1 != nullptr && j < P.H) ? 0.5f * __half2float(p.b1[j]) : 0.f;
+    const float v1 = (p.b1 != nullptr && j + 1 < P.H) ? 0.5f * __half2float(p.b1[j + 1]) : 0.f;
+    sb1[i] = pack_half2(v0, v1);
+  }
   for (int i = threadIdx.x; i < P.BD2; i += blockDim.x)
     sb2[i] = (p.b2 != nullptr && i < P.Co) ? __half2float(p.b2[i]) : 0.f;
   if (warp == 1) {
@@ -409,7 +413,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
         tc_fence_after();
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * 4 * hs;
         uint8_t *hb = smem + L.h0 + b * L.htile + row * 32;
-        const float *bias = sb1 + s * hs;
+        const uint32_t *bias = sb1 + s * hs / 2;
         for (int c8 = c8_0; c8 < c8_1; ++c8) {
           uint32_t y0[8], y2[8], yr[8], yi[8];
           __syncwarp();
@@ -423,24 +427,29 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&a1empty[b]);
           }
-          // half the group values of the 8 channels (inverse rDFT + b1, scales
-          // folded into the weights), then GELU, as fp16 pairs
-          uint32_t ga[8], gb[8];  // (g0, g1), (g2, g3) of channel i
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float A0 = __uint_as_float(y0[i]), A2 = __uint_as_float(y2[i]);
-            const float Ar = __uint_as_float(yr[i]), Ai = __uint_as_float(yi[i]);
-            const float pb = A0 + bias[c8 * 8 + i];
-            const float e = pb + A2, o = pb - A2;
-            ga[i] = gelu_half_arg_h2(pack_half2(e + Ar, o - Ai));
-            gb[i] = gelu_half_arg_h2(pack_half2(e - Ar, o + Ai));
-          }
-          // rDFT of the activations, channel pairs packed: fc2's four planes
+          // Per channel pair (c, c+1), packed as fp16 pairs: half the group
+          // values u_t = h_t / 2 (inverse rDFT + b1 / 2, the scales folded into
+          // the weights), GELU, and the rDFT of the activations, whose four bins
+          // are fc2's operand planes (channel pairs are the planes' word layout).
           uint32_t pl[4][4];
 #pragma unroll
-          for (int i2 = 0; i2 < 4; ++i2)
-            rdft4_pair(make_uint4(ga[2 * i2], gb[2 * i2], ga[2 * i2 + 1], gb[2 * i2 + 1]),
-                       pl[0][i2], pl[1][i2], pl[2][i2], pl[3][i2]);
+          for (int i2 = 0; i2 < 4; ++i2) {
+            const __half2 a0 = as_h2(pack_half2(__uint_as_float(y0[2 * i2]), __uint_as_float(y0[2 * i2 + 1])));
+            const __half2 a2 = as_h2(pack_half2(__uint_as_float(y2[2 * i2]), __uint_as_float(y2[2 * i2 + 1])));
+            const __half2 ar = as_h2(pack_half2(__uint_as_float(yr[2 * i2]), __uint_as_float(yr[2 * i2 + 1])));
+            const __half2 ai = as_h2(pack_half2(__uint_as_float(yi[2 * i2]), __uint_as_float(yi[2 * i2 + 1])));
+            const __half2 pb = __hadd2(a0, as_h2(bias[c8 * 4 + i2]));
+            const __half2 e = __hadd2(pb, a2), o = __hsub2(pb, a2);
+            const __half2 g0 = as_h2(gelu_half_arg_h2(as_u32(__hadd2(e, ar))));
+            const __half2 g1 = as_h2(gelu_half_arg_h2(as_u32(__hsub2(o, ai))));
+            const __half2 g2 = as_h2(gelu_half_arg_h2(as_u32(__hsub2(e, ar))));
+            const __half2 g3 = as_h2(gelu_half_arg_h2(as_u32(__hadd2(o, ai))));
+            const __half2 s02 = __hadd2(g0, g2), s13 = __hadd2(g1, g3);
+            pl[0][i2] = as_u32(__hadd2(s02, s13));   // V0
+            pl[1][i2] = as_u32(__hsub2(s02, s13));   // V2
+            pl[2][i2] = as_u32(__hsub2(g0, g2));     // Re V1
+            pl[3][i2] = as_u32(__hsub2(g1, g3));     // -Im V1
+          }
           uint8_t *dst = hb + (c8 >> 1) * kMlpChunkBytes + ((((c8 & 1) ^ (row >> 2)) & 1) << 4);
 #pragma unroll
           for (int pp = 0; pp < 4; ++pp)
