@@ -16,17 +16,18 @@
 // (Hendrycks and Gimpel), on packed fp16 pairs with the hardware tanh; it is
 // within 5e-4 of the exact z*Phi(z) for every z.
 //
-// One persistent CTA per SM, 128-token tiles, 18 warps:
+// One persistent CTA per SM, 128-token tiles, 22 warps:
 //   warp 0        TMA: the resident Fourier weights of both layers (once), then
 //                 each tile's x chunks [128 tokens x 16 channels x 4] into one
 //                 of `nx` tile buffers
 //   warp 1        TMEM allocator + single-thread MMA issuer
 //   warps 2..5    transform: rDFT of the x tile in place into four K-major
 //                 planes per chunk (V0, V2, Re V1, -Im V1)
-//   warps 6..13   GELU: per hidden slice of HS channels (two warps per TMEM
-//                 lane quadrant, half the channels each) inverse rDFT + b1 ->
-//                 GELU -> rDFT -> fp16 planes in one of two hidden buffers
-//   warps 14..17  fc2 epilogue: inverse rDFT + b2, TMA stores of y
+//   warps 6..17   GELU: per hidden slice of HS channels (three warps per TMEM
+//                 lane quadrant, every third 8-channel group each) inverse
+//                 rDFT + b1 -> GELU -> rDFT -> fp16 planes in one of two
+//                 hidden buffers
+//   warps 18..21  fc2 epilogue: inverse rDFT + b2, TMA stores of y
 // TMEM: fc1 accumulators 2 x 4*HS columns (Y0 | Y2 | Re Y1 | Im Y1 of a
 // slice), fc2 accumulators (one or two, by tile) of 4*BD2 columns from 8*HS.
 // Issue order over the CTA's hidden slices gs (tile-major, across tiles):
@@ -45,7 +46,13 @@
 
 namespace feql {
 
-constexpr int kMlpThreads = 18 * 32;
+constexpr int kMlpGeluParts = 3;                         // GELU warps per TMEM lane quadrant
+constexpr int kMlpGeluWarps = 4 * kMlpGeluParts;
+constexpr int kMlpEpiWarp0 = 6 + kMlpGeluWarps;           // first fc2 epilogue warp
+constexpr int kMlpThreads = (kMlpEpiWarp0 + 4) * 32;      // 22 warps
+// registers per thread: the busiest SM sub-partition holds ceil(warps / 4)
+// warps in its 16K-register slice
+constexpr int kMlpMaxRegs = (16384 / (((kMlpThreads / 32 + 3) / 4) * 32)) / 8 * 8;  // 80
 constexpr int kMlpYBoxes = 2;                    // output staging boxes per epilogue warp
 constexpr int kMlpChunkBytes = kBM * kCK * kT * 2;  // 16 KB: 128 tokens x 16 channels x 4
 constexpr int kMlpPlaneBytes = kBM * kCK * 2;       // 4 KB: one plane of a chunk
@@ -179,8 +186,8 @@ __device__ __forceinline__ uint32_t gelu_half_arg_h2(uint32_t uu) {
   return as_u32(__hfma2(u, t, u));
 }
 
-// 18 warps: 5 on one register slice of an SM sub-partition, 96 registers each.
-__global__ void __maxnreg__(96)
+// 22 warps: six on the busiest 16K-register sub-partition, 80 registers each.
+__global__ void __maxnreg__(kMlpMaxRegs)
 tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
               const TcMlpParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -208,8 +215,8 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       mbar_init(&xready[b], 4);
       mbar_init(&xempty[b], 1);
       mbar_init(&a1full[b], 1);
-      mbar_init(&a1empty[b], 8);
-      mbar_init(&hready[b], 8);
+      mbar_init(&a1empty[b], kMlpGeluWarps);
+      mbar_init(&hready[b], kMlpGeluWarps);
       mbar_init(&hempty[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -392,17 +399,19 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       if (lane == 0 && ok) mbar_arrive(&xready[xb]);
       if (++xb == p.nx) { xb = 0; xph ^= 1; }
     }
-  } else if (warp < 14) {
+  } else if (warp < kMlpEpiWarp0) {
     // --------------------------------------------------------------- GELU
-    // All eight warps take every hidden slice gs (fc1 accumulator and hidden
+    // All GELU warps take every hidden slice gs (fc1 accumulator and hidden
     // buffer gs % 2): warp quadrant q = warp % 4 reads TMEM lanes 32q..32q+31,
-    // i.e. token rows row = 32q + lane, and each of the two warps of a
-    // quadrant takes half of the slice's 8-channel groups.
-    const int half = (warp - 6) / 4;
+    // i.e. token rows row = 32q + lane, and the kMlpGeluParts warps of a
+    // quadrant take every kMlpGeluParts-th 8-channel group of the slice.
+    const int part = (warp - 6) / 4;
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const int groups = hs / 8;  // 8 hidden channels per step
-    const int c8_0 = half * (groups / 2), c8_1 = c8_0 + groups / 2;
+    // this warp's last group (-1: none; it still arrives on both barriers)
+    const int c8_last =
+        part < groups ? part + (groups - 1 - part) / kMlpGeluParts * kMlpGeluParts : -1;
     int g = 0;
     for (int m = blockIdx.x; m < p.nM; m += gridDim.x, g += nS) {
       for (int s = 0; s < nS; ++s) {
@@ -414,7 +423,12 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + b * 4 * hs;
         uint8_t *hb = smem + L.h0 + b * L.htile + row * 32;
         const uint32_t *bias = sb1 + s * hs / 2;
-        for (int c8 = c8_0; c8 < c8_1; ++c8) {
+        if (c8_last < 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && ok) mbar_arrive(&a1empty[b]);
+        }
+        for (int c8 = part; c8 < groups; c8 += kMlpGeluParts) {
           uint32_t y0[8], y2[8], yr[8], yi[8];
           __syncwarp();
           tmem_ld8(tl + c8 * 8, y0);
@@ -422,7 +436,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           tmem_ld8(tl + 2 * hs + c8 * 8, yr);
           tmem_ld8(tl + 3 * hs + c8 * 8, yi);
           tmem_ld_wait();
-          if (c8 == c8_1 - 1) {
+          if (c8 == c8_last) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&a1empty[b]);
@@ -464,7 +478,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
   } else {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;
-    const int ew = warp - 14;
+    const int ew = warp - kMlpEpiWarp0;
     uint8_t *obase = smem + L.y0 + ew * kMlpYBoxes * 4096;
     const int groups = P.BD2 / 16;
     int oi = 0, it = 0;
