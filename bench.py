@@ -15,7 +15,8 @@ no flush is needed between steps.
 for the cyclic group C_8 (feql_ct_* entry points, dX and dW as two passes), and
 workload 7 the Swin stage-1 MLP block (fc1 -> GELU -> fc2, one fused kernel,
 feql_mlp_forward; its "unfused" line times the same block as fc1 forward, a
-torch GELU and fc2 forward, for context).
+torch GELU and fc2 forward, for context); workload 8 is the Swin stream for
+p4m (rotations and reflections, feql_p4m_* entry points).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the full workload on
 its own tokens (weak scaling); the data-parallel weight gradient is summed
@@ -49,8 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
-                    help="workload id 1-7 (group_dft_structured_b200/workloads.py; 6 is the "
-                         "cyclic group C_8, 7 the MLP block)")
+                    help="workload id 1-8 (group_dft_structured_b200/workloads.py; 6 is the "
+                         "cyclic group C_8, 7 the MLP block, 8 p4m)")
     ap.add_argument("--dtype", choices=["fp16", "fp32"], default=None,
                     help="override the workload's dtype (e.g. the fp32 run of the square layer)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -113,9 +114,11 @@ def mlp_bytes(w, elt):
 
 def layer_macs(w):
     """Real MACs of one contraction pass with the Fourier method: (2T-2) NCD for
-    even T (bins 0 and T/2 real, the others complex), and of the unrolled
+    the cyclic group of even order T (bins 0 and T/2 real, the others complex),
+    12 NCD for p4m (four 1-dim irreps and one 2 x 2 block); and of the unrolled
     dense method: T^2 NCD."""
-    return (2 * w.T - 2) * w.N * w.C * w.D, w.T * w.T * w.N * w.C * w.D
+    fourier = 12 if w.group == "p4m" else 2 * w.T - 2
+    return fourier * w.N * w.C * w.D, w.T * w.T * w.N * w.C * w.D
 
 
 def kernel_source_hash():
@@ -204,7 +207,9 @@ def time_oracle(w, n_sample):
         t0 = time.perf_counter()
         M.forward(f["x"], f["W1"], f["b1"], f["W2"], f["b2"])
         return time.perf_counter() - t0
-    if w.T == 4:
+    if w.group == "p4m":
+        from oracle import feql_p4m_oracle as O
+    elif w.T == 4:
         from oracle import feql_oracle as O
     else:
         from oracle import feql_ct_oracle as O
@@ -276,25 +281,38 @@ def setup_layer(args, w, rank, s, F, torch):
     inp = make_inputs(rank_seed_id(w.wid, rank), N, C, D, w.dtype, T=T)
     dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
     x, W, b, dy = dev["x"], dev["W"], dev["b"], dev["dy"]
-    What = torch.empty(F.feql_ct_weight_fft_bytes(T, C, D, mode), dtype=torch.uint8,
-                       device="cuda")
+    p4m = w.group == "p4m"
+    wbytes = (F.feql_p4m_weight_fft_bytes(C, D, mode) if p4m
+              else F.feql_ct_weight_fft_bytes(T, C, D, mode))
+    What = torch.empty(wbytes, dtype=torch.uint8, device="cuda")
     y = torch.empty((N, D, T), dtype=x.dtype, device="cuda")
     dx = torch.empty((N, C, T), dtype=x.dtype, device="cuda")
     dW = torch.empty((D, C, T), dtype=x.dtype, device="cuda")
     db = torch.empty((D,), dtype=x.dtype, device="cuda")
-    ws = torch.empty(max(F.feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode), 16),
-                     dtype=torch.uint8, device="cuda")
+    wsb = (F.feql_p4m_backward_dw_workspace_bytes(N, C, D, mode) if p4m
+           else F.feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode))
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
     # One step = every row of the path: weight rDFT, forward, and the backward
     # (dX and dW/db, fused into one pass over dy for p4 unless --separate-backward).
-    calls = {
-        "wfft": lambda: F.feql_ct_weight_fft(T, W, What, C, D, mode, s),
-        "fwd": lambda: F.feql_ct_forward(T, x, What, b, y, N, C, D, mode, s),
-        "dx": lambda: F.feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, s),
-        "dw": lambda: F.feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
-        "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode, s),
-    }
+    if p4m:
+        calls = {
+            "wfft": lambda: F.feql_p4m_weight_fft(W, What, C, D, mode, s),
+            "fwd": lambda: F.feql_p4m_forward(x, What, b, y, N, C, D, mode, s),
+            "dx": lambda: F.feql_p4m_backward_dx(dy, What, dx, N, C, D, mode, s),
+            "dw": lambda: F.feql_p4m_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
+        }
+    else:
+        calls = {
+            "wfft": lambda: F.feql_ct_weight_fft(T, W, What, C, D, mode, s),
+            "fwd": lambda: F.feql_ct_forward(T, x, What, b, y, N, C, D, mode, s),
+            "dx": lambda: F.feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, s),
+            "dw": lambda: F.feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode,
+                                                s),
+            "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode,
+                                           s),
+        }
     passes = ["wfft"] + (["fwd"] if "fwd" in w.passes else [])
-    if "dx" in w.passes and "dw" in w.passes and not args.separate_backward and T == 4:
+    if "dx" in w.passes and "dw" in w.passes and not args.separate_backward and T == 4 and not p4m:
         passes.append("bwd")
     else:
         passes += [p for p in ("dx", "dw") if p in w.passes]
@@ -315,7 +333,7 @@ def setup_layer(args, w, rank, s, F, torch):
         "host": {k: inp[k] for k in ins}, "dev": {k: dev[k] for k in ins},
         "outs": {k: src[k] for k in outs},
         "allreduce": (lambda: dp_allreduce_grads(dW, db)) if has_bwd else None,
-        "config": {"N": N, "C": C, "D": D, "T": T},
+        "config": {"N": N, "C": C, "D": D, "T": T, "group": "p4m (D4)" if p4m else f"C_{T}"},
         "extra": {},
     }
 

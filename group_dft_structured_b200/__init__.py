@@ -62,6 +62,12 @@ _SIGNATURES = {
     "feql_ct_backward_dx": (_I, [_I, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
     "feql_ct_backward_dw_workspace_bytes": (_SZ, [_I, _I64, _I, _I, _I]),
     "feql_ct_backward_dw": (_I, [_I, _VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
+    "feql_p4m_weight_fft_bytes": (_SZ, [_I, _I, _I]),
+    "feql_p4m_weight_fft": (_I, [_VP, _VP, _I, _I, _I, _VP]),
+    "feql_p4m_forward": (_I, [_VP, _VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
+    "feql_p4m_backward_dx": (_I, [_VP, _VP, _VP, _I64, _I, _I, _I, _VP]),
+    "feql_p4m_backward_dw_workspace_bytes": (_SZ, [_I64, _I, _I, _I]),
+    "feql_p4m_backward_dw": (_I, [_VP, _VP, _VP, _VP, _VP, _SZ, _I64, _I, _I, _I, _VP]),
     "feql_mlp_weight_fft_bytes": (_SZ, [_I, _I, _I, _I]),
     "feql_mlp_weight_fft": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _VP]),
     "feql_mlp_forward": (_I, [_VP, _VP, _VP, _VP, _VP, _I64, _I, _I, _I, _I, _VP]),
@@ -187,6 +193,35 @@ def feql_ct_backward_dw(T: int, x, dy, dW, db, ws, ws_bytes: int, N: int, C: int
     _check(load().feql_ct_backward_dw(T, _ptr(x), _ptr(dy), _ptr(dW), _ptr(db), _ptr(ws),
                                       ws_bytes, N, C, D, dtype, _stream(stream)),
            "feql_ct_backward_dw")
+
+
+def feql_p4m_weight_fft_bytes(C: int, D: int, dtype: int) -> int:
+    return int(load().feql_p4m_weight_fft_bytes(C, D, dtype))
+
+
+def feql_p4m_weight_fft(W, What, C: int, D: int, dtype: int, stream=None) -> None:
+    _check(load().feql_p4m_weight_fft(_ptr(W), _ptr(What), C, D, dtype, _stream(stream)),
+           "feql_p4m_weight_fft")
+
+
+def feql_p4m_forward(x, What, b, y, N: int, C: int, D: int, dtype: int, stream=None) -> None:
+    _check(load().feql_p4m_forward(_ptr(x), _ptr(What), _ptr(b), _ptr(y), N, C, D, dtype,
+                                   _stream(stream)), "feql_p4m_forward")
+
+
+def feql_p4m_backward_dx(dy, What, dx, N: int, C: int, D: int, dtype: int, stream=None) -> None:
+    _check(load().feql_p4m_backward_dx(_ptr(dy), _ptr(What), _ptr(dx), N, C, D, dtype,
+                                       _stream(stream)), "feql_p4m_backward_dx")
+
+
+def feql_p4m_backward_dw_workspace_bytes(N: int, C: int, D: int, dtype: int) -> int:
+    return int(load().feql_p4m_backward_dw_workspace_bytes(N, C, D, dtype))
+
+
+def feql_p4m_backward_dw(x, dy, dW, db, ws, ws_bytes: int, N: int, C: int, D: int, dtype: int,
+                         stream=None) -> None:
+    _check(load().feql_p4m_backward_dw(_ptr(x), _ptr(dy), _ptr(dW), _ptr(db), _ptr(ws), ws_bytes,
+                                       N, C, D, dtype, _stream(stream)), "feql_p4m_backward_dw")
 
 
 def feql_mlp_weight_fft_bytes(C: int, H: int, Co: int, dtype: int) -> int:

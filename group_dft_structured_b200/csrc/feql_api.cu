@@ -17,7 +17,7 @@
 #include "tc_bwd.cuh"
 #include "tc_dw.cuh"
 #include "tc_fwd.cuh"
-#include "ct8.cuh"
+#include "group8.cuh"
 #include "tc_mlp.cuh"
 #include "wfft.cuh"
 
@@ -347,15 +347,16 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
 }
 
 // ---------------------------------------------------------------------------
-// Cyclic group C_8 (fp16, tensor cores)
+// Groups of order 8: C_8 and the point group D4 of p4m (fp16, tensor cores)
 // ---------------------------------------------------------------------------
-int launch_ct8_fwd(const void *in, const uint8_t *wt, const Ct8Plan &P, const __half *bias,
+template <class Gp>
+int launch_g8_fwd(const void *in, const uint8_t *wt, const G8Plan &P, const __half *bias,
                    void *out, int64_t N, cudaStream_t stream) {
   DeviceInfo dev;
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
   if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
-  Ct8FwdParams p;
+  G8FwdParams p;
   p.wt = wt;
   p.bias = bias;
   p.out = static_cast<__half *>(out);
@@ -370,28 +371,28 @@ int launch_ct8_fwd(const void *in, const uint8_t *wt, const Ct8Plan &P, const __
   p.n_units = p.nM * p.nD;
   p.nacc = 16 * p.BD <= 512 ? 2 : 1;
   p.acc_stride = 8 * p.BD;
-  p.stage_bytes = kCt8XChunk + static_cast<int>(align_up(p.chunk_bytes, 1024));
+  p.stage_bytes = kG8XChunk + static_cast<int>(align_up(p.chunk_bytes, 1024));
   p.bias_floats = p.nD * p.BD;
   const int budget = dev.smem_optin - 1024;
   p.stages = 6;
-  while (p.stages > 2 && ct8_fwd_smem(p).total > budget) --p.stages;
-  if (ct8_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  while (p.stages > 2 && g8_fwd_smem(p).total > budget) --p.stages;
+  if (g8_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
   CUtensorMap tm, tm_out;
   st = make_tmap_f16(&tm, in, N, static_cast<int64_t>(P.Ci) * kT8, kBM);
   if (st != FEQL_OK) return st;
   st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT8, 32);
   if (st != FEQL_OK) return st;
-  const int smem = ct8_fwd_smem(p).total + 1024;
-  if (cudaFuncSetAttribute(tc_ct8_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  const int smem = g8_fwd_smem(p).total + 1024;
+  if (cudaFuncSetAttribute(tc_g8_fwd_kernel<Gp>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FEQL_ERR_CUDA;
   const int grid = p.n_units < dev.sms ? p.n_units : dev.sms;
-  tc_ct8_fwd_kernel<<<grid, kCt8Threads, smem, stream>>>(tm, tm_out, p);
+  tc_g8_fwd_kernel<Gp><<<grid, kG8Threads, smem, stream>>>(tm, tm_out, p);
   return launch_status();
 }
 
-Ct8DwParams make_ct8_dw_plan(int64_t N, int C, int D, int sms) {
-  Ct8DwParams p;
+G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms) {
+  G8DwParams p;
   p.N = N;
   p.C = C;
   p.D = D;
@@ -401,52 +402,53 @@ Ct8DwParams make_ct8_dw_plan(int64_t N, int C, int D, int sms) {
   p.tiles_c = static_cast<int>(cdiv(C, p.CT));
   const int tiles = p.tiles_d * p.tiles_c;
   int64_t s = sms / tiles > 1 ? sms / tiles : 1;
-  const int64_t chunks = cdiv(N, kCt8DwTB);
+  const int64_t chunks = cdiv(N, kG8DwTB);
   if (s > chunks) s = chunks;
-  p.split_len = N > 0 ? align_up(cdiv(N, s), kCt8DwTB) : kCt8DwTB;
+  p.split_len = N > 0 ? align_up(cdiv(N, s), kG8DwTB) : kG8DwTB;
   p.splits = N > 0 ? static_cast<int>(cdiv(N, p.split_len)) : 0;
-  p.slot_boxes = kCt8DwDySlots + 2 * (p.CT / 16);
+  p.slot_boxes = kG8DwDySlots + 2 * (p.CT / 16);
   p.stages = 1;
   p.ws = nullptr;
   p.ws_db = nullptr;
   return p;
 }
 
-int64_t ct8_dw_ws_floats(const Ct8DwParams &p) {
+int64_t g8_dw_ws_floats(const G8DwParams &p) {
   return static_cast<int64_t>(p.splits) * (8ll * p.D * p.Cs + p.D);
 }
 
-int launch_ct8_dw(const void *x, const void *dy, __half *dW, __half *db, float *ws,
+template <class Gp>
+int launch_g8_dw(const void *x, const void *dy, __half *dW, __half *db, float *ws,
                   size_t ws_bytes, int64_t N, int C, int D, cudaStream_t stream) {
   DeviceInfo dev;
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
   if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
-  Ct8DwParams p = make_ct8_dw_plan(N, C, D, dev.sms);
-  if (ws_bytes < static_cast<size_t>(ct8_dw_ws_floats(p)) * 4) return FEQL_ERR_INVALID_ARG;
+  G8DwParams p = make_g8_dw_plan(N, C, D, dev.sms);
+  if (ws_bytes < static_cast<size_t>(g8_dw_ws_floats(p)) * 4) return FEQL_ERR_INVALID_ARG;
   p.ws = ws;
   p.ws_db = ws + static_cast<int64_t>(p.splits) * 8 * p.D * p.Cs;
   const int budget = dev.smem_optin - 1024;
   p.stages = 4;
-  while (p.stages > 1 && ct8_dw_smem(p).total > budget) --p.stages;
-  if (ct8_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  while (p.stages > 1 && g8_dw_smem(p).total > budget) --p.stages;
+  if (g8_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
   if (p.splits > 0) {
     CUtensorMap tm_dy, tm_x;
-    st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kCt8DwTB);
+    st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB);
     if (st != FEQL_OK) return st;
-    st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kCt8DwTB);
+    st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB);
     if (st != FEQL_OK) return st;
-    const int smem = ct8_dw_smem(p).total + 1024;
-    if (cudaFuncSetAttribute(tc_ct8_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+    const int smem = g8_dw_smem(p).total + 1024;
+    if (cudaFuncSetAttribute(tc_g8_dw_kernel<Gp>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return FEQL_ERR_CUDA;
     const int64_t grid = static_cast<int64_t>(p.splits) * p.tiles_d * p.tiles_c;
     if (grid > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-    tc_ct8_dw_kernel<<<static_cast<unsigned>(grid), kCt8DwThreads, smem, stream>>>(tm_dy, tm_x, p);
+    tc_g8_dw_kernel<Gp><<<static_cast<unsigned>(grid), kG8DwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  const int64_t rblocks = ct8_reduce_blocks(C, D);
+  const int64_t rblocks = g8_reduce_blocks(C, D);
   if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-  ct8_dw_reduce_kernel<<<static_cast<unsigned>(rblocks), kRed8Out * kRed8Groups, 0, stream>>>(
+  g8_dw_reduce_kernel<Gp><<<static_cast<unsigned>(rblocks), kRed8Out * kRed8Groups, 0, stream>>>(
       p.ws, p.ws_db, dW, db, p.splits, C, D, p.Cs);
   return launch_status();
 }
@@ -519,6 +521,71 @@ int ct_check(int T, int dtype) {
   if (!valid_dtype(dtype)) return FEQL_ERR_INVALID_ARG;
   if (resolve(dtype) != FEQL_FP16) return FEQL_ERR_UNSUPPORTED;
   return FEQL_OK;
+}
+
+
+// FEQL_FP16 is the one mode of the p4m kernels.
+int p4m_check(int dtype) {
+  if (!valid_dtype(dtype)) return FEQL_ERR_INVALID_ARG;
+  if (resolve(dtype) != FEQL_FP16) return FEQL_ERR_UNSUPPORTED;
+  return FEQL_OK;
+}
+
+// The order-8 entry points after their group/mode check: argument checks,
+// then the templated launches.
+template <class Gp>
+size_t g8_weight_fft_bytes(int C, int D) {
+  if (check_shape(C, D) != FEQL_OK) return 0;
+  return static_cast<size_t>(make_g8_layout(C, D, Gp::kWRows).bytes);
+}
+
+template <class Gp>
+int g8_weight_fft(const void *W, void *What, int C, int D, feql_stream stream) {
+  if (W == nullptr || What == nullptr || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  const int st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  const G8Layout L = make_g8_layout(C, D, Gp::kWRows);
+  wfft_g8_kernel<Gp><<<grid_for((L.fwd.bytes + L.dx.bytes) / 2, 256, dev.sms), 256, 0,
+                       reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half *>(W), static_cast<uint8_t *>(What), L, C);
+  return launch_status();
+}
+
+template <class Gp>
+int g8_pass(const void *in, const void *What, const void *bias, void *out, int64_t N, int C, int D,
+            feql_stream stream, int dir) {
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
+  if (N == 0) return FEQL_OK;
+  const G8Layout L = make_g8_layout(C, D, Gp::kWRows);
+  const uint8_t *wt = static_cast<const uint8_t *>(What) + (dir == 0 ? L.off_fwd : L.off_dx);
+  return launch_g8_fwd<Gp>(in, wt, dir == 0 ? L.fwd : L.dx, static_cast<const __half *>(bias),
+                           out, N, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t g8_dw_workspace_bytes(int64_t N, int C, int D) {
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
+  DeviceInfo dev;
+  if (device_info(&dev) != FEQL_OK) return 0;
+  return static_cast<size_t>(g8_dw_ws_floats(make_g8_dw_plan(N, C, D, dev.sms))) * 4;
+}
+
+template <class Gp>
+int g8_dw(const void *x, const void *dy, void *dW, void *db, void *ws, size_t ws_bytes, int64_t N,
+          int C, int D, feql_stream stream) {
+  if (dW == nullptr || ws == nullptr || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
+    return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws) ||
+      (db != nullptr && !aligned16(db)))
+    return FEQL_ERR_INVALID_ARG;
+  return launch_g8_dw<Gp>(x, dy, static_cast<__half *>(dW), static_cast<__half *>(db),
+                          static_cast<float *>(ws), ws_bytes, N, C, D,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -685,77 +752,86 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws
 // ---------------------------------------------------------------------------
 size_t feql_ct_weight_fft_bytes(int T, int C, int D, int dtype) {
   if (T == 4) return feql_weight_fft_bytes(C, D, dtype);
-  if (ct_check(T, dtype) != FEQL_OK || check_shape(C, D) != FEQL_OK) return 0;
-  return static_cast<size_t>(make_ct8_layout(C, D).bytes);
+  if (ct_check(T, dtype) != FEQL_OK) return 0;
+  return g8_weight_fft_bytes<Cyclic8>(C, D);
 }
 
 int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype,
                        feql_stream stream) {
   if (T == 4) return feql_weight_fft(W, What, C, D, dtype, stream);
-  int st = ct_check(T, dtype);
+  const int st = ct_check(T, dtype);
   if (st != FEQL_OK) return st;
-  if (W == nullptr || What == nullptr || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
-  if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
-  DeviceInfo dev;
-  st = device_info(&dev);
-  if (st != FEQL_OK) return st;
-  const Ct8Layout L = make_ct8_layout(C, D);
-  wfft_ct8_kernel<<<grid_for((L.fwd.bytes + L.dx.bytes) / 2, 256, dev.sms), 256, 0,
-                    reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<const __half *>(W),
-                                                            static_cast<uint8_t *>(What), L, C);
-  return launch_status();
-}
-
-static int ct_pass(int T, const void *in, const void *What, const void *bias, void *out, int64_t N,
-                   int C, int D, int dtype, feql_stream stream, int dir) {
-  int st = ct_check(T, dtype);
-  if (st != FEQL_OK) return st;
-  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
-  if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
-  if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
-  if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
-  if (N == 0) return FEQL_OK;
-  const Ct8Layout L = make_ct8_layout(C, D);
-  const uint8_t *wt = static_cast<const uint8_t *>(What) + (dir == 0 ? L.off_fwd : L.off_dx);
-  return launch_ct8_fwd(in, wt, dir == 0 ? L.fwd : L.dx, static_cast<const __half *>(bias), out, N,
-                        reinterpret_cast<cudaStream_t>(stream));
+  return g8_weight_fft<Cyclic8>(W, What, C, D, stream);
 }
 
 int feql_ct_forward(int T, const void *x, const void *What, const void *b, void *y, int64_t N,
                     int C, int D, int dtype, feql_stream stream) {
   if (T == 4) return feql_forward(x, What, b, y, N, C, D, dtype, stream);
-  return ct_pass(T, x, What, b, y, N, C, D, dtype, stream, 0);
+  const int st = ct_check(T, dtype);
+  if (st != FEQL_OK) return st;
+  return g8_pass<Cyclic8>(x, What, b, y, N, C, D, stream, 0);
 }
 
 int feql_ct_backward_dx(int T, const void *dy, const void *What, void *dx, int64_t N, int C, int D,
                         int dtype, feql_stream stream) {
   if (T == 4) return feql_backward_dx(dy, What, dx, N, C, D, dtype, stream);
-  return ct_pass(T, dy, What, nullptr, dx, N, C, D, dtype, stream, 1);
+  const int st = ct_check(T, dtype);
+  if (st != FEQL_OK) return st;
+  return g8_pass<Cyclic8>(dy, What, nullptr, dx, N, C, D, stream, 1);
 }
 
 size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int dtype) {
   if (T == 4) return feql_backward_dw_workspace_bytes(N, C, D, dtype);
-  if (ct_check(T, dtype) != FEQL_OK || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
-    return 0;
-  DeviceInfo dev;
-  if (device_info(&dev) != FEQL_OK) return 0;
-  return static_cast<size_t>(ct8_dw_ws_floats(make_ct8_dw_plan(N, C, D, dev.sms))) * 4;
+  if (ct_check(T, dtype) != FEQL_OK) return 0;
+  return g8_dw_workspace_bytes(N, C, D);
 }
 
 int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db, void *ws,
                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream) {
   if (T == 4) return feql_backward_dw(x, dy, dW, db, ws, ws_bytes, N, C, D, dtype, stream);
-  int st = ct_check(T, dtype);
+  const int st = ct_check(T, dtype);
   if (st != FEQL_OK) return st;
-  if (dW == nullptr || ws == nullptr || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
-    return FEQL_ERR_INVALID_ARG;
-  if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws) ||
-      (db != nullptr && !aligned16(db)))
-    return FEQL_ERR_INVALID_ARG;
-  return launch_ct8_dw(x, dy, static_cast<__half *>(dW), static_cast<__half *>(db),
-                       static_cast<float *>(ws), ws_bytes, N, C, D,
-                       reinterpret_cast<cudaStream_t>(stream));
+  return g8_dw<Cyclic8>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
+}
+
+// ---------------------------------------------------------------------------
+// p4m (point group D4)
+// ---------------------------------------------------------------------------
+size_t feql_p4m_weight_fft_bytes(int C, int D, int dtype) {
+  if (p4m_check(dtype) != FEQL_OK) return 0;
+  return g8_weight_fft_bytes<Dihedral4>(C, D);
+}
+
+int feql_p4m_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_stream stream) {
+  const int st = p4m_check(dtype);
+  if (st != FEQL_OK) return st;
+  return g8_weight_fft<Dihedral4>(W, What, C, D, stream);
+}
+
+int feql_p4m_forward(const void *x, const void *What, const void *b, void *y, int64_t N, int C,
+                     int D, int dtype, feql_stream stream) {
+  const int st = p4m_check(dtype);
+  if (st != FEQL_OK) return st;
+  return g8_pass<Dihedral4>(x, What, b, y, N, C, D, stream, 0);
+}
+
+int feql_p4m_backward_dx(const void *dy, const void *What, void *dx, int64_t N, int C, int D,
+                         int dtype, feql_stream stream) {
+  const int st = p4m_check(dtype);
+  if (st != FEQL_OK) return st;
+  return g8_pass<Dihedral4>(dy, What, nullptr, dx, N, C, D, stream, 1);
+}
+
+size_t feql_p4m_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
+  if (p4m_check(dtype) != FEQL_OK) return 0;
+  return g8_dw_workspace_bytes(N, C, D);
+}
+
+int feql_p4m_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws,
+                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream) {
+  const int st = p4m_check(dtype);
+  if (st != FEQL_OK) return st;
+  return g8_dw<Dihedral4>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
 }
 
 size_t feql_mlp_weight_fft_bytes(int C, int H, int Co, int dtype) {

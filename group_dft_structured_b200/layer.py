@@ -11,7 +11,9 @@ from . import (FEQL_FP16, FEQL_FP16_SIMT, feql_backward, feql_backward_dw,
                feql_backward_dw_workspace_bytes, feql_backward_dx, feql_ct_backward_dw,
                feql_ct_backward_dw_workspace_bytes, feql_ct_backward_dx, feql_ct_forward,
                feql_ct_weight_fft, feql_ct_weight_fft_bytes, feql_forward, feql_mlp_forward,
-               feql_mlp_weight_fft, feql_mlp_weight_fft_bytes, feql_weight_fft,
+               feql_mlp_weight_fft, feql_mlp_weight_fft_bytes, feql_p4m_backward_dw,
+               feql_p4m_backward_dw_workspace_bytes, feql_p4m_backward_dx, feql_p4m_forward,
+               feql_p4m_weight_fft, feql_p4m_weight_fft_bytes, feql_weight_fft,
                feql_weight_fft_bytes)
 
 
@@ -115,6 +117,44 @@ def ct_backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, with_db: bool =
     dW = torch.empty((D, C, T), dtype=x.dtype, device=x.device)
     db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
     feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
+    return dW, db
+
+
+# --------------------------------------------------------- p4m (D4, order 8)
+
+def p4m_weight_fft(W: torch.Tensor, mode: int, stream=None) -> torch.Tensor:
+    D, C, _ = W.shape
+    nbytes = feql_p4m_weight_fft_bytes(C, D, mode)
+    if nbytes == 0:
+        raise ValueError("unsupported (C, D, mode) for p4m")
+    What = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    feql_p4m_weight_fft(W, What, C, D, mode, stream)
+    return What
+
+
+def p4m_forward(x: torch.Tensor, What: torch.Tensor, b, D: int, mode: int, stream=None):
+    N, C, _ = x.shape
+    y = torch.empty((N, D, 8), dtype=x.dtype, device=x.device)
+    feql_p4m_forward(x, What, b, y, N, C, D, mode, stream)
+    return y
+
+
+def p4m_backward_dx(dy: torch.Tensor, What: torch.Tensor, C: int, mode: int, stream=None):
+    N, D, _ = dy.shape
+    dx = torch.empty((N, C, 8), dtype=dy.dtype, device=dy.device)
+    feql_p4m_backward_dx(dy, What, dx, N, C, D, mode, stream)
+    return dx
+
+
+def p4m_backward_dw(x: torch.Tensor, dy: torch.Tensor, mode: int, with_db: bool = True,
+                    stream=None):
+    N, C, _ = x.shape
+    D = dy.shape[1]
+    nbytes = feql_p4m_backward_dw_workspace_bytes(N, C, D, mode)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    dW = torch.empty((D, C, 8), dtype=x.dtype, device=x.device)
+    db = torch.empty((D,), dtype=x.dtype, device=x.device) if with_db else None
+    feql_p4m_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, stream)
     return dW, db
 
 

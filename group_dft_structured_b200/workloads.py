@@ -26,7 +26,8 @@ Rete"): a ViT MLP fc1 at 64 x 197 tokens and a Swin stage-1 stream at
 128 x 3136 tokens; no dataset is involved.  The C_8 workload keeps the Swin
 stream's token count and unrolled widths (96 -> 384) with T = 8.  The MLP
 workload is the Swin-T stage-1 block (96 -> 384 -> 96 unrolled) on the same
-token stream.
+token stream, and the p4m workload the same stream for the point group D4
+(8 group elements: rotations and reflections, element (r, m) at index 4 m + r).
 """
 
 from __future__ import annotations
@@ -47,6 +48,7 @@ class Workload:
     passes: tuple       # subset of ("fwd", "dx", "dw")
     note: str
     T: int = 4          # group order
+    group: str = "cyclic"  # "cyclic" (C_T) or "p4m" (point group D4, T = 8)
 
 
 WORKLOADS = {
@@ -64,6 +66,10 @@ WORKLOADS = {
     6: Workload(6, "c8_fwdbwd_fp16_swin_N401408_C12_D48", 401408, 12, 48, "fp16",
                 ("fwd", "dx", "dw"),
                 "cyclic group C_8, Swin stage-1-like stream (96->384 unrolled)", T=8),
+    8: Workload(8, "p4m_fwdbwd_fp16_swin_N401408_C12_D48", 401408, 12, 48, "fp16",
+                ("fwd", "dx", "dw"),
+                "p4m (rotations and reflections, D4), Swin stage-1-like stream (96->384 unrolled)",
+                T=8, group="p4m"),
     7: Workload(7, "p4_mlp_fp16_swin_N401408_C24_H96", 401408, 24, 96, "fp16", ("mlp",),
                 "Swin stage-1-like MLP block fc1 -> GELU -> fc2 (96->384->96 unrolled); "
                 "D is the hidden width, the output has C channels"),

@@ -173,6 +173,33 @@ int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db
                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * The wallpaper group p4m: rotations by 90 degrees and reflections, point group
+ * D4 of order 8 (Flash EQ-Linear, technical summary "Limitazioni e Lavoro
+ * Futuro": reflection groups are the named next step).  Group element
+ * g = (r, m), rotation by r * 90 degrees after the reflection m, stored at index
+ * 4 m + r of the group axis: x[N][C][8], y[N][D][8], W[D][C][8], dW[D][C][8].
+ * The layer is the group convolution
+ *   y[n,d,g] = b[d] + sum_c sum_h W[d,c,h^-1 g] x[n,c,h],
+ *   (r1, m1)(r2, m2) = (r1 + (-1)^m1 r2 mod 4, m1 xor m2),
+ * which on the rotations alone is the p4 layer.  D4 is not abelian: its Fourier
+ * transform has four 1-dim irreps and one 2-dim irrep E, so per token the layer
+ * is four scalar channel contractions and one 2 x 2 block contraction, 12 real
+ * products of N x C x D instead of the 64 of the unrolled matrix (forward:
+ * y^ = x^ W^; dX: dx^ = dy^ W^^T; dW: dW^ = x^^T dy^ summed over tokens).
+ * FEQL_FP16 only (other modes FEQL_ERR_UNSUPPORTED); any C, D >= 1.  Argument
+ * checks, N == 0, ownership, streams and errors are as for the p4 functions;
+ * the Fourier buffer has its own layout (feql_p4m_weight_fft_bytes). */
+size_t feql_p4m_weight_fft_bytes(int C, int D, int dtype);
+int feql_p4m_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_stream stream);
+int feql_p4m_forward(const void *x, const void *What, const void *b, void *y, int64_t N, int C,
+                     int D, int dtype, feql_stream stream);
+int feql_p4m_backward_dx(const void *dy, const void *What, void *dx, int64_t N, int C, int D,
+                         int dtype, feql_stream stream);
+size_t feql_p4m_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype);
+int feql_p4m_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws,
+                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream);
+
+/* ---------------------------------------------------------------------------
  * p4-equivariant MLP block, forward (Flash EQ-Linear, technical summary
  * "Livello di Rete": the EQ-ViT / EQ-Swin networks built from the layer; their
  * MLP is two EQ-Linear layers around a pointwise GELU):
