@@ -1,5 +1,6 @@
 """Drop-in PyTorch module for the equivariant linear layer of the cyclic group
-C_T (T = 4: the rotation group p4; T = 8), with autograd.
+C_T (T = 4: the rotation group p4; T = 8) and of p4m (rotations and
+reflections, point group D4), with autograd.
 
 Flash EQ-Linear (arXiv abstract) presents the method as a plug-and-play
 replacement for the EQ-Linear layers of existing equivariant models: the layer
@@ -9,8 +10,10 @@ computes the same function as the naive form, an ``nn.Linear`` whose (T*D) x
     A[d*T + t, c*T + s] = W[d, c, (t - s) mod T],   bias[d*T + t] = b[d],
 
 acting on features laid out as (channel, group element) with the group index
-innermost.  ``EqLinear.from_unrolled`` takes such a dense layer apart into
-(W, b); ``EqLinear.forward`` runs the library's kernels.
+innermost.  For p4m (group="p4m", 8 elements (r, m) at index 4 m + r) the
+unrolling is A[d*8 + g, c*8 + h] = W[d, c, h^-1 g].  ``EqLinear.from_unrolled``
+takes such a dense layer apart into (W, b); ``EqLinear.forward`` runs the
+library's kernels.
 
 Argument marshalling only: every step of the forward and backward passes runs
 in libfeql.so through the C ABI (``layer`` allocates outputs with torch).
@@ -35,8 +38,20 @@ def mode_for(dtype: torch.dtype) -> int:
     raise TypeError(f"EqLinear computes in float16 or float32, not {dtype}")
 
 
+def _p4m_index(r: int, m: int) -> int:
+    return 4 * m + (r % 4)
+
+
+def p4m_kernel_index(g: int, h: int) -> int:
+    """Index of h^-1 g in p4m's point group D4, elements (r, m) at 4 m + r."""
+    rg, mg = g % 4, g // 4
+    rh, mh = h % 4, h // 4
+    return _p4m_index((-1) ** mh * (rg - rh), mh ^ mg)
+
+
 class EqLinearFunction(torch.autograd.Function):
-    """y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod T] x[n,c,s] on (N, C, T) tensors.
+    """y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod T] x[n,c,s] on (N, C, T) tensors
+    (group "cyclic"), or the p4m group convolution W[d,c,h^-1 g] (group "p4m").
 
     ``What`` is the layer's Fourier weight buffer (``layer.ct_weight_fft`` of W),
     passed in so that callers can reuse it while W is unchanged.  Backward
@@ -45,11 +60,13 @@ class EqLinearFunction(torch.autograd.Function):
     """
 
     @staticmethod
-    def forward(ctx, x, W, b, What, mode: int):
+    def forward(ctx, x, W, b, What, mode: int, group: str = "cyclic"):
         D = W.shape[0]
-        y = _L.ct_forward(x, What, b, D, mode)
+        y = (_L.p4m_forward(x, What, b, D, mode) if group == "p4m"
+             else _L.ct_forward(x, What, b, D, mode))
         ctx.save_for_backward(x, What)
         ctx.mode = mode
+        ctx.group = group
         ctx.shape = (x.shape[1], D, x.shape[2])
         return y
 
@@ -60,29 +77,43 @@ class EqLinearFunction(torch.autograd.Function):
         need_x, need_W, need_b = ctx.needs_input_grad[:3]
         dy = dy.contiguous()
         dx = dW = db = None
-        if T == 4 and need_x and need_W:
+        if ctx.group == "p4m":
+            if need_x:
+                dx = _L.p4m_backward_dx(dy, What, C, ctx.mode)
+            if need_W or need_b:
+                dW, db = _L.p4m_backward_dw(x, dy, ctx.mode, with_db=need_b)
+        elif T == 4 and need_x and need_W:
             dx, dW, db = _L.backward(x, dy, What, ctx.mode, with_db=need_b)
         else:
             if need_x:
                 dx = _L.ct_backward_dx(dy, What, C, ctx.mode)
             if need_W or need_b:
                 dW, db = _L.ct_backward_dw(x, dy, ctx.mode, with_db=need_b)
-        return dx, (dW if need_W else None), (db if need_b else None), None, None
+        return dx, (dW if need_W else None), (db if need_b else None), None, None, None
 
 
 class EqLinear(torch.nn.Module):
-    """Equivariant linear layer of C_T on features (..., C*T), group index innermost.
+    """Equivariant linear layer of C_T (or p4m) on features (..., C*T), group index innermost.
 
     Parameters: ``weight`` [D][C][T] and ``bias`` [D] (or None), in float16
-    (T = 4 or 8) or float32 (T = 4).  The Fourier weight buffer is rebuilt when
-    the weight changes (tracked by its storage and version counter), so it is
-    computed once per optimizer step, or once for inference.
+    (T = 4 or 8, p4m) or float32 (T = 4).  ``group="p4m"`` selects the point
+    group D4 (T = 8: rotations (r, 0) at 0..3, reflected (r, 1) at 4..7).  The
+    Fourier weight buffer is rebuilt when the weight changes (tracked by its
+    storage and version counter), so it is computed once per optimizer step, or
+    once for inference.
     """
 
     def __init__(self, in_channels: int, out_channels: int, group_order: int = 4,
-                 bias: bool = True, dtype: torch.dtype = torch.float16, device=None):
+                 bias: bool = True, dtype: torch.dtype = torch.float16, device=None,
+                 group: str = "cyclic"):
         super().__init__()
-        self.in_channels, self.out_channels, self.group_order = in_channels, out_channels, group_order
+        if group not in ("cyclic", "p4m"):
+            raise ValueError(f"group is 'cyclic' or 'p4m', not {group!r}")
+        if group == "p4m" and group_order != 8:
+            raise ValueError("p4m has 8 group elements")
+        self.group = group
+        self.in_channels, self.out_channels = in_channels, out_channels
+        self.group_order = group_order
         mode_for(dtype)
         self.weight = torch.nn.Parameter(
             torch.empty((out_channels, in_channels, group_order), dtype=dtype, device=device))
@@ -105,7 +136,9 @@ class EqLinear(torch.nn.Module):
         key = (W.device, W.dtype, W.data_ptr(), W._version, tuple(W.shape))
         if self._what is None or self._what_key != key:
             with torch.no_grad():
-                self._what = _L.ct_weight_fft(W.detach().contiguous(), mode_for(W.dtype))
+                Wc = W.detach().contiguous()
+                self._what = (_L.p4m_weight_fft(Wc, mode_for(W.dtype)) if self.group == "p4m"
+                              else _L.ct_weight_fft(Wc, mode_for(W.dtype)))
             self._what_key = key
         return self._what
 
@@ -120,16 +153,17 @@ class EqLinear(torch.nn.Module):
         if x3.dtype != self.weight.dtype:
             raise TypeError(f"input dtype {x3.dtype} differs from the weight's {self.weight.dtype}")
         y = EqLinearFunction.apply(x3, self.weight, self.bias, self.fourier_weight(),
-                                   mode_for(self.weight.dtype))
+                                   mode_for(self.weight.dtype), self.group)
         return y.reshape(*lead, D * T)
 
     def extra_repr(self) -> str:
         return (f"in_channels={self.in_channels}, out_channels={self.out_channels}, "
-                f"group_order={self.group_order}, bias={self.bias is not None}")
+                f"group_order={self.group_order}, group={self.group}, "
+                f"bias={self.bias is not None}")
 
     @classmethod
     def from_unrolled(cls, weight: torch.Tensor, bias: torch.Tensor | None, group_order: int,
-                      atol: float = 0.0) -> "EqLinear":
+                      atol: float = 0.0, group: str = "cyclic") -> "EqLinear":
         """The layer equal to the dense (T*D) x (T*C) map ``weight`` (+ ``bias``).
 
         ``weight`` must be group-circulant in the layout above (entries that
@@ -143,9 +177,15 @@ class EqLinear(torch.nn.Module):
             raise ValueError(f"dense shape {tuple(weight.shape)} is not a multiple of T = {T}")
         D, C = rows // T, cols // T
         A = weight.detach().reshape(D, T, C, T)  # [d][t][c][s]
-        W = A[:, :, :, 0].permute(0, 2, 1).contiguous()  # W[d,c,u] = A[d, u, c, s=0]
-        t = torch.arange(T, device=weight.device)
-        u = (t[:, None] - t[None, :]) % T  # u[t][s] = (t - s) mod T
+        W = A[:, :, :, 0].permute(0, 2, 1).contiguous()  # W[d,c,u] = A[d, u, c, s=e]
+        if group == "p4m":
+            if T != 8:
+                raise ValueError("p4m has 8 group elements")
+            u = torch.tensor([[p4m_kernel_index(g, h) for h in range(8)] for g in range(8)],
+                             device=weight.device)  # u[g][h] = h^-1 g
+        else:
+            t = torch.arange(T, device=weight.device)
+            u = (t[:, None] - t[None, :]) % T  # u[t][s] = (t - s) mod T
         rebuilt = W[:, :, u].permute(0, 2, 1, 3)  # [d][t][c][s] = W[d, c, (t-s) mod T]
         if not torch.allclose(rebuilt, A, rtol=0.0, atol=atol):
             raise ValueError("weight is not group-circulant for this T")
@@ -155,7 +195,8 @@ class EqLinear(torch.nn.Module):
             if not torch.allclose(B, B[:, :1].expand(D, T), rtol=0.0, atol=atol):
                 raise ValueError("bias is not constant over the group index")
             b = B[:, 0].contiguous()
-        m = cls(C, D, T, bias=b is not None, dtype=weight.dtype, device=weight.device)
+        m = cls(C, D, T, bias=b is not None, dtype=weight.dtype, device=weight.device,
+                group=group)
         with torch.no_grad():
             m.weight.copy_(W)
             if b is not None:

@@ -15,6 +15,7 @@ import group_dft_structured_b200 as F
 from group_dft_structured_b200.module import EqLinear, mode_for
 from group_dft_structured_b200.workloads import make_inputs
 from oracle import feql_ct_oracle as O
+from oracle import feql_p4m_oracle as P4M
 
 
 def dense_layer(W, b):
@@ -75,6 +76,21 @@ def test_from_unrolled_rejects_non_equivariant_layers():
         EqLinear.from_unrolled(At, bt, 8)  # 12 x 8 is not a multiple of 8 x 8
     with pytest.raises(ValueError):
         EqLinear.from_unrolled(At[:, :6], None, 2)  # the 2-group reading is not circulant
+
+
+def test_from_unrolled_p4m_recovers_the_weights_and_rejects_the_cyclic_reading():
+    rng = np.random.default_rng(73)
+    C, D = 3, 5
+    W = rng.standard_normal((D, C, 8)).astype(np.float32)
+    b = rng.standard_normal(D).astype(np.float32)
+    A = torch.from_numpy(P4M.unrolled(W.astype(np.float64)).astype(np.float32))
+    bd = torch.from_numpy(np.repeat(b, 8))
+    m = EqLinear.from_unrolled(A, bd, 8, group="p4m")
+    assert m.group == "p4m" and np.array_equal(m.weight.detach().numpy(), W)
+    with pytest.raises(ValueError):
+        EqLinear.from_unrolled(A, bd, 8)  # a p4m layer is not C_8-circulant
+    with pytest.raises(ValueError):
+        EqLinear(3, 5, 4, group="p4m")
 
 
 def test_module_has_no_cpu_path():
@@ -175,6 +191,27 @@ def test_module_tracks_weight_updates_and_batch_shapes():
     ref2 = O.forward(x64, 2.0 * W64, b64).reshape(B, L, D * T)
     assert O.rel_err(_host(y2), ref2) <= 5e-3
     assert O.rel_err(_host(y1), O.forward(x64, W64, b64).reshape(B, L, D * T)) <= 5e-3
+
+
+@pytest.mark.gpu
+def test_module_p4m_forward_and_autograd_match_oracle():
+    _cuda_ready()
+    N, C, D = 300, 12, 48
+    inp = make_inputs(35, N, C, D, "fp16", T=8)
+    m = EqLinear(C, D, 8, dtype=torch.float16, device="cuda", group="p4m")
+    with torch.no_grad():
+        m.weight.copy_(torch.from_numpy(inp["W"]))
+        m.bias.copy_(torch.from_numpy(inp["b"]))
+    x = torch.from_numpy(inp["x"].reshape(N, C * 8)).cuda().requires_grad_(True)
+    g = torch.from_numpy(inp["dy"].reshape(N, D * 8)).cuda()
+    y = m(x)
+    (y * g).sum().backward()
+    x64, W64, b64, dy64 = (inp[k].astype(np.float64) for k in ("x", "W", "b", "dy"))
+    dW, db = P4M.backward_dw(x64, dy64)
+    assert P4M.rel_err(_host(y).reshape(N, D, 8), P4M.forward(x64, W64, b64)) <= 5e-3
+    assert P4M.rel_err(_host(x.grad).reshape(N, C, 8), P4M.backward_dx(dy64, W64)) <= 5e-3
+    assert P4M.rel_err(_host(m.weight.grad), dW) <= 5e-3
+    assert P4M.rel_err(_host(m.bias.grad), db) <= 5e-3
 
 
 @pytest.mark.gpu
