@@ -457,21 +457,27 @@ int launch_g8_dw(const void *x, const void *dy, __half *dW, __half *db, float *w
 // Shared memory a block may use on sm_100 (227 KB), less the base alignment.
 constexpr int kMlpSmemBudget = 227 * 1024 - 1024;
 
-// The plan depends only on (C, H, Co), so the weight buffer's layout does too:
-// the widest hidden slice (fewest fc1 MMAs: the kernel is bound by its MMA
+// The plan depends only on (C, H, Co), so the weight buffer's layout does too.
+// The widest hidden slice (fewest fc1 MMAs: the kernel is bound by its MMA
 // issue) whose two fc1 accumulators and the fc2 accumulator fit 512 TMEM
-// columns, with two x tile buffers if they fit, else one.
+// columns; for it, both layers' weights resident if they fit beside the
+// buffers, else streamed per hidden slice through a ring of 3 or 2 slots; two
+// x tile buffers if they fit, else one.
 int plan_mlp(int C, int H, int Co, TcMlpParams *out) {
-  if (align_up(Co, 16) > 64) return FEQL_ERR_UNSUPPORTED;
+  if (align_up(Co, 16) > 96) return FEQL_ERR_UNSUPPORTED;  // fc2 accumulator: 4 * 96 columns
   const int hs_opts[4] = {64, 48, 32, 16};
+  const int slot_opts[3] = {0, 3, 2};  // 0: resident
   for (int hs_max : hs_opts) {
-    for (int nx = 2; nx >= 1; --nx) {
-      TcMlpParams p;
-      p.P = make_mlp_plan(C, H, Co, hs_max);
-      p.nx = nx;
-      if (mlp_tmem_cols(p.P) > 512 || mlp_smem(p).total > kMlpSmemBudget) continue;
-      *out = p;
-      return FEQL_OK;
+    for (int wslots : slot_opts) {
+      for (int nx = 2; nx >= 1; --nx) {
+        TcMlpParams p;
+        p.P = make_mlp_plan(C, H, Co, hs_max);
+        p.nx = nx;
+        p.wslots = wslots;
+        if (mlp_tmem_cols(p.P) > 512 || mlp_smem(p).total > kMlpSmemBudget) continue;
+        *out = p;
+        return FEQL_OK;
+      }
     }
   }
   return FEQL_ERR_UNSUPPORTED;

@@ -17,9 +17,10 @@
 // within 5e-4 of the exact z*Phi(z) for every z.
 //
 // One persistent CTA per SM, 128-token tiles, 22 warps:
-//   warp 0        TMA: the resident Fourier weights of both layers (once), then
-//                 each tile's x chunks [128 tokens x 16 channels x 4] into one
-//                 of `nx` tile buffers
+//   warp 0        TMA: the Fourier weights of both layers, resident (loaded
+//                 once) or, when they do not fit, streamed per hidden slice
+//                 through a ring of slots; each tile's x chunks [128 tokens x 16
+//                 channels x 4] into one of `nx` tile buffers
 //   warp 1        TMEM allocator + single-thread MMA issuer
 //   warps 2..5    transform: rDFT of the x tile in place into four K-major
 //                 planes per chunk (V0, V2, Re V1, -Im V1)
@@ -132,6 +133,8 @@ __global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__r
   }
 }
 
+constexpr int kMlpMaxWSlots = 4;  // weight ring slots (streaming mode)
+
 struct TcMlpParams {
   MlpPlan P;
   const uint8_t *wt;   // Fourier weights (MlpPlan layout)
@@ -140,26 +143,37 @@ struct TcMlpParams {
   int64_t N;
   int nM;              // token tiles
   int nx;              // x tile buffers (1 or 2)
+  int wslots;          // 0: both layers' weights resident; else a ring of this many
+                       // slots, each holding one hidden slice's fc1 and fc2 weights
 };
 
 struct MlpSmem {
   int w1, w2, x0, h0, y0, b1, b2, bars, total;
   int xtile, htile;    // bytes of one x tile buffer / one hidden buffer
+  int w1s, w2s, wslot; // streaming: a slice's fc1 / fc2 weight bytes, one ring slot
 };
 
 __host__ __device__ inline MlpSmem mlp_smem(const TcMlpParams &p) {
   MlpSmem s;
   s.xtile = p.P.nK1 * kMlpChunkBytes;
   s.htile = (p.P.HS / kCK) * kMlpChunkBytes;
+  s.w1s = p.P.nK1 * p.P.w1_chunk;
+  s.w2s = (p.P.HS / kCK) * p.P.w2_chunk;
+  s.wslot = static_cast<int>(align_up(s.w1s, 1024) + align_up(s.w2s, 1024));
   s.w1 = 0;
-  s.w2 = static_cast<int>(align_up(p.P.w1_bytes, 1024));
-  s.x0 = s.w2 + static_cast<int>(align_up(p.P.w2_bytes, 1024));
+  if (p.wslots == 0) {
+    s.w2 = static_cast<int>(align_up(p.P.w1_bytes, 1024));
+    s.x0 = s.w2 + static_cast<int>(align_up(p.P.w2_bytes, 1024));
+  } else {  // slot k: fc1 part at k * wslot, fc2 part after it
+    s.w2 = static_cast<int>(align_up(s.w1s, 1024));
+    s.x0 = p.wslots * s.wslot;
+  }
   s.h0 = s.x0 + p.nx * s.xtile;
   s.y0 = s.h0 + 2 * s.htile;
   s.b1 = s.y0 + 4 * kMlpYBoxes * 4096;
   s.b2 = s.b1 + p.P.nS * p.P.HS * 4;
   s.bars = s.b2 + static_cast<int>(align_up(p.P.BD2 * 4, 16));
-  s.total = s.bars + 24 * 8 + 16;
+  s.total = s.bars + 32 * 8 + 16;
   return s;
 }
 
@@ -203,7 +217,8 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
   uint64_t *a1full = bars + 7, *a1empty = bars + 9;
   uint64_t *hready = bars + 11, *hempty = bars + 13;
   uint64_t *a2full = bars + 15, *a2empty = bars + 17, *final_bar = bars + 19;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
+  uint64_t *wsfull = bars + 20, *wsempty = bars + 24;  // weight ring (streaming mode)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 28);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int hs = P.HS, nS = P.nS;
@@ -224,6 +239,10 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       mbar_init(&a2empty[b], 4);
     }
     mbar_init(final_bar, 1);
+    for (int k = 0; k < kMlpMaxWSlots; ++k) {
+      mbar_init(&wsfull[k], 1);
+      mbar_init(&wsempty[k], 1);
+    }
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < nS * hs / 2; i += blockDim.x) {  // b1 / 2, like fc1's accumulators
@@ -255,13 +274,15 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
       tma_prefetch_desc(&tm_out);
-      if (static_cast<int>(blockIdx.x) < p.nM) {
+      if (p.wslots == 0 && static_cast<int>(blockIdx.x) < p.nM) {
         mbar_arrive_expect_tx(wfull, static_cast<uint32_t>(P.w1_bytes + P.w2_bytes));
         bulk_load(smem + L.w1, p.wt, static_cast<uint32_t>(P.w1_bytes), wfull);
         bulk_load(smem + L.w2, p.wt + P.off_w2, static_cast<uint32_t>(P.w2_bytes), wfull);
       }
-      int xb = 0;
-      uint32_t xph = 0;
+      // in the order the MMA warp consumes them: a tile's x, then (streaming) the
+      // weights of each of its hidden slices
+      int xb = 0, ws = 0;
+      uint32_t xph = 0, wph = 0;
       for (int m = blockIdx.x; m < p.nM; m += gridDim.x) {
         if (ok) ok = mbar_wait(&xempty[xb], xph ^ 1);
         if (ok) {
@@ -271,6 +292,18 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             tma_load_2d(xt + kc * kMlpChunkBytes, &tm_in, kc * (kCK * kT), m * kBM, &xfull[xb]);
         }
         if (++xb == p.nx) { xb = 0; xph ^= 1; }
+        for (int sl = 0; p.wslots > 0 && sl < nS; ++sl) {
+          if (ok) ok = mbar_wait(&wsempty[ws], wph ^ 1);
+          if (ok) {
+            uint8_t *dst = smem + ws * L.wslot;
+            mbar_arrive_expect_tx(&wsfull[ws], static_cast<uint32_t>(L.w1s + L.w2s));
+            bulk_load(dst, p.wt + static_cast<int64_t>(sl) * L.w1s, static_cast<uint32_t>(L.w1s),
+                      &wsfull[ws]);
+            bulk_load(dst + L.w2, p.wt + P.off_w2 + static_cast<int64_t>(sl) * L.w2s,
+                      static_cast<uint32_t>(L.w2s), &wsfull[ws]);
+          }
+          if (++ws == p.wslots) { ws = 0; wph ^= 1; }
+        }
       }
     }
   } else if (warp == 1) {
@@ -292,27 +325,34 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       const uint32_t w1r16 = (hs * 32) >> 4, w1c16 = P.w1_chunk >> 4;
       const uint32_t w2r16 = (P.BD2 * 32) >> 4, w2c16 = P.w2_chunk >> 4;
       const int kh_per = hs / kCK;
-      if (static_cast<int>(blockIdx.x) < p.nM) ok = __all_sync(0xffffffffu, mbar_wait(wfull, 0));
+      if (p.wslots == 0 && static_cast<int>(blockIdx.x) < p.nM)
+        ok = __all_sync(0xffffffffu, mbar_wait(wfull, 0));
+      const uint32_t wslot16 = L.wslot >> 4, w2off16 = L.w2 >> 4;
       // The issuing thread's scalar work adds to every MMA, so the two cursors
       // below advance by increments (no divisions).
       int s1 = 0, xb = 0;      // fc1 cursor: slice s1 of the tile in x buffer xb
       uint32_t xph = 0;
       int s2 = 0, ab = 0;      // fc2 cursor: slice s2 of the tile in fc2 accumulator ab
       uint32_t abph = 0;
+      int w1s = 0, w2s = 0;    // streaming: weight ring slots of fc1's and fc2's slice
+      uint32_t w1ph = 0;
       // fc1 of hidden slice gs: its x tile (ready once per tile), fc1 accumulator gs % 2
       auto fc1 = [&](int gs) {
-        const int b = gs & 1, s = s1, x = xb;
+        const int b = gs & 1, s = s1, x = xb, wsl = w1s;
         if (s == 0 && ok) ok = mbar_wait(&xready[x], xph);
         if (ok) ok = mbar_wait(&a1empty[b], ((gs >> 1) & 1) ^ 1);
+        if (p.wslots > 0 && ok) ok = mbar_wait(&wsfull[wsl], w1ph);
         ok = __all_sync(0xffffffffu, ok);
         if (++s1 == nS) {
           s1 = 0;
           if (++xb == p.nx) { xb = 0; xph ^= 1; }
         }
+        if (p.wslots > 0 && ++w1s == p.wslots) { w1s = 0; w1ph ^= 1; }
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc = tmem_base + b * 4 * hs;
-        uint32_t xd = x0 + x * xt16, wd = w1_0 + s * P.nK1 * w1c16;
+        uint32_t xd = x0 + x * xt16;
+        uint32_t wd = p.wslots > 0 ? w1_0 + wsl * wslot16 : w1_0 + s * P.nK1 * w1c16;
         if (elect_one()) {
           for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
@@ -328,7 +368,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       };
       // fc2 over the activations of slice gs into fc2 accumulator (tile % nacc2)
       auto fc2 = [&](int gs) {
-        const int b = gs & 1, s = s2, a = ab;
+        const int b = gs & 1, s = s2, a = ab, wsl = w2s;
         if (s == 0 && ok) ok = mbar_wait(&a2empty[a], abph ^ 1);
         if (ok) ok = mbar_wait(&hready[b], (gs >> 1) & 1);
         ok = __all_sync(0xffffffffu, ok);
@@ -336,10 +376,13 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           s2 = 0;
           if (++ab == nacc2) { ab = 0; abph ^= 1; }
         }
+        if (p.wslots > 0 && ++w2s == p.wslots) w2s = 0;
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc2 = tmem_base + acc2_col + a * 4 * P.BD2;
-        uint32_t hd = h0 + b * ht16, wd = w2_0 + s * kh_per * w2c16;
+        uint32_t hd = h0 + b * ht16;
+        // (streaming: the slot's fc1 part was waited for by fc1 of the same slice)
+        uint32_t wd = p.wslots > 0 ? w1_0 + wsl * wslot16 + w2off16 : w2_0 + s * kh_per * w2c16;
         if (elect_one()) {
           for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
             const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
@@ -350,6 +393,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           }
           mma_commit(&hempty[b]);
           if (s == nS - 1) mma_commit(&a2full[a]);
+          if (p.wslots > 0) mma_commit(&wsempty[wsl]);  // the slice's weights are consumed
         }
         __syncwarp();
       };

@@ -26,7 +26,7 @@ Rete"): a ViT MLP fc1 at 64 x 197 tokens and a Swin stage-1 stream at
 128 x 3136 tokens; no dataset is involved.  The C_8 workload keeps the Swin
 stream's token count and unrolled widths (96 -> 384) with T = 8.  The MLP
 workload is the Swin-T stage-1 block (96 -> 384 -> 96 unrolled) on the same
-token stream, and the p4m workload the same stream for the point group D4
+token stream (and the ViT-Ti block, 192 -> 768 -> 192, at the ViT batch), and the p4m workload the same stream for the point group D4
 (8 group elements: rotations and reflections, element (r, m) at index 4 m + r).
 """
 
@@ -73,6 +73,9 @@ WORKLOADS = {
     7: Workload(7, "p4_mlp_fp16_swin_N401408_C24_H96", 401408, 24, 96, "fp16", ("mlp",),
                 "Swin stage-1-like MLP block fc1 -> GELU -> fc2 (96->384->96 unrolled); "
                 "D is the hidden width, the output has C channels"),
+    9: Workload(9, "p4_mlp_fp16_vit_ti_N12608_C48_H192", 12608, 48, 192, "fp16", ("mlp",),
+                "ViT-Ti-like MLP block at 64x197 tokens (192->768->192 unrolled; weights "
+                "streamed); D is the hidden width, the output has C channels"),
 }
 
 

@@ -210,12 +210,15 @@ int feql_p4m_backward_dw(const void *x, const void *dy, void *dW, void *db, void
  *   x  : device [N][C][4]     y : device [N][Co][4] (written)
  *   W1 : device [H][C][4]     b1: device [H] or NULL
  *   W2 : device [Co][H][4]    b2: device [Co] or NULL
- * FEQL_FP16 only (other modes FEQL_ERR_UNSUPPORTED).  C and Co even; Co <= 64;
- * the Fourier weights of both layers must fit in shared memory beside the
- * tile buffers (e.g. C = 24, H = 96, Co = 24, the Swin stage-1 block): shapes
- * that do not fit return FEQL_ERR_UNSUPPORTED (feql_mlp_weight_fft_bytes
- * returns 0 for them).  Conventions otherwise as above (device pointers,
- * 16-byte alignment, stream-ordered, N == 0 is a no-op). */
+ * FEQL_FP16 only (other modes FEQL_ERR_UNSUPPORTED).  C and Co even; Co <= 96;
+ * one 128-token tile of x (C rounded up to 16 channels, 2 KB per channel) must
+ * fit in shared memory beside the other buffers (C <= 96).  The Fourier weights
+ * of both layers stay resident in shared memory when they fit (e.g. the Swin
+ * stage-1 block, C = 24, H = 96, Co = 24) and are otherwise streamed per hidden
+ * slice (e.g. the ViT-Ti block 48 -> 192 -> 48 or ViT-S 96 -> 384 -> 96); other
+ * shapes return FEQL_ERR_UNSUPPORTED (feql_mlp_weight_fft_bytes returns 0 for
+ * them).  Conventions otherwise as above (device pointers, 16-byte alignment,
+ * stream-ordered, N == 0 is a no-op). */
 size_t feql_mlp_weight_fft_bytes(int C, int H, int Co, int dtype);
 /* Fourier weights of both layers in the kernel's tile layout (opaque; depends
  * only on C, H, Co): What must hold feql_mlp_weight_fft_bytes(C, H, Co, dtype) bytes. */

@@ -61,9 +61,11 @@ def ref_mlp(inp, with_bias=True, rows=None):
 
 
 # (N, C, H, Co): the Swin stage-1 block with a ragged tail, tiny, single hidden slice,
-# padded hidden and output channels, many slices, one x tile buffer (wide C, Co = 64)
+# padded hidden and output channels, many slices, one x tile buffer (wide C, Co = 64);
+# streamed weights: the ViT-Ti and ViT-S blocks, padded output channels (Co = 80)
 SHAPES = [(300, 24, 96, 24), (1, 8, 16, 8), (1000, 16, 64, 16), (129, 6, 40, 10),
-          (517, 32, 128, 32), (2000, 48, 64, 64), (333, 2, 16, 2)]
+          (517, 32, 128, 32), (2000, 48, 64, 64), (333, 2, 16, 2),
+          (1000, 48, 192, 48), (400, 96, 384, 96), (300, 64, 256, 80), (260, 24, 96, 80)]
 
 
 @pytest.mark.parametrize("N,C,H,Co", SHAPES)
@@ -106,8 +108,9 @@ def test_mlp_zero_tokens_and_output_stays_in_its_buffer():
 
 
 def test_mlp_unsupported_shapes_and_modes():
-    assert F.feql_mlp_weight_fft_bytes(24, 96, 80, FP16) == 0       # Co > 64
-    assert F.feql_mlp_weight_fft_bytes(48, 192, 48, FP16) == 0      # weights do not fit
+    assert F.feql_mlp_weight_fft_bytes(24, 96, 112, FP16) == 0      # Co > 96
+    assert F.feql_mlp_weight_fft_bytes(192, 768, 96, FP16) == 0     # x tile does not fit
+    assert F.feql_mlp_weight_fft_bytes(48, 192, 48, FP16) > 0       # streamed weights
     assert F.feql_mlp_weight_fft_bytes(24, 96, 24, F.FEQL_FP32) == 0
     assert F.feql_mlp_weight_fft_bytes(24, 96, 24, FP16) > 0
     x = torch.zeros((16, 5, 4), dtype=torch.float16, device="cuda")
