@@ -512,11 +512,11 @@ int launch_mlp(const void *x, const uint8_t *wt, const __half *b1, const __half 
   if (st != FEQL_OK) return st;
   st = make_tmap_f16(&tm_out, y, N, static_cast<int64_t>(p.P.Co) * kT, 32);
   if (st != FEQL_OK) return st;
-  if (cudaFuncSetAttribute(tc_mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  auto kernel = p.wslots > 0 ? tc_mlp_kernel<true> : tc_mlp_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FEQL_ERR_CUDA;
   const int grid = p.nM < dev.sms ? p.nM : dev.sms;
-  tc_mlp_kernel<<<grid, kMlpThreads, smem, stream>>>(tm_in, tm_out, p);
+  kernel<<<grid, kMlpThreads, smem, stream>>>(tm_in, tm_out, p);
   return launch_status();
 }
 

@@ -201,6 +201,8 @@ __device__ __forceinline__ uint32_t gelu_half_arg_h2(uint32_t uu) {
 }
 
 // 22 warps: six on the busiest 16K-register sub-partition, 80 registers each.
+// kStream: weights streamed per hidden slice (p.wslots > 0) or resident.
+template <bool kStream>
 __global__ void __maxnreg__(kMlpMaxRegs)
 tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
               const TcMlpParams p) {
@@ -274,7 +276,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
       tma_prefetch_desc(&tm_out);
-      if (p.wslots == 0 && static_cast<int>(blockIdx.x) < p.nM) {
+      if (!kStream && static_cast<int>(blockIdx.x) < p.nM) {
         mbar_arrive_expect_tx(wfull, static_cast<uint32_t>(P.w1_bytes + P.w2_bytes));
         bulk_load(smem + L.w1, p.wt, static_cast<uint32_t>(P.w1_bytes), wfull);
         bulk_load(smem + L.w2, p.wt + P.off_w2, static_cast<uint32_t>(P.w2_bytes), wfull);
@@ -292,7 +294,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             tma_load_2d(xt + kc * kMlpChunkBytes, &tm_in, kc * (kCK * kT), m * kBM, &xfull[xb]);
         }
         if (++xb == p.nx) { xb = 0; xph ^= 1; }
-        for (int sl = 0; p.wslots > 0 && sl < nS; ++sl) {
+        for (int sl = 0; kStream && sl < nS; ++sl) {
           if (ok) ok = mbar_wait(&wsempty[ws], wph ^ 1);
           if (ok) {
             uint8_t *dst = smem + ws * L.wslot;
@@ -325,7 +327,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
       const uint32_t w1r16 = (hs * 32) >> 4, w1c16 = P.w1_chunk >> 4;
       const uint32_t w2r16 = (P.BD2 * 32) >> 4, w2c16 = P.w2_chunk >> 4;
       const int kh_per = hs / kCK;
-      if (p.wslots == 0 && static_cast<int>(blockIdx.x) < p.nM)
+      if (!kStream && static_cast<int>(blockIdx.x) < p.nM)
         ok = __all_sync(0xffffffffu, mbar_wait(wfull, 0));
       const uint32_t wslot16 = L.wslot >> 4, w2off16 = L.w2 >> 4;
       // The issuing thread's scalar work adds to every MMA, so the two cursors
@@ -341,18 +343,18 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
         const int b = gs & 1, s = s1, x = xb, wsl = w1s;
         if (s == 0 && ok) ok = mbar_wait(&xready[x], xph);
         if (ok) ok = mbar_wait(&a1empty[b], ((gs >> 1) & 1) ^ 1);
-        if (p.wslots > 0 && ok) ok = mbar_wait(&wsfull[wsl], w1ph);
+        if (kStream && ok) ok = mbar_wait(&wsfull[wsl], w1ph);
         ok = __all_sync(0xffffffffu, ok);
         if (++s1 == nS) {
           s1 = 0;
           if (++xb == p.nx) { xb = 0; xph ^= 1; }
         }
-        if (p.wslots > 0 && ++w1s == p.wslots) { w1s = 0; w1ph ^= 1; }
+        if (kStream && ++w1s == p.wslots) { w1s = 0; w1ph ^= 1; }
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc = tmem_base + b * 4 * hs;
         uint32_t xd = x0 + x * xt16;
-        uint32_t wd = p.wslots > 0 ? w1_0 + wsl * wslot16 : w1_0 + s * P.nK1 * w1c16;
+        uint32_t wd = kStream ? w1_0 + wsl * wslot16 : w1_0 + s * P.nK1 * w1c16;
         if (elect_one()) {
           for (int kc = 0; kc < P.nK1; ++kc, xd += ch16, wd += w1c16) {
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
@@ -376,13 +378,13 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           s2 = 0;
           if (++ab == nacc2) { ab = 0; abph ^= 1; }
         }
-        if (p.wslots > 0 && ++w2s == p.wslots) w2s = 0;
+        if (kStream && ++w2s == p.wslots) w2s = 0;
         tc_fence_after();
         if (!ok) return;
         const uint32_t acc2 = tmem_base + acc2_col + a * 4 * P.BD2;
         uint32_t hd = h0 + b * ht16;
         // (streaming: the slot's fc1 part was waited for by fc1 of the same slice)
-        uint32_t wd = p.wslots > 0 ? w1_0 + wsl * wslot16 + w2off16 : w2_0 + s * kh_per * w2c16;
+        uint32_t wd = kStream ? w1_0 + wsl * wslot16 + w2off16 : w2_0 + s * kh_per * w2c16;
         if (elect_one()) {
           for (int kh = 0; kh < kh_per; ++kh, hd += ch16, wd += w2c16) {
             const uint32_t acc_in = (s == 0 && kh == 0) ? 0u : 1u;
@@ -393,7 +395,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           }
           mma_commit(&hempty[b]);
           if (s == nS - 1) mma_commit(&a2full[a]);
-          if (p.wslots > 0) mma_commit(&wsempty[wsl]);  // the slice's weights are consumed
+          if (kStream) mma_commit(&wsempty[wsl]);  // the slice's weights are consumed
         }
         __syncwarp();
       };
