@@ -100,3 +100,57 @@ def test_product_path_has_no_oracle_dependency():
                 src = open(os.path.join(root, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", src, flags=re.M), f
                 assert "feql_oracle" not in src, f
+
+
+def test_group_and_block_entry_points_reject_bad_arguments_before_cuda(lib):
+    p = 1 << 20  # aligned fake address; never dereferenced
+    FP16, FP32 = F.FEQL_FP16, F.FEQL_FP32
+    INV, UNS = F.FEQL_ERR_INVALID_ARG, F.FEQL_ERR_UNSUPPORTED
+    # cyclic C_T: orders other than 4 and 8, fp32 for T = 8, bad sizes and pointers
+    assert lib.feql_ct_forward(6, p, p, None, p, 8, 4, 4, FP16, None) == UNS
+    assert lib.feql_ct_forward(8, p, p, None, p, 8, 4, 4, FP32, None) == UNS
+    assert lib.feql_ct_forward(8, p, p, None, p, -1, 4, 4, FP16, None) == INV
+    assert lib.feql_ct_forward(8, p + 4, p, None, p, 8, 4, 4, FP16, None) == INV
+    assert lib.feql_ct_backward_dx(8, p, None, p, 8, 4, 4, FP16, None) == INV
+    assert lib.feql_ct_backward_dw(8, p, p, None, None, p, 0, 8, 4, 4, FP16, None) == INV
+    assert lib.feql_ct_weight_fft(8, None, p, 4, 4, FP16, None) == INV
+    # p4m
+    assert lib.feql_p4m_forward(p, p, None, p, 8, 4, 4, FP32, None) == UNS
+    assert lib.feql_p4m_forward(p, p, None, p, 8, 0, 4, FP16, None) == INV
+    assert lib.feql_p4m_backward_dx(p, None, p, 8, 4, 4, FP16, None) == INV
+    assert lib.feql_p4m_backward_dw(p, p, None, None, p, 0, 8, 4, 4, FP16, None) == INV
+    assert lib.feql_p4m_weight_fft(None, p, 4, 4, FP16, None) == INV
+    assert lib.feql_p4m_weight_fft(p, p, 4, 4, 17, None) == INV
+    # MLP block: odd C or Co (TMA rows), bad sizes and pointers
+    assert lib.feql_mlp_forward(p, p, None, None, p, 8, 5, 16, 8, FP16, None) == UNS
+    assert lib.feql_mlp_forward(p, p, None, None, p, 8, 4, 16, 7, FP16, None) == UNS
+    assert lib.feql_mlp_forward(p, p, None, None, p, -1, 4, 16, 8, FP16, None) == INV
+    assert lib.feql_mlp_forward(p, p, p + 2, None, p, 8, 4, 16, 8, FP16, None) == INV
+    assert lib.feql_mlp_weight_fft(None, p, p, 4, 16, 8, FP16, None) == INV
+
+
+def _g8_bytes(C, D, rows):
+    def plan(Ci, Do):
+        nK, nD = -(-Ci // 16), -(-Do // 64)
+        BD = -(-(-(-Do // nD)) // 16) * 16
+        return nD * nK * rows * BD * 16 * 2
+    al = lambda v: -(-v // 1024) * 1024
+    return al(plan(C, D)) + al(plan(D, C))
+
+
+@pytest.mark.parametrize("C,D", [(12, 48), (8, 8), (40, 130), (64, 16)])
+def test_order8_weight_buffer_sizes(lib, C, D):
+    # C_8: 11 weight rows per output channel (W0, W4, (Re, Im, -Re) of bins 1..3); p4m: 8
+    assert F.feql_ct_weight_fft_bytes(8, C, D, F.FEQL_FP16) == _g8_bytes(C, D, 11)
+    assert F.feql_p4m_weight_fft_bytes(C, D, F.FEQL_FP16) == _g8_bytes(C, D, 8)
+    assert F.feql_ct_weight_fft_bytes(4, C, D, F.FEQL_FP16) == F.feql_weight_fft_bytes(C, D, F.FEQL_FP16)
+    assert F.feql_p4m_weight_fft_bytes(C, D, F.FEQL_FP32) == 0
+
+
+def test_mlp_weight_buffer_covers_both_layers(lib):
+    # at least the tiled Fourier weights of fc1 and fc2 (5 planes per 16 channels of each)
+    for C, H, Co in [(24, 96, 24), (48, 192, 48), (96, 384, 96), (6, 40, 10)]:
+        n = F.feql_mlp_weight_fft_bytes(C, H, Co, F.FEQL_FP16)
+        a16 = lambda v: -(-v // 16) * 16
+        assert n >= 5 * 2 * (a16(C) * a16(H) + a16(H) * a16(Co)), (C, H, Co)
+    assert F.feql_mlp_weight_fft_bytes(192, 768, 192, F.FEQL_FP16) == 0
