@@ -13,6 +13,7 @@
 #include "../../include/feql.h"
 #include "plan.cuh"
 #include "simt.cuh"
+#include "simt_ct.cuh"
 #include "sm100.cuh"
 #include "tc_bwd.cuh"
 #include "tc_dw.cuh"
@@ -522,11 +523,116 @@ int launch_mlp(const void *x, const uint8_t *wt, const __half *b1, const __half 
 
 // Checks shared by the C_T entry points: a supported group order and mode.
 // Returns FEQL_OK for T = 8 in FEQL_FP16 (T = 4 is forwarded before this).
-int ct_check(int T, int dtype) {
-  if (T != 8) return FEQL_ERR_UNSUPPORTED;
+// For T != 4: the tensor-core kernels serve T = 8 in FEQL_FP16, the CUDA-core
+// kernels every order 2..16 in the other modes (and every other order in fp16).
+enum CtPath { kCtTensor8 = 1, kCtSimt = 2 };
+
+int ct_route(int T, int dtype, int *path) {
   if (!valid_dtype(dtype)) return FEQL_ERR_INVALID_ARG;
-  if (resolve(dtype) != FEQL_FP16) return FEQL_ERR_UNSUPPORTED;
+  if (T < 2 || T > kCtMaxT) return FEQL_ERR_UNSUPPORTED;
+  const int dt = resolve(dtype);
+  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  *path = (T == 8 && dt == FEQL_FP16) ? kCtTensor8 : kCtSimt;
   return FEQL_OK;
+}
+
+// ---------------------------------------------------------- C_T on CUDA cores
+#define FEQL_CT_ORDERS(X) X(2) X(3) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
+
+template <int T, typename Ty>
+int ct_simt_wfft_launch(const void *W, void *What, int C, int D, cudaStream_t s, int sms) {
+  ct_simt_wfft_kernel<T, Ty><<<grid_for(static_cast<int64_t>(C) * D, 256, sms), 256, 0, s>>>(
+      static_cast<const Ty *>(W), static_cast<float *>(What), C, D);
+  return launch_status();
+}
+
+template <int T, typename Ty>
+int ct_simt_pass_launch(const void *in, const float *Wp, const void *bias, void *out, int64_t N,
+                        int Ci, int Do, cudaStream_t s) {
+  const int64_t gx = cdiv(N, kCtTile);
+  if (gx > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(cdiv(Do, kCtTile)));
+  if (grid.y > 65535) return FEQL_ERR_UNSUPPORTED;
+  ct_simt_fwd_kernel<T, Ty><<<grid, kCtThreads, 0, s>>>(
+      static_cast<const Ty *>(in), Wp, static_cast<const Ty *>(bias), static_cast<Ty *>(out), N,
+      Ci, Do);
+  return launch_status();
+}
+
+struct CtDwPlan {
+  int tiles_d, tiles_c, splits;
+  int64_t split_len;
+};
+
+// Token splits: about two blocks per SM over all (d, c) tiles, at most 64 (the
+// reduce sums them serially per output).
+CtDwPlan make_ct_dw_plan(int64_t N, int C, int D, int sms) {
+  CtDwPlan p;
+  p.tiles_d = static_cast<int>(cdiv(D, kCtTile));
+  p.tiles_c = static_cast<int>(cdiv(C, kCtTile));
+  int64_t s = 2 * static_cast<int64_t>(sms) / (p.tiles_d * p.tiles_c);
+  if (s < 1) s = 1;
+  if (s > 64) s = 64;
+  const int64_t chunks = cdiv(N, kCtK);
+  if (s > chunks) s = chunks;
+  p.split_len = N > 0 ? align_up(cdiv(N, s), kCtK) : kCtK;
+  p.splits = N > 0 ? static_cast<int>(cdiv(N, p.split_len)) : 0;
+  return p;
+}
+
+int64_t ct_dw_ws_floats(const CtDwPlan &p, int T, int C, int D) {
+  return static_cast<int64_t>(p.splits) * (static_cast<int64_t>(T) * D * C + D);
+}
+
+template <int T, typename Ty>
+int ct_simt_dw_launch(const void *x, const void *dy, void *dW, void *db, float *ws, size_t ws_bytes,
+                      int64_t N, int C, int D, cudaStream_t s, int sms) {
+  const CtDwPlan p = make_ct_dw_plan(N, C, D, sms);
+  if (ws_bytes < static_cast<size_t>(ct_dw_ws_floats(p, T, C, D)) * 4) return FEQL_ERR_INVALID_ARG;
+  float *ws_db = ws + static_cast<int64_t>(p.splits) * T * D * C;
+  if (p.splits > 0) {
+    const int64_t grid = static_cast<int64_t>(p.splits) * p.tiles_d * p.tiles_c;
+    if (grid > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+    ct_simt_dw_kernel<T, Ty><<<static_cast<unsigned>(grid), kCtThreads, 0, s>>>(
+        static_cast<const Ty *>(x), static_cast<const Ty *>(dy), ws, ws_db, N, C, D, p.split_len,
+        p.tiles_d, p.tiles_c);
+  }
+  ct_simt_dw_reduce_kernel<T, Ty><<<grid_for(static_cast<int64_t>(D) * C + D, 256, sms), 256, 0, s>>>(
+      ws, ws_db, static_cast<Ty *>(dW), static_cast<Ty *>(db), p.splits, C, D);
+  return launch_status();
+}
+
+template <typename Ty>
+int ct_simt_wfft(int T, const void *W, void *What, int C, int D, cudaStream_t s, int sms) {
+  switch (T) {
+#define FEQL_CASE(t) case t: return ct_simt_wfft_launch<t, Ty>(W, What, C, D, s, sms);
+    FEQL_CT_ORDERS(FEQL_CASE)
+#undef FEQL_CASE
+    default: return FEQL_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename Ty>
+int ct_simt_pass(int T, const void *in, const float *Wp, const void *bias, void *out, int64_t N,
+                 int Ci, int Do, cudaStream_t s) {
+  switch (T) {
+#define FEQL_CASE(t) case t: return ct_simt_pass_launch<t, Ty>(in, Wp, bias, out, N, Ci, Do, s);
+    FEQL_CT_ORDERS(FEQL_CASE)
+#undef FEQL_CASE
+    default: return FEQL_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename Ty>
+int ct_simt_dw(int T, const void *x, const void *dy, void *dW, void *db, float *ws, size_t ws_bytes,
+               int64_t N, int C, int D, cudaStream_t s, int sms) {
+  switch (T) {
+#define FEQL_CASE(t) \
+  case t: return ct_simt_dw_launch<t, Ty>(x, dy, dW, db, ws, ws_bytes, N, C, D, s, sms);
+    FEQL_CT_ORDERS(FEQL_CASE)
+#undef FEQL_CASE
+    default: return FEQL_ERR_UNSUPPORTED;
+  }
 }
 
 
@@ -758,46 +864,91 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws
 // ---------------------------------------------------------------------------
 size_t feql_ct_weight_fft_bytes(int T, int C, int D, int dtype) {
   if (T == 4) return feql_weight_fft_bytes(C, D, dtype);
-  if (ct_check(T, dtype) != FEQL_OK) return 0;
-  return g8_weight_fft_bytes<Cyclic8>(C, D);
+  int path = 0;
+  if (ct_route(T, dtype, &path) != FEQL_OK || check_shape(C, D) != FEQL_OK) return 0;
+  if (path == kCtTensor8) return g8_weight_fft_bytes<Cyclic8>(C, D);
+  return static_cast<size_t>(2) * T * C * D * 4;  // fp32 planes [dir][plane][Do][Ci]
 }
 
 int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype,
                        feql_stream stream) {
   if (T == 4) return feql_weight_fft(W, What, C, D, dtype, stream);
-  const int st = ct_check(T, dtype);
+  int path = 0;
+  int st = ct_route(T, dtype, &path);
   if (st != FEQL_OK) return st;
-  return g8_weight_fft<Cyclic8>(W, What, C, D, stream);
+  if (path == kCtTensor8) return g8_weight_fft<Cyclic8>(W, What, C, D, stream);
+  if (W == nullptr || What == nullptr || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return is_half(resolve(dtype)) ? ct_simt_wfft<__half>(T, W, What, C, D, s, dev.sms)
+                                 : ct_simt_wfft<float>(T, W, What, C, D, s, dev.sms);
+}
+
+static int ct_pass(int T, const void *in, const void *What, const void *bias, void *out, int64_t N,
+                   int C, int D, int dtype, feql_stream stream, int dir) {
+  int path = 0;
+  const int st = ct_route(T, dtype, &path);
+  if (st != FEQL_OK) return st;
+  if (path == kCtTensor8) return g8_pass<Cyclic8>(in, What, bias, out, N, C, D, stream, dir);
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
+  if (N == 0) return FEQL_OK;
+  const float *Wp = static_cast<const float *>(What) + (dir == 0 ? 0 : static_cast<int64_t>(T) * C * D);
+  const int Ci = dir == 0 ? C : D, Do = dir == 0 ? D : C;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return is_half(resolve(dtype)) ? ct_simt_pass<__half>(T, in, Wp, bias, out, N, Ci, Do, s)
+                                 : ct_simt_pass<float>(T, in, Wp, bias, out, N, Ci, Do, s);
 }
 
 int feql_ct_forward(int T, const void *x, const void *What, const void *b, void *y, int64_t N,
                     int C, int D, int dtype, feql_stream stream) {
   if (T == 4) return feql_forward(x, What, b, y, N, C, D, dtype, stream);
-  const int st = ct_check(T, dtype);
-  if (st != FEQL_OK) return st;
-  return g8_pass<Cyclic8>(x, What, b, y, N, C, D, stream, 0);
+  return ct_pass(T, x, What, b, y, N, C, D, dtype, stream, 0);
 }
 
 int feql_ct_backward_dx(int T, const void *dy, const void *What, void *dx, int64_t N, int C, int D,
                         int dtype, feql_stream stream) {
   if (T == 4) return feql_backward_dx(dy, What, dx, N, C, D, dtype, stream);
-  const int st = ct_check(T, dtype);
-  if (st != FEQL_OK) return st;
-  return g8_pass<Cyclic8>(dy, What, nullptr, dx, N, C, D, stream, 1);
+  return ct_pass(T, dy, What, nullptr, dx, N, C, D, dtype, stream, 1);
 }
 
 size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int dtype) {
   if (T == 4) return feql_backward_dw_workspace_bytes(N, C, D, dtype);
-  if (ct_check(T, dtype) != FEQL_OK) return 0;
-  return g8_dw_workspace_bytes(N, C, D);
+  int path = 0;
+  if (ct_route(T, dtype, &path) != FEQL_OK) return 0;
+  if (path == kCtTensor8) return g8_dw_workspace_bytes(N, C, D);
+  if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
+  DeviceInfo dev;
+  if (device_info(&dev) != FEQL_OK) return 0;
+  return static_cast<size_t>(ct_dw_ws_floats(make_ct_dw_plan(N, C, D, dev.sms), T, C, D)) * 4;
 }
 
 int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db, void *ws,
                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream) {
   if (T == 4) return feql_backward_dw(x, dy, dW, db, ws, ws_bytes, N, C, D, dtype, stream);
-  const int st = ct_check(T, dtype);
+  int path = 0;
+  int st = ct_route(T, dtype, &path);
   if (st != FEQL_OK) return st;
-  return g8_dw<Cyclic8>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
+  if (path == kCtTensor8) return g8_dw<Cyclic8>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
+  if (dW == nullptr || ws == nullptr || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
+    return FEQL_ERR_INVALID_ARG;
+  if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws) ||
+      (db != nullptr && !aligned16(db)))
+    return FEQL_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  st = device_info(&dev);
+  if (st != FEQL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float *w = static_cast<float *>(ws);
+  return is_half(resolve(dtype))
+             ? ct_simt_dw<__half>(T, x, dy, dW, db, w, ws_bytes, N, C, D, s, dev.sms)
+             : ct_simt_dw<float>(T, x, dy, dW, db, w, ws_bytes, N, C, D, s, dev.sms);
 }
 
 // ---------------------------------------------------------------------------

@@ -154,13 +154,16 @@ int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW, void *db,
  * x[N][C][T], y[N][D][T], W[D][C][T], dW[D][C][T]; b, db [D].
  *   y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod T] x[n,c,s]
  * T = 4 is the p4 layer: every call forwards to the function above with the
- * same arguments (all modes).  T = 8: FEQL_FP16 only (kernels on the tensor
- * cores: bins 0 and 4 real, 1..3 complex, 14 real products instead of 64);
- * FEQL_FP32 modes return FEQL_ERR_UNSUPPORTED, and so does every other T.
- * Any C, D >= 1 for T = 8 (the row of 8C or 8D fp16 values is always a
- * multiple of 16 bytes).  Argument checks, N == 0, ownership, streams and
- * errors are as for the p4 functions; the Fourier buffer of T = 8 has its own
- * layout and size (feql_ct_weight_fft_bytes). */
+ * same arguments (all modes).  T = 8 in FEQL_FP16: tensor-core kernels (bins 0
+ * and 4 real, 1..3 complex, 14 real products instead of 64).  Every order
+ * 2 <= T <= 16 in FEQL_FP32 / FEQL_FP32_SIMT / FEQL_FP16_SIMT, and in
+ * FEQL_FP16 for T other than 4 and 8: CUDA-core kernels of the same method
+ * with the DFT twiddles of order T (non-dyadic for T = 3, 5, 6, 7, 12 ...;
+ * (2T-2)/T^2 or, for odd T, (2T-1)/T^2 of the dense products), fp32
+ * arithmetic on fp32 or fp16 data.  FEQL_FP32_3XTF32 and orders outside 2..16
+ * return FEQL_ERR_UNSUPPORTED.  Any C, D >= 1.  Argument checks, N == 0,
+ * ownership, streams and errors are as for the p4 functions; the Fourier
+ * buffer has its own layout and size per (T, dtype) (feql_ct_weight_fft_bytes). */
 size_t feql_ct_weight_fft_bytes(int T, int C, int D, int dtype);
 int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype,
                        feql_stream stream);

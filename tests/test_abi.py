@@ -106,9 +106,14 @@ def test_group_and_block_entry_points_reject_bad_arguments_before_cuda(lib):
     p = 1 << 20  # aligned fake address; never dereferenced
     FP16, FP32 = F.FEQL_FP16, F.FEQL_FP32
     INV, UNS = F.FEQL_ERR_INVALID_ARG, F.FEQL_ERR_UNSUPPORTED
-    # cyclic C_T: orders other than 4 and 8, fp32 for T = 8, bad sizes and pointers
-    assert lib.feql_ct_forward(6, p, p, None, p, 8, 4, 4, FP16, None) == UNS
-    assert lib.feql_ct_forward(8, p, p, None, p, 8, 4, 4, FP32, None) == UNS
+    # cyclic C_T: orders outside 2..16, split-TF32 for T != 4, bad sizes and pointers
+    assert lib.feql_ct_forward(17, p, p, None, p, 8, 4, 4, FP16, None) == UNS
+    assert lib.feql_ct_forward(1, p, p, None, p, 8, 4, 4, FP32, None) == UNS
+    assert lib.feql_ct_forward(8, p, p, None, p, 8, 4, 4, F.FEQL_FP32_3XTF32, None) == UNS
+    assert lib.feql_ct_forward(6, p, p, None, p, -1, 4, 4, FP16, None) == INV
+    assert lib.feql_ct_forward(6, p + 4, p, None, p, 8, 4, 4, FP32, None) == INV
+    assert lib.feql_ct_backward_dw(12, p, p, None, None, p, 0, 8, 4, 4, FP32, None) == INV
+    assert lib.feql_ct_weight_fft(5, None, p, 4, 4, FP32, None) == INV
     assert lib.feql_ct_forward(8, p, p, None, p, -1, 4, 4, FP16, None) == INV
     assert lib.feql_ct_forward(8, p + 4, p, None, p, 8, 4, 4, FP16, None) == INV
     assert lib.feql_ct_backward_dx(8, p, None, p, 8, 4, 4, FP16, None) == INV
@@ -144,6 +149,8 @@ def test_order8_weight_buffer_sizes(lib, C, D):
     assert F.feql_ct_weight_fft_bytes(8, C, D, F.FEQL_FP16) == _g8_bytes(C, D, 11)
     assert F.feql_p4m_weight_fft_bytes(C, D, F.FEQL_FP16) == _g8_bytes(C, D, 8)
     assert F.feql_ct_weight_fft_bytes(4, C, D, F.FEQL_FP16) == F.feql_weight_fft_bytes(C, D, F.FEQL_FP16)
+    for T in (2, 3, 6, 8, 12, 16):  # CUDA-core orders: fp32 planes of both directions
+        assert F.feql_ct_weight_fft_bytes(T, C, D, F.FEQL_FP32) == 2 * T * C * D * 4
     assert F.feql_p4m_weight_fft_bytes(C, D, F.FEQL_FP32) == 0
 
 

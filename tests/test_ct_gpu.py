@@ -136,13 +136,17 @@ def test_ct_order_4_is_the_p4_path():
 
 
 def test_ct_unsupported_orders_and_modes():
-    x = torch.zeros((16, 4, 6), dtype=torch.float16, device="cuda")
-    W = torch.zeros((4, 4, 6), dtype=torch.float16, device="cuda")
-    assert F.feql_ct_weight_fft_bytes(6, 4, 4, FP16) == 0
-    assert F.feql_ct_weight_fft_bytes(8, 4, 4, F.FEQL_FP32) == 0
-    y = torch.empty((16, 4, 6), dtype=torch.float16, device="cuda")
+    # orders outside 2..16 and the split-TF32 mode (p4 only) are rejected before any launch
+    assert F.feql_ct_weight_fft_bytes(17, 4, 4, FP16) == 0
+    assert F.feql_ct_weight_fft_bytes(1, 4, 4, FP16) == 0
+    assert F.feql_ct_weight_fft_bytes(8, 4, 4, F.FEQL_FP32_3XTF32) == 0
+    # the CUDA-core orders size their buffer as fp32 planes of both directions
+    assert F.feql_ct_weight_fft_bytes(6, 4, 4, FP16) == 2 * 6 * 4 * 4 * 4
+    x = torch.zeros((16, 4, 17), dtype=torch.float16, device="cuda")
+    W = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
+    y = torch.empty((16, 4, 17), dtype=torch.float16, device="cuda")
     with pytest.raises(F.FeqlError) as e:
-        F.feql_ct_forward(6, x, W, None, y, 16, 4, 4, FP16)
+        F.feql_ct_forward(17, x, W, None, y, 16, 4, 4, FP16)
     assert e.value.status == F.FEQL_ERR_UNSUPPORTED
 
 
