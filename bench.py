@@ -50,8 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
-                    help="workload id 1-9 (group_dft_structured_b200/workloads.py; 6 is the "
-                         "cyclic group C_8, 7 and 9 MLP blocks, 8 p4m)")
+                    help="workload id 1-10 (group_dft_structured_b200/workloads.py; 6 is the "
+                         "cyclic group C_8, 7 and 9 MLP blocks, 8 p4m, 10 C_6)")
     ap.add_argument("--dtype", choices=["fp16", "fp32"], default=None,
                     help="override the workload's dtype (e.g. the fp32 run of the square layer)")
     ap.add_argument("--e2e-steps", type=int, default=5)
