@@ -94,6 +94,25 @@ int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
 }
 
+// A [rows][boxes x 16 channels x 4] fp16 tensor seen as a stack of 16-channel
+// boxes: dims (64 elements, rows, boxes), strides (channels*8 B, 128 B).  One
+// load of a (64, box_rows, box_count) box writes box_count boxes of box_rows
+// 128-byte rows one after the other, the shared-memory image of box_count 2-D
+// loads.  Needs channels % 16 == 0 (else a box would run into the next row).
+int make_tmap_f16_boxes(CUtensorMap *m, const void *base, int64_t rows, int64_t channels,
+                        int box_rows, int box_count) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || channels % 16 != 0) return FEQL_ERR_CUDA;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(channels / 16)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(channels) * kT * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_count)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_dtype(int dt) { return dt >= FEQL_FP16 && dt <= FEQL_FP16_SIMT; }
@@ -250,6 +269,8 @@ TcDwParams make_tc_dw_plan(int64_t N, int C, int D, int sms) {
   while (cols < (p.merged ? 6 : 4) * p.CT) cols *= 2;
   p.tmem_cols = cols;
   p.stages = 0;
+  p.stack_dy = 0;
+  p.stack_x = 0;
   p.ws = nullptr;
   p.ws_db = nullptr;
   return p;
@@ -270,10 +291,15 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     while (p.stages > 2 && tc_dw_smem(p).total > budget) --p.stages;
     if (tc_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
     const int smem = tc_dw_smem(p).total + 1024;
+    // one load per operand and chunk when the channels form whole boxes, else
+    // one 2-D load per 16-channel box
     CUtensorMap tm_dy, tm_x;
-    int st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB);
+    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, p.N, p.D, p.TB, p.nqd_max) == FEQL_OK;
+    int st = FEQL_OK;
+    if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB);
     if (st != FEQL_OK) return st;
-    st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB);
+    p.stack_x = make_tmap_f16_boxes(&tm_x, x, p.N, p.C, p.TB, p.nqc_max) == FEQL_OK;
+    if (!p.stack_x) st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB);
     if (st != FEQL_OK) return st;
     if (cudaFuncSetAttribute(tc_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
@@ -281,10 +307,10 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     const int grid = p.tiles_d * p.tiles_c * p.splits;
     tc_dw_kernel<<<grid, kDwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  const int64_t rblocks = dw_reduce_blocks(p.C, p.D);
-  if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-  dw_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), kRedOut * kRedGroups, 0, stream>>>(
-      p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs);
+  const RedPlan rp = make_red_plan(p.C, p.D, dev.sms);
+  if (rp.blocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
+      p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs, rp.q, rp.wblocks);
   return launch_status();
 }
 
@@ -340,10 +366,10 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
       cudaSuccess)
     return FEQL_ERR_CUDA;
   tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, p);
-  const int64_t rblocks = dw_reduce_blocks(p.C, p.D);
-  if (rblocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-  dw_tc_reduce_kernel<<<static_cast<unsigned>(rblocks), kRedOut * kRedGroups, 0, stream>>>(
-      p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs);
+  const RedPlan rp = make_red_plan(p.C, p.D, dev.sms);
+  if (rp.blocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
+  dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
+      p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs, rp.q, rp.wblocks);
   return launch_status();
 }
 

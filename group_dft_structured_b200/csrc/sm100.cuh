@@ -80,6 +80,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Waits for two phases.  Both are tested (non-blocking) in one round trip
+// first: a satisfied mbarrier test issued behind tcgen05.mma instructions costs
+// ~250 cycles, so an issuing thread that needs two barriers pays that once.
+__device__ __forceinline__ bool mbar_wait2(uint64_t *bar0, uint32_t parity0, uint64_t *bar1,
+                                           uint32_t parity1) {
+  uint32_t both;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
+      "and.pred p, p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(both)
+      : "r"(smem_u32(bar0)), "r"(parity0), "r"(smem_u32(bar1)), "r"(parity1)
+      : "memory");
+  if (both) return true;
+  return mbar_wait(bar0, parity0) && mbar_wait(bar1, parity1);
+}
+
 // ----------------------------------------------------------------------------
 // Proxy fences, named barriers
 // ----------------------------------------------------------------------------
@@ -107,6 +126,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, int
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 3-D tiled load global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, int32_t c0,
+                                            int32_t c1, int32_t c2, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -185,8 +185,11 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       int s = 0;
       uint32_t ph = 0;
       for (int ch = 0; ch < nst; ++ch) {
-        if (ok) ok = mbar_wait(&full[s], ph);
-        if (ok) ok = mbar_wait(&tready[s], ph);
+        // tready implies full (the transform waited for the slot's TMA bytes
+        // before its release-arrive); the dX accumulator buffer of this stage
+        // is tested in the same round trip
+        const int b = ch % p.ndx;
+        if (ok) ok = mbar_wait2(&tready[s], ph, &dxempty[b], ((ch / p.ndx) & 1) ^ 1);
         tc_fence_after();
         const uint32_t st = stage_base + s * p.slots * kBwBox;
         // every operand below is the low descriptor word of one of these bases plus a
@@ -216,9 +219,6 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
             }
           }
         }
-        const int b = ch % p.ndx;
-        if (ok) ok = mbar_wait(&dxempty[b], ((ch / p.ndx) & 1) ^ 1);
-        tc_fence_after();
         if (ok) {
           const uint32_t acc = tmem_base + dx0 + b * 4 * p.BD;
           uint32_t ab = kl, wb = wl;  // running box and weight-chunk descriptor words

@@ -52,6 +52,7 @@ struct TcDwParams {
   int plane_bytes;       // 4 * (8 + nqc_max) * TB * 32
   int tmem_cols;
   int merged;            // 1: bin-1 products as two N = 2*CT MMAs (needs 6*CT TMEM columns)
+  int stack_dy, stack_x; // 1: the tensor map loads all of a tile's boxes at once (3-D box stack)
   float *ws;             // [splits][4][D][Cs]
   float *ws_db;          // [splits][D]
 };
@@ -172,12 +173,22 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
         if (ok) {
           uint8_t *raw = smem + L.raw0 + s * p.raw_bytes;
           const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * p.TB);
-          mbar_arrive_expect_tx(&full[s], nbox * p.TB * 128);
-          for (int q = 0; q < nqd; ++q)
-            tma_load_2d(raw + q * p.TB * 128, &tm_dy, (ti * kDwMT + q * 16) * kT, row, &full[s]);
-          for (int q = 0; q < nqc; ++q)
-            tma_load_2d(raw + (nqd + q) * p.TB * 128, &tm_x, (tj * p.CT + q * 16) * kT, row,
-                        &full[s]);
+          uint8_t *rawx = raw + p.nqd_max * p.TB * 128;
+          // a box stack always lands whole (boxes past the last channel read as zeros)
+          const int bd = p.stack_dy ? p.nqd_max : nqd, bc = p.stack_x ? p.nqc_max : nqc;
+          mbar_arrive_expect_tx(&full[s], (bd + bc) * p.TB * 128);
+          if (p.stack_dy) {
+            tma_load_3d(raw, &tm_dy, 0, row, ti * (kDwMT / 16), &full[s]);
+          } else {
+            for (int q = 0; q < nqd; ++q)
+              tma_load_2d(raw + q * p.TB * 128, &tm_dy, (ti * kDwMT + q * 16) * kT, row, &full[s]);
+          }
+          if (p.stack_x) {
+            tma_load_3d(rawx, &tm_x, 0, row, tj * (p.CT / 16), &full[s]);
+          } else {
+            for (int q = 0; q < nqc; ++q)
+              tma_load_2d(rawx + q * p.TB * 128, &tm_x, (tj * p.CT + q * 16) * kT, row, &full[s]);
+          }
         }
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
@@ -253,7 +264,9 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
       if (ok) ok = mbar_wait(&full[s], ph);
       if (ok) ok = mbar_wait(&pempty[pb], ((ch >> 1) & 1) ^ 1);
       if (active) {
-        const uint8_t *src = smem + L.raw0 + s * p.raw_bytes + b * p.TB * 128 + r * 128;
+        // dy boxes from the start of the slot, x boxes after nqd_max dy boxes
+        const int slot_box = is_dy ? b : p.nqd_max + (b - nqd);
+        const uint8_t *src = smem + L.raw0 + s * p.raw_bytes + slot_box * p.TB * 128 + r * 128;
         uint8_t *planes = smem + L.plane0 + pb * p.plane_bytes;
         uint32_t pl[4][8];
 #pragma unroll
@@ -342,63 +355,101 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
 
 // Sum of the split partials in a fixed order, inverse rDFT, fp16 cast:
 //   dW[d][c][u] = (G0 + (-1)^u G2)/4 + Re(G1 i^u)/2,   db[d] = sum of partials.
-// A block takes 32 consecutive (d, c) outputs (the last blocks take db); its
-// 16 warps each sum every 16th split, then warp 0 adds the 16 partial sums in
-// warp order — the same grouping on every run, so the result is bit-stable.
-constexpr int kRedOut = 32, kRedGroups = 16;
+// A dW block owns `q` quads (one d, four consecutive c, all four bins: 16
+// floats) and 256/q split groups; thread (group g, quad) adds splits g, g +
+// groups, ... with 16-byte loads, then the groups are folded pairwise in a fixed
+// tree through shared memory — the same order on every run, so the result is
+// bit-stable.  db blocks do the same for 32 scalars with 8 groups.  Many
+// independent loads per thread keep the partials (mostly still in L2) streaming.
+constexpr int kRedThreads = 256;
+constexpr int kRedDbItems = 32;
 
-__global__ void __launch_bounds__(kRedOut * kRedGroups)
+struct RedPlan {
+  int q;            // quads per dW block (4..32, a power of two)
+  int64_t wblocks;  // dW blocks, followed by the db blocks
+  int64_t blocks;
+};
+
+__host__ __device__ inline RedPlan make_red_plan(int C, int D, int sms) {
+  RedPlan r;
+  const int64_t nq = static_cast<int64_t>(D) * (align_up(C, 16) / 4);
+  r.q = 32;
+  while (r.q > 4 && cdiv(nq, r.q) < 2 * static_cast<int64_t>(sms)) r.q /= 2;
+  r.wblocks = cdiv(nq, r.q);
+  r.blocks = r.wblocks + cdiv(D, kRedDbItems);
+  return r;
+}
+
+__global__ void __launch_bounds__(kRedThreads)
 dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
                     __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
-                    int Cs) {
-  __shared__ float part[kRedGroups][4][kRedOut];
-  const int64_t plane = static_cast<int64_t>(D) * Cs;
-  const int64_t n = static_cast<int64_t>(D) * C;
-  const int64_t nblk_w = cdiv(n, kRedOut);
-  const int lo = threadIdx.x % kRedOut, grp = threadIdx.x / kRedOut;
-  if (blockIdx.x < nblk_w) {
-    const int64_t e = blockIdx.x * static_cast<int64_t>(kRedOut) + lo;
-    float g[4] = {0.f, 0.f, 0.f, 0.f};
-    if (e < n) {
-      const float *src = ws + (e / C) * Cs + (e % C);
-      for (int s = grp; s < splits; s += kRedGroups) {
-        const float *q = src + static_cast<int64_t>(s) * 4 * plane;
+                    int Cs, int q, int64_t wblocks) {
+  __shared__ float red[16][kRedThreads];
+  const int t = threadIdx.x;
+  if (blockIdx.x < wblocks) {
+    const int groups = kRedThreads / q;
+    const int quad = t % q, grp = t / q;
+    const int64_t plane = static_cast<int64_t>(D) * Cs;
+    const int nqr = Cs / 4;  // quads per d row
+    const int64_t item = blockIdx.x * static_cast<int64_t>(q) + quad;
+    const bool live = item < static_cast<int64_t>(D) * nqr;
+    float acc[16];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) g[k] += q[k * plane];
+    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+    if (live) {
+      const float *src = ws + item * 4;  // d * Cs + 4 * cq
+#pragma unroll 2
+      for (int sp = grp; sp < splits; sp += groups) {
+        const float *b0 = src + static_cast<int64_t>(sp) * 4 * plane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 v = *reinterpret_cast<const float4 *>(b0 + k * plane);
+          acc[4 * k + 0] += v.x;
+          acc[4 * k + 1] += v.y;
+          acc[4 * k + 2] += v.z;
+          acc[4 * k + 3] += v.w;
+        }
       }
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) part[grp][k][lo] = g[k];
-    __syncthreads();
-    if (grp == 0 && e < n) {
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int q = 0; q < kRedGroups; ++q)
+    for (int k = 0; k < 16; ++k) red[k][t] = acc[k];
+    for (int h = groups / 2; h >= 1; h /= 2) {
+      __syncthreads();
+      if (grp < h)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) t[k] += part[q][k][lo];
-      const float ev = 0.25f * (t[0] + t[1]), od = 0.25f * (t[0] - t[1]);
-      uint2 pk;
-      pk.x = pack_half2(ev + 0.5f * t[2], od - 0.5f * t[3]);
-      pk.y = pack_half2(ev - 0.5f * t[2], od + 0.5f * t[3]);
-      *reinterpret_cast<uint2 *>(dW + e * kT) = pk;
+        for (int k = 0; k < 16; ++k) red[k][t] += red[k][t + h * q];
+    }
+    __syncthreads();
+    if (grp == 0 && live) {
+      const int d = static_cast<int>(item / nqr), c0 = static_cast<int>(item % nqr) * 4;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + i;
+        if (c >= C) break;
+        const float g0 = red[i][t], g2 = red[4 + i][t], gr = red[8 + i][t], gi = red[12 + i][t];
+        const float ev = 0.25f * (g0 + g2), od = 0.25f * (g0 - g2);
+        uint2 pk;
+        pk.x = pack_half2(ev + 0.5f * gr, od - 0.5f * gi);
+        pk.y = pack_half2(ev - 0.5f * gr, od + 0.5f * gi);
+        *reinterpret_cast<uint2 *>(dW + (static_cast<int64_t>(d) * C + c) * kT) = pk;
+      }
     }
   } else if (db != nullptr) {
-    const int64_t d = (blockIdx.x - nblk_w) * kRedOut + lo;
+    constexpr int kGroups = kRedThreads / kRedDbItems;
+    const int di = t % kRedDbItems, grp = t / kRedDbItems;
+    const int64_t d = (blockIdx.x - wblocks) * kRedDbItems + di;
     float sdb = 0.f;
     if (d < D)
-      for (int s = grp; s < splits; s += kRedGroups) sdb += ws_db[static_cast<int64_t>(s) * D + d];
-    part[grp][0][lo] = sdb;
-    __syncthreads();
-    if (grp == 0 && d < D) {
-      float t = 0.f;
-      for (int q = 0; q < kRedGroups; ++q) t += part[q][0][lo];
-      db[d] = __float2half_rn(t);
+#pragma unroll 4
+      for (int sp = grp; sp < splits; sp += kGroups) sdb += ws_db[static_cast<int64_t>(sp) * D + d];
+    red[0][t] = sdb;
+    for (int h = kGroups / 2; h >= 1; h /= 2) {
+      __syncthreads();
+      if (grp < h) red[0][t] += red[0][t + h * kRedDbItems];
     }
+    __syncthreads();
+    if (grp == 0 && d < D) db[d] = __float2half_rn(red[0][t]);
   }
-}
-
-// Blocks for dw_tc_reduce_kernel: the dW outputs, then the db outputs.
-__host__ __device__ inline int64_t dw_reduce_blocks(int C, int D) {
-  return cdiv(static_cast<int64_t>(D) * C, kRedOut) + cdiv(D, kRedOut);
 }
 
 }  // namespace feql

@@ -208,7 +208,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
         const uint32_t acc = tmem_base + a * p.acc_stride;
         uint32_t wr = wr0;
         for (int kc = 0; kc < p.nK; ++kc, wr += chunk16) {
-          if (ok) ok = mbar_wait(&full[s], ph);
+          // tready implies full: every transform thread waited for the slot's
+          // TMA bytes before its release-arrive, so one acquire covers both
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
