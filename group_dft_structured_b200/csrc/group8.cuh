@@ -423,13 +423,28 @@ __host__ __device__ inline G8Smem g8_fwd_smem(const G8FwdParams &p) {
   return s;
 }
 
-__device__ __forceinline__ bool g8_unit(const G8FwdParams &p, int k, int &m, int &j) {
-  const int u = blockIdx.x + k * gridDim.x;
-  if (u >= p.n_units) return false;
-  m = u / p.nD;
-  j = u % p.nD;
-  return true;
-}
+// This CTA's work units u = blockIdx.x + k * gridDim.x as (token tile m,
+// output tile j), stepped without divisions (see TcUnits in tc_fwd.cuh).
+struct G8Units {
+  int m, j, dm, dj, nD, nM;
+  bool valid;
+  __device__ __forceinline__ explicit G8Units(const G8FwdParams &p) : nD(p.nD), nM(p.nM) {
+    m = static_cast<int>(blockIdx.x) / p.nD;
+    j = static_cast<int>(blockIdx.x) % p.nD;
+    dm = static_cast<int>(gridDim.x) / p.nD;
+    dj = static_cast<int>(gridDim.x) % p.nD;
+    valid = m < nM;
+  }
+  __device__ __forceinline__ void next() {
+    m += dm;
+    j += dj;
+    if (j >= nD) {
+      j -= nD;
+      ++m;
+    }
+    valid = m < nM;
+  }
+};
 
 // 14 warps over the 4 SM sub-partitions put 4 warps on one 16K-register slice.
 template <class Gp>
@@ -481,9 +496,10 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
       tma_prefetch_desc(&tm_out);
-      int s = 0, m, j;
+      int s = 0;
       uint32_t ph = 0;
-      for (int k = 0; g8_unit(p, k, m, j); ++k) {
+      for (G8Units U(p); U.valid; U.next()) {
+        const int m = U.m, j = U.j;
         for (int kc = 0; kc < p.nK; ++kc) {
           if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
           if (ok) {
@@ -509,14 +525,14 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
       const uint32_t x0 = desc_lo(desc_at(dsw32, smem_u32(smem + L.stage0)));
       const uint32_t stage16 = p.stage_bytes >> 4, pl16 = kG8Plane >> 4;
       const uint32_t w16 = 2 * p.BD;  // BD rows of 32 B, in 16-byte units
-      int s = 0, a = 0, m, j;
+      int s = 0, a = 0;
       uint32_t ph = 0, aph = 0;
-      for (int it = 0; g8_unit(p, it, m, j); ++it) {
+      for (G8Units U(p); U.valid; U.next()) {
         if (ok) ok = mbar_wait(&acc_empty[a], aph ^ 1);
         tc_fence_after();
         const uint32_t acc = tmem_base + a * p.acc_stride;
         for (int kc = 0; kc < p.nK; ++kc) {
-          if (ok) ok = mbar_wait(&full[s], ph);
+          // tready implies full (the transform waited for the TMA bytes first)
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
@@ -541,9 +557,9 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     // ---------------------------------------------------------- transform
     const int t = threadIdx.x - 64;
     const int r = t % kBM, bx = t / kBM;  // token row, box (channels 8 bx .. 8 bx + 7)
-    int s = 0, m, j;
+    int s = 0;
     uint32_t ph = 0;
-    for (int k = 0; g8_unit(p, k, m, j); ++k) {
+    for (G8Units U(p); U.valid; U.next()) {
       for (int kc = 0; kc < p.nK; ++kc) {
         if (ok) ok = mbar_wait(&full[s], ph);
         uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
@@ -574,9 +590,10 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     const int quad = warp & 3;
     const int groups = p.BD / 8;
     uint8_t *obase = smem + L.out0 + (warp - 10) * kG8NumOut * kG8OutBox;
-    int a = 0, oi = 0, m, j;
+    int a = 0, oi = 0;
     uint32_t aph = 0;
-    for (int it = 0; g8_unit(p, it, m, j); ++it) {
+    for (G8Units U(p); U.valid; U.next()) {
+      const int m = U.m, j = U.j;
       if (ok) ok = mbar_wait(&acc_full[a], aph);
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;

@@ -182,14 +182,13 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const uint32_t xb16 = (p.nqc * kBwPlane) >> 4;  // one x bin
       const uint32_t wl = desc_lo(desc_at(dk, wres)), chunk16 = p.chunk_bytes >> 4;
       const uint32_t w1 = (p.BD * 32) >> 4;
-      int s = 0;
-      uint32_t ph = 0;
+      int s = 0, b = 0;         // ring slot; dX accumulator buffer (stepped, no divisions)
+      uint32_t ph = 0, bph = 0;
       for (int ch = 0; ch < nst; ++ch) {
         // tready implies full (the transform waited for the slot's TMA bytes
         // before its release-arrive); the dX accumulator buffer of this stage
         // is tested in the same round trip
-        const int b = ch % p.ndx;
-        if (ok) ok = mbar_wait2(&tready[s], ph, &dxempty[b], ((ch / p.ndx) & 1) ^ 1);
+        if (ok) ok = mbar_wait2(&tready[s], ph, &dxempty[b], bph ^ 1);
         tc_fence_after();
         const uint32_t st = stage_base + s * p.slots * kBwBox;
         // every operand below is the low descriptor word of one of these bases plus a
@@ -233,6 +232,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           mma_commit(&empty[s]);
         }
         if (++s == p.stages) { s = 0; ph ^= 1; }
+        if (++b == p.ndx) { b = 0; bph ^= 1; }
       }
       mma_commit(dwfull);
     }
@@ -340,9 +340,10 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     const int quad = warp & 3;
     const int groups = p.BD / 16;
     const int64_t row_elems = static_cast<int64_t>(p.C) * kT;
-    for (int ch = 0; ch < nst; ++ch) {
-      const int b = ch % p.ndx;
-      if (ok) ok = mbar_wait(&dxfull[b], (ch / p.ndx) & 1);
+    int b = 0;
+    uint32_t bph = 0;
+    for (int ch = 0; ch < nst; ++ch, b = b + 1 == p.ndx ? 0 : b + 1, bph ^= (b == 0)) {
+      if (ok) ok = mbar_wait(&dxfull[b], bph);
       tc_fence_after();
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + dx0 + b * 4 * p.BD;
       // lanes 0..15 hold this warp's 16 tokens
@@ -350,41 +351,38 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const bool row_ok = lane < 16 && n < t_end;
       __half *drow = p.dx + n * row_elems;
       for (int g = 0; g < groups; ++g) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t y0[8], y2[8], y1r[8], y1i[8];
-          const uint32_t col = tl + g * 16 + h * 8;
-          // the TMEM loads are warp-collective: reconverge after the wait and the
-          // per-lane stores of the previous step
+        uint32_t y0[16], y2[16], y1r[16], y1i[16];
+        const uint32_t col = tl + g * 16;
+        // the TMEM loads are warp-collective: reconverge after the wait and the
+        // per-lane stores of the previous group
+        __syncwarp();
+        tmem_ld16(col, y0);
+        tmem_ld16(col + p.BD, y2);
+        tmem_ld16(col + 2 * p.BD, y1r);
+        tmem_ld16(col + 3 * p.BD, y1i);
+        tmem_ld_wait();
+        if (g == groups - 1) {
+          tc_fence_before();
           __syncwarp();
-          tmem_ld8(col, y0);
-          tmem_ld8(col + p.BD, y2);
-          tmem_ld8(col + 2 * p.BD, y1r);
-          tmem_ld8(col + 3 * p.BD, y1i);
-          tmem_ld_wait();
-          if (h == 1 && g == groups - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
-          }
-          uint32_t packed[16];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
+          if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
+        }
+        uint32_t packed[32];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-            const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
-            packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-            packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
-          }
-          // C is even, so channels go out in 16-byte pairs
-          const int c0 = g * 16 + h * 8;
-          if (row_ok) {
+        for (int i = 0; i < 16; ++i) {
+          const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+          const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
+          const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
+          packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+          packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+        }
+        // C is even, so channels go out in 16-byte pairs
+        const int c0 = g * 16;
+        if (row_ok) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (c0 + 2 * j + 2 <= p.C)
-                *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
-                    packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
+          for (int j = 0; j < 8; ++j)
+            if (c0 + 2 * j + 2 <= p.C)
+              *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
+                  packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         }
       }
     }

@@ -82,23 +82,40 @@ __host__ __device__ inline TcSmem tc_fwd_smem(const TcFwdParams &p) {
   return s;
 }
 
-// k-th work unit of this CTA: token tile m and output-channel tile j.  With
-// resident weights every CTA keeps one j (neighbouring CTAs share a token tile,
-// so its second read comes from L2); otherwise units are dealt round-robin.
-__device__ __forceinline__ bool tc_unit(const TcFwdParams &p, int k, int &m, int &j) {
-  if (p.resident) {
-    const int g = gridDim.x / p.nD;
-    if (static_cast<int>(blockIdx.x) >= g * p.nD) return false;
-    j = blockIdx.x % p.nD;
-    m = blockIdx.x / p.nD + k * g;
-    return m < p.nM;
+// The work units of this CTA in order: token tile m and output-channel tile j.
+// With resident weights every CTA keeps one j (neighbouring CTAs share a token
+// tile, so its second read comes from L2); otherwise units are dealt
+// round-robin.  The divisions happen once: the issuing threads share their SM
+// sub-partition with busy warps, so a per-unit division chain (several hundred
+// cycles there) would stall the tensor pipe.
+struct TcUnits {
+  int m, j;
+  int dm, dj, nD, nM;
+  bool valid;
+  __device__ __forceinline__ explicit TcUnits(const TcFwdParams &p) : nD(p.nD), nM(p.nM) {
+    m = static_cast<int>(blockIdx.x) / p.nD;
+    j = static_cast<int>(blockIdx.x) % p.nD;
+    if (p.resident) {
+      const int g = static_cast<int>(gridDim.x) / p.nD;
+      dm = g;
+      dj = 0;
+      valid = static_cast<int>(blockIdx.x) < g * p.nD && m < nM;
+    } else {
+      dm = static_cast<int>(gridDim.x) / p.nD;
+      dj = static_cast<int>(gridDim.x) % p.nD;
+      valid = m < nM;
+    }
   }
-  const int u = blockIdx.x + k * gridDim.x;
-  if (u >= p.n_units) return false;
-  m = u / p.nD;
-  j = u % p.nD;
-  return true;
-}
+  __device__ __forceinline__ void next() {
+    m += dm;
+    j += dj;
+    if (j >= nD) {
+      j -= nD;
+      ++m;
+    }
+    valid = m < nM;
+  }
+};
 
 // 18 warps over the 4 SM sub-partitions put 5 warps on one 16K-register
 // slice: 5 x 32 x 96 = 15,360 registers fits, 104 would not.
@@ -153,15 +170,16 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
       tma_prefetch_desc(&tm_out);
-      int m, j;
-      if (p.resident && tc_unit(p, 0, m, j)) {
+      TcUnits U(p);
+      if (p.resident && U.valid) {
         mbar_arrive_expect_tx(wfull, p.nK * p.chunk_bytes);
-        bulk_load(smem + L.wres, p.wt + static_cast<int64_t>(j) * p.nK * p.chunk_bytes,
+        bulk_load(smem + L.wres, p.wt + static_cast<int64_t>(U.j) * p.nK * p.chunk_bytes,
                   p.nK * p.chunk_bytes, wfull);
       }
       int s = 0;
       uint32_t ph = 0;
-      for (int k = 0; tc_unit(p, k, m, j); ++k) {
+      for (; U.valid; U.next()) {
+        const int m = U.m, j = U.j;
         for (int kc = 0; kc < p.nK; ++kc) {
           if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
           if (ok) {
@@ -189,8 +207,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       const uint32_t wrow = 32;  // bytes per weight row (16 fp16)
       const uint64_t dsw32 = smem_desc(0, 16, 256, kSw32);  // K-major, 32-byte swizzle
       const uint32_t stage_base = smem_u32(smem + L.stage0), wres_base = smem_u32(smem + L.wres);
-      int m, j;
-      if (p.resident && tc_unit(p, 0, m, j)) ok = mbar_wait(wfull, 0);
+      TcUnits U(p);
+      if (p.resident && U.valid) ok = mbar_wait(wfull, 0);
       int s = 0;
       uint32_t ph = 0;
       // every operand is the low descriptor word of a chunk's base plus a 16-byte-unit
@@ -202,7 +220,7 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       const uint32_t wr0 = desc_lo(desc_at(dsw32, wres_base));
       int a = 0;        // accumulator buffer of this unit
       uint32_t aph = 0;  // its phase
-      for (int it = 0; tc_unit(p, it, m, j); ++it) {
+      for (; U.valid; U.next()) {
         if (ok) ok = mbar_wait(&acc_empty[a], aph ^ 1);
         tc_fence_after();
         const uint32_t acc = tmem_base + a * p.acc_stride;
@@ -238,8 +256,7 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     const int r = (threadIdx.x - 64) % 128;  // row of the chunk (token within the tile)
     int s = 0, c = 0;
     uint32_t ph = 0;
-    int m, j;
-    for (int k = 0; tc_unit(p, k, m, j); ++k) {
+    for (TcUnits U(p); U.valid; U.next()) {
       for (int kc = 0; kc < p.nK; ++kc, ++c) {
         if (c % kTeams != team) {
           if (++s == p.stages) { s = 0; ph ^= 1; }
@@ -286,11 +303,13 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     const int g0 = split ? eteam : 0, gstep = split ? kTeams : 1;
     int last_g = -1;
     for (int g = g0; g < groups; g += gstep) last_g = g;
-    int oi = 0, m, j;
-    for (int it = 0; tc_unit(p, it, m, j); ++it) {
+    int oi = 0, it = 0;
+    for (TcUnits U(p); U.valid; U.next(), ++it) {
+      const int m = U.m, j = U.j;
       if (!split && it % kTeams != eteam) continue;
-      const int a = it % p.nacc;
-      const uint32_t aph = (it / p.nacc) & 1;
+      // accumulator buffer and phase of unit `it` (nacc is 1 or 2)
+      const int a = p.nacc == 2 ? (it & 1) : 0;
+      const uint32_t aph = (p.nacc == 2 ? it >> 1 : it) & 1;
       if (ok) ok = mbar_wait(&acc_full[a], aph);
       tc_fence_after();
       if (last_g < 0) {  // this team reads nothing of the tile
