@@ -7,16 +7,17 @@
 // contractions, bin 1 is one complex contraction; the Fourier tiles live only
 // in shared memory / tensor memory (no intermediate global writes).
 //
-// One persistent CTA per SM, warp-specialised (576 threads):
+// One persistent CTA per SM, warp-specialised (640 threads, warps 5 and 9 idle):
 //   warp 0       TMA producer: input chunks [128 tokens x 16 channels x 4] into
 //                a ring of `stages` slots; the weight chunks either ride along
 //                in each slot or, when the CTA's whole weight slice fits, are
 //                loaded once into a resident buffer
 //   warp 1       TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..9   transform, two 4-warp teams taking alternate chunks: 4-point
+//   warps 2-4, 6-8, 10, 11
+//                transform, two 4-warp teams taking alternate chunks: 4-point
 //                rDFT of the chunk (packed fp16 pairs), in place, into four
 //                K-major operand planes (X0, X2, Re X1, -Im X1)
-//   warps 10..17 epilogue, two 4-warp teams: tcgen05.ld of the four fp32
+//   warps 12..19 epilogue, two 4-warp teams: tcgen05.ld of the four fp32
 //                accumulators, inverse rDFT + bias, fp16 pack, swizzled smem
 //                staging; each warp owns 32 token rows and issues its own TMA
 //                stores
@@ -42,7 +43,18 @@
 namespace feql {
 
 constexpr int kTeams = 2;                         // transform teams and epilogue teams
-constexpr int kTcThreads = 64 + 2 * kTeams * 128; // TMA + MMA warps, 4-warp teams
+// Warp w runs on SM sub-partition w % 4.  Sub-partition 1 holds the MMA issuer
+// (warp 1), so warps 5 and 9 stay idle and the transform warps sit on the other
+// three sub-partitions: warps 2-4, 6-8, 10-11 transform, 12-19 epilogue.
+constexpr int kTcWarps = 20;
+constexpr int kTcThreads = kTcWarps * 32;
+constexpr int kTcEpi0 = 12;                       // first epilogue warp
+
+// Transform ordinal (0..4*kTeams-1) of warp w, or -1 when w is not a transform warp.
+__device__ __forceinline__ int tc_xf_ordinal(int w) {
+  if (w < 2 || w >= kTcEpi0 || w == 5 || w == 9) return -1;
+  return w - 2 - (w > 5) - (w > 9);
+}
 constexpr int kXChunkBytes = kBM * kCK * kT * 2;  // 16 KB: 128 rows x 128 B
 constexpr int kPlaneBytes = kBM * kCK * 2;        // 4 KB: 128 rows x 32 B
 constexpr int kOutRows = 32;                      // rows per epilogue TMA store (one warp)
@@ -117,7 +129,7 @@ struct TcUnits {
   }
 };
 
-// 18 warps over the 4 SM sub-partitions put 5 warps on one 16K-register
+// 20 warps over the 4 SM sub-partitions put 5 warps on each 16K-register
 // slice: 5 x 32 x 96 = 15,360 registers fits, 104 would not.
 __global__ void __maxnreg__(96)
 tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
@@ -249,11 +261,12 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
       mma_commit(final_bar);
       mbar_wait(final_bar, 0);
     }
-  } else if (warp < 2 + 4 * kTeams) {
+  } else if (tc_xf_ordinal(warp) >= 0) {
     // ---------------------------------------------------------- transform
     // kTeams teams of 4 warps take alternate chunks of the ring.
-    const int team = (warp - 2) / 4;
-    const int r = (threadIdx.x - 64) % 128;  // row of the chunk (token within the tile)
+    const int xo = tc_xf_ordinal(warp);
+    const int team = xo / 4;
+    const int r = (xo % 4) * 32 + lane;  // row of the chunk (token within the tile)
     int s = 0, c = 0;
     uint32_t ph = 0;
     for (TcUnits U(p); U.valid; U.next()) {
@@ -288,13 +301,13 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
     }
-  } else {
+  } else if (warp >= kTcEpi0) {
     // ----------------------------------------------------------- epilogue
     // kTeams teams of 4 warps.  With double-buffered accumulators each team
     // owns one TMEM buffer (alternate tiles); with a single buffer the teams
     // split each tile's 16-column groups.  Each warp owns one TMEM lane
     // quadrant (32 token rows) and stores its rows with its own TMA stores.
-    const int ew = warp - 2 - 4 * kTeams;   // epilogue warp index
+    const int ew = warp - kTcEpi0;           // epilogue warp index
     const int eteam = ew / 4;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
     uint8_t *obase = smem + L.out0 + ew * kNumOut * kOutBoxBytes;
