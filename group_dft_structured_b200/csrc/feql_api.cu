@@ -94,17 +94,18 @@ int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
   return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
 }
 
-// A [rows][boxes x 16 channels x 4] fp16 tensor seen as a stack of 16-channel
-// boxes: dims (64 elements, rows, boxes), strides (channels*8 B, 128 B).  One
-// load of a (64, box_rows, box_count) box writes box_count boxes of box_rows
-// 128-byte rows one after the other, the shared-memory image of box_count 2-D
-// loads.  Needs channels % 16 == 0 (else a box would run into the next row).
-int make_tmap_f16_boxes(CUtensorMap *m, const void *base, int64_t rows, int64_t channels,
+// A [rows][row_elems] fp16 tensor seen as a stack of 64-element (128-byte)
+// column boxes: dims (64 elements, rows, boxes), strides (row_elems*2 B, 128 B).
+// One load of a (64, box_rows, box_count) box writes box_count boxes of
+// box_rows 128-byte rows one after the other, the shared-memory image of
+// box_count 2-D loads.  Needs row_elems % 64 == 0 (else a box would run into
+// the next row).
+int make_tmap_f16_boxes(CUtensorMap *m, const void *base, int64_t rows, int64_t row_elems,
                         int box_rows, int box_count) {
   EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr || channels % 16 != 0) return FEQL_ERR_CUDA;
-  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(channels / 16)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(channels) * kT * 2, 128};
+  if (enc == nullptr || row_elems % 64 != 0) return FEQL_ERR_CUDA;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(row_elems / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_elems) * 2, 128};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_count)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides,
@@ -294,11 +295,13 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     // one load per operand and chunk when the channels form whole boxes, else
     // one 2-D load per 16-channel box
     CUtensorMap tm_dy, tm_x;
-    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, p.N, p.D, p.TB, p.nqd_max) == FEQL_OK;
+    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB,
+                                     p.nqd_max) == FEQL_OK;
     int st = FEQL_OK;
     if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB);
     if (st != FEQL_OK) return st;
-    p.stack_x = make_tmap_f16_boxes(&tm_x, x, p.N, p.C, p.TB, p.nqc_max) == FEQL_OK;
+    p.stack_x = make_tmap_f16_boxes(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB,
+                                    p.nqc_max) == FEQL_OK;
     if (!p.stack_x) st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB);
     if (st != FEQL_OK) return st;
     if (cudaFuncSetAttribute(tc_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -346,6 +349,8 @@ bool make_tc_bwd_plan(int64_t N, int C, int D, const WhatLayout &L, const Device
   p.dx = nullptr;
   p.ws = nullptr;
   p.ws_db = nullptr;
+  p.stack_dy = 0;
+  p.stack_x = 0;
   return true;
 }
 
@@ -357,10 +362,16 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
   p.ws = ws;
   p.ws_db = ws + static_cast<int64_t>(p.splits) * 4 * p.D * p.Cs;
   const int smem = tc_bwd_smem(p).total + 1024;
+  // one load per operand and stage when the channels form whole boxes
   CUtensorMap tm_dy, tm_x;
-  int st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, kBwTB);
+  int st = FEQL_OK;
+  p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, kBwTB,
+                                   p.nqd) == FEQL_OK;
+  if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, kBwTB);
   if (st != FEQL_OK) return st;
-  st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB);
+  p.stack_x = make_tmap_f16_boxes(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB,
+                                  p.nqc) == FEQL_OK;
+  if (!p.stack_x) st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB);
   if (st != FEQL_OK) return st;
   if (cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
@@ -435,6 +446,9 @@ G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms) {
   p.splits = N > 0 ? static_cast<int>(cdiv(N, p.split_len)) : 0;
   p.slot_boxes = kG8DwDySlots + 2 * (p.CT / 16);
   p.stages = 1;
+  p.stack_dy = 0;
+  p.stack_x = 0;
+  p.nqd_stack = 0;
   p.ws = nullptr;
   p.ws_db = nullptr;
   return p;
@@ -461,9 +475,17 @@ int launch_g8_dw(const void *x, const void *dy, __half *dW, __half *db, float *w
   if (g8_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
   if (p.splits > 0) {
     CUtensorMap tm_dy, tm_x;
-    st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB);
+    // one load per operand and chunk when the channels form whole 8-channel
+    // boxes (the dy stack spans the largest tile's boxes), else one per box
+    const int dt0 = D < 128 ? D : 128;
+    p.nqd_stack = 2 * static_cast<int>(cdiv(dt0, 16));
+    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB,
+                                     p.nqd_stack) == FEQL_OK;
+    if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB);
     if (st != FEQL_OK) return st;
-    st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB);
+    p.stack_x = make_tmap_f16_boxes(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB,
+                                    2 * (p.CT / 16)) == FEQL_OK;
+    if (!p.stack_x) st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB);
     if (st != FEQL_OK) return st;
     const int smem = g8_dw_smem(p).total + 1024;
     if (cudaFuncSetAttribute(tc_g8_dw_kernel<Gp>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

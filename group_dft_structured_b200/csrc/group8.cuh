@@ -677,6 +677,8 @@ struct G8DwParams {
   int64_t split_len;   // tokens per split, multiple of kG8DwTB
   int stages;
   int slot_boxes;      // kG8DwDySlots + 2 * CT / 16
+  int stack_dy, stack_x;  // 1: one 3-D load brings all of a chunk's dy (x) boxes
+  int nqd_stack;       // boxes in the dy stack (those of the largest d tile)
   float *ws;           // [splits][8][D][Cs]: G0, G4, Re G1, Im G1, Re G2, Im G2, Re G3, Im G3
   float *ws_db;        // [splits][D]
 };
@@ -758,11 +760,21 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
         if (ok) {
           uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kG8DwBox;
           const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * kG8DwTB);
-          mbar_arrive_expect_tx(&full[s], nbox * kG8DwBox);
-          for (int q = 0; q < nqd; ++q)
-            tma_load_2d(st + q * kG8DwBox, &tm_dy, (d0 + 8 * q) * kT8, row, &full[s]);
-          for (int q = 0; q < nqc; ++q)
-            tma_load_2d(st + xoff + q * kG8DwBox, &tm_x, (c0 + 8 * q) * kT8, row, &full[s]);
+          // a stack lands whole (boxes past the last channel read as zeros)
+          const int bd = p.stack_dy ? p.nqd_stack : nqd;
+          mbar_arrive_expect_tx(&full[s], (bd + nqc) * kG8DwBox);
+          if (p.stack_dy) {
+            tma_load_3d(st, &tm_dy, 0, row, d0 / 8, &full[s]);
+          } else {
+            for (int q = 0; q < nqd; ++q)
+              tma_load_2d(st + q * kG8DwBox, &tm_dy, (d0 + 8 * q) * kT8, row, &full[s]);
+          }
+          if (p.stack_x) {
+            tma_load_3d(st + xoff, &tm_x, 0, row, c0 / 8, &full[s]);
+          } else {
+            for (int q = 0; q < nqc; ++q)
+              tma_load_2d(st + xoff + q * kG8DwBox, &tm_x, (c0 + 8 * q) * kT8, row, &full[s]);
+          }
         }
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
@@ -782,7 +794,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
       int s = 0;
       uint32_t ph = 0;
       for (int ch = 0; ch < nch; ++ch) {
-        if (ok) ok = mbar_wait(&full[s], ph);
+        // tready implies full (the transform waited for the TMA bytes first)
         if (ok) ok = mbar_wait(&tready[s], ph);
         tc_fence_after();
         if (ok) {

@@ -64,6 +64,7 @@ struct TcBwdParams {
   int64_t split_len;   // tokens per CTA, multiple of 64
   int ndx;             // dX accumulator buffers (1 or 2)
   int merged;          // dW bin 1 as two N = 2*CT MMAs (6*CT TMEM columns), see tc_dw.cuh
+  int stack_dy, stack_x;  // 1: one 3-D load brings all of a stage's dy (x) boxes
   float *ws;           // [splits][4][D][Cs]
   float *ws_db;        // [splits][D]
 };
@@ -151,10 +152,18 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           uint8_t *st = smem + L.stage0 + s * p.slots * kBwBox;
           const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * kBwTB);
           mbar_arrive_expect_tx(&full[s], nbox * kBwBox);
-          for (int q = 0; q < p.nqd; ++q)
-            tma_load_2d(st + q * kBwBox, &tm_dy, q * 16 * kT, row, &full[s]);
-          for (int q = 0; q < p.nqc; ++q)
-            tma_load_2d(st + (p.nqd + q) * kBwBox, &tm_x, q * 16 * kT, row, &full[s]);
+          if (p.stack_dy) {
+            tma_load_3d(st, &tm_dy, 0, row, 0, &full[s]);
+          } else {
+            for (int q = 0; q < p.nqd; ++q)
+              tma_load_2d(st + q * kBwBox, &tm_dy, q * 16 * kT, row, &full[s]);
+          }
+          if (p.stack_x) {
+            tma_load_3d(st + p.nqd * kBwBox, &tm_x, 0, row, 0, &full[s]);
+          } else {
+            for (int q = 0; q < p.nqc; ++q)
+              tma_load_2d(st + (p.nqd + q) * kBwBox, &tm_x, q * 16 * kT, row, &full[s]);
+          }
         }
         if (++s == p.stages) { s = 0; ph ^= 1; }
       }
