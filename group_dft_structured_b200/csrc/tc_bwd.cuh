@@ -12,22 +12,30 @@
 // One CTA per token split (a multiple of 64 tokens); shapes with C <= 64 and
 // D <= 128 (one dW tile, one dX output tile).  Per stage of 64 tokens:
 //   warp 0      TMA: every 16-channel box of dy and x for the 64 tokens
-//   warps 2..9  4-point rDFT of every (token, channel) fibre, in place: each
-//               8 KB box becomes four 2 KB planes (V0, V2, Re V1, -Im V1),
-//               rows = tokens, 32-byte swizzle; db sums in registers
+//   warps 2..17 4-point rDFT of every (token, channel) fibre, in place, one
+//               fibre row per thread: each 8 KB box becomes four 2 KB planes
+//               (V0, V2, Re V1, -Im V1), rows = tokens, 32-byte swizzle; in a
+//               dy box the first 4 KB hold V0 and V2 interleaved in blocks of
+//               16 token rows (V0 of tokens 16j.., then V2 of the same
+//               tokens); db sums in registers
 //   warp 1      TMEM allocator + MMA issuer:
 //                 dW: per 16 tokens six M=128 (d) x N=CT (c) MMAs, both
 //                     operands MN-major (the planes read column-wise)
-//                 dX: per 16-channel d chunk four M=64 (tokens) MMAs against
-//                     the resident conj(What)^T tiles, K-major (the same planes
-//                     read row-wise) into a double-buffered accumulator
-//   warps 10..13 dX epilogue: the M=64 accumulator sits in TMEM lanes
-//               (m mod 16) + 32 * (m / 16), so warp q's lanes 0..15 hold
-//               tokens 16q..16q+15; inverse rDFT, fp16, direct 16-byte stores
+//                 dX: per 16-channel d chunk, against the resident
+//                     conj(What)^T tiles, K-major (the same planes read
+//                     row-wise), into a double-buffered accumulator: bins 0
+//                     and 2 as one M=128 MMA over the interleaved V0/V2 rows
+//                     with N = 2 BD (What0 | What2; the cross products in the
+//                     other halves are not read), bin 1 as two M=64 MMAs
+//   warps 18..21 dX epilogue: warp q's TMEM lane quadrant holds tokens
+//               16q..16q+15: in lanes 0..15 for bin 0 and for the M=64 bin-1
+//               accumulator (lanes (m mod 16) + 32 * (m / 16)), in lanes
+//               16..31 for bin 2 (moved down by a shuffle); inverse rDFT,
+//               fp16, direct 16-byte stores
 //               (each lane writes whole channels of its own token row), which
 //               leaves the shared memory to the stages (three fit for C = 24,
 //               D = 96)
-// After the last stage warps 2..9 write the dW partials and db to the
+// After the last stage warps 2..17 write the dW partials and db to the
 // workspace.  Every wait is bounded.
 #pragma once
 
@@ -43,10 +51,10 @@ namespace feql {
 constexpr int kBwTB = 64;                    // tokens per stage (dX MMA M)
 constexpr int kBwBox = kBwTB * 128;          // 8 KB: 64 tokens x 16 channels x 4 fp16
 constexpr int kBwPlane = kBwTB * 32;         // 2 KB: one bin of one box
-constexpr int kBwXfWarps = 8;
+constexpr int kBwXfWarps = 16;               // one (box, token) item per thread and stage
 constexpr int kBwEpWarps = 4;
 constexpr int kBwThreads = 64 + (kBwXfWarps + kBwEpWarps) * 32;
-constexpr int kBwMaxItems = 2 * kBwXfWarps * 32;  // (box, token) items a stage may hold
+constexpr int kBwMaxItems = kBwXfWarps * 32;  // (box, token) items a stage may hold
 
 struct TcBwdParams {
   const uint8_t *wt;   // conj(What)^T tiles of the dX direction (one output tile)
@@ -69,6 +77,14 @@ struct TcBwdParams {
   float *ws_db;        // [splits][D]
 };
 
+// Byte offset of token row r of plane pp (0..3) inside a transformed dy box:
+// V0 and V2 interleaved in 16-row blocks (a 128-row K-major operand for the
+// merged bins-0/2 dX MMA, one 512-byte block per 16-token dW step), then the
+// Re V1 and -Im V1 planes.
+__device__ __forceinline__ int bw_dy_row(int pp, int r) {
+  return pp < 2 ? ((r >> 4) << 10) + (pp << 9) + ((r & 15) << 5) : pp * kBwPlane + (r << 5);
+}
+
 struct BwSmem {
   int wres, stage0, bars, total;
 };
@@ -83,9 +99,10 @@ __host__ __device__ inline BwSmem tc_bwd_smem(const TcBwdParams &p) {
   return s;
 }
 
-// 14 warps over the 4 SM sub-partitions put 4 warps on one 16K-register slice:
-// 4 x 32 x 128 = 16,384.
-__global__ void __maxnreg__(128)
+// 22 warps over the 4 SM sub-partitions put 6 warps on one 16K-register slice:
+// 6 x 32 x 80 = 15,360 (88 would not fit).  The transform is latency-bound, so
+// it gets many warps with one item each rather than few with several.
+__global__ void __maxnreg__(80)
 tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
               const TcBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -175,7 +192,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const uint32_t id_w = instr_desc(128, p.CT, 0, 0, 1, 1);
       const uint32_t id_wneg = instr_desc(128, p.CT, 0, 0, 1, 1, 1);
       // dX: M = 64 tokens, K-major operands
-      const uint32_t id_x1 = instr_desc(64, p.BD, 0, 0);
+      const uint32_t id_x02 = instr_desc(128, 2 * p.BD, 0, 0);  // bins 0 and 2, interleaved rows
       const uint32_t id_x2 = instr_desc(64, 2 * p.BD, 0, 0);
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
@@ -207,10 +224,11 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         if (ok) {
 #pragma unroll
           for (int k = 0; k < kBwTB / 16; ++k) {
-            // dy planes: d chunks 8 KB apart; x planes: plane-major, c chunks 2 KB apart;
-            // 16 tokens = 512 B
-            const uint32_t A0 = mn + k * 32, A1 = A0 + (kBwPlane >> 4);
-            const uint32_t A2 = A0 + 2 * (kBwPlane >> 4), A3 = A0 + 3 * (kBwPlane >> 4);
+            // dy planes: d chunks 8 KB apart, V0/V2 blocks of 16 tokens interleaved
+            // (1 KB per step), Re/-Im V1 planes 2 KB each; x planes: plane-major,
+            // c chunks 2 KB apart; 16 tokens = 512 B
+            const uint32_t A0 = mn + k * 64, A1 = A0 + 32;
+            const uint32_t A2 = mn + 2 * (kBwPlane >> 4) + k * 32, A3 = A2 + (kBwPlane >> 4);
             const uint32_t B0 = mx + k * 32, B1 = B0 + xb16;
             const uint32_t B2 = B1 + xb16, B3 = B2 + xb16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
@@ -232,8 +250,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           uint32_t ab = kl, wb = wl;  // running box and weight-chunk descriptor words
           for (int q = 0; q < p.nqd; ++q, ab += kBwBox >> 4, wb += chunk16) {
             const uint32_t in = q > 0 ? 1u : 0u;
-            mma_f16_lo(acc, ab, wb, dhi, id_x1, in);
-            mma_f16_lo(acc + p.BD, ab + (kBwPlane >> 4), wb + w1, dhi, id_x1, in);
+            mma_f16_lo(acc, ab, wb, dhi, id_x02, in);
             mma_f16_lo(acc + 2 * p.BD, ab + 2 * (kBwPlane >> 4), wb + 2 * w1, dhi, id_x2, in);
             mma_f16_lo(acc + 2 * p.BD, ab + 3 * (kBwPlane >> 4), wb + 3 * w1, dhi, id_x2, 1u);
           }
@@ -248,7 +265,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
   } else if (warp < 2 + kBwXfWarps) {
     // ---------------------------------------------------------- transform
     const int t = threadIdx.x - 64;
-    constexpr int kPer = kBwMaxItems / (kBwXfWarps * 32);  // items per thread (2)
+    constexpr int kPer = kBwMaxItems / (kBwXfWarps * 32);  // items per thread (1)
     float db_acc[kPer][16];
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
@@ -279,13 +296,18 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         const int e = t + k * kBwXfWarps * 32;
         const int b = e / kBwTB, r = e % kBwTB;
         if (b < nbox) {
-          // dy box: its four planes in place; x box q: plane pp at x + (pp * nqc + q) planes
-          uint8_t *base = b < p.nqd ? st + b * kBwBox
-                                    : st + p.nqd * kBwBox + (b - p.nqd) * kBwPlane;
-          const int pstride = b < p.nqd ? kBwPlane : p.nqc * kBwPlane;
+          // dy box: its four planes in place (bw_dy_row); x box q: plane pp at
+          // x + (pp * nqc + q) planes
+          const bool is_dy = b < p.nqd;
+          uint8_t *base = is_dy ? st + b * kBwBox : st + p.nqd * kBwBox + (b - p.nqd) * kBwPlane;
+          // planes 0, 1 and 2, 3 are each one stride apart
+          const int o01 = is_dy ? bw_dy_row(0, r) : r * 32;
+          const int s01 = is_dy ? 512 : p.nqc * kBwPlane;
+          const int o23 = is_dy ? bw_dy_row(2, r) : 2 * p.nqc * kBwPlane + r * 32;
+          const int s23 = is_dy ? kBwPlane : p.nqc * kBwPlane;
 #pragma unroll
           for (int pp = 0; pp < 4; ++pp) {
-            uint8_t *row = base + pp * pstride + r * 32;
+            uint8_t *row = base + (pp < 2 ? o01 + pp * s01 : o23 + (pp - 2) * s23);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
               *reinterpret_cast<uint4 *>(row + (((hh ^ (r >> 2)) & 1) << 4)) =
@@ -311,12 +333,12 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     // ---------------------------------------------- dW partials -> workspace
     if (ok) ok = mbar_wait(dwfull, 0);
     tc_fence_after();
-    const int quad = warp & 3, half = (warp - 2) / 4;
+    const int quad = warp & 3, part = (warp - 2) / 4;  // kBwXfWarps / 4 warps per quadrant
     const int d = quad * 32 + lane;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     float *dst = p.ws + (static_cast<int64_t>(split) * 4 * p.D + d) * p.Cs;
     const int64_t bin_stride = static_cast<int64_t>(p.D) * p.Cs;
-    for (int g = half; g < p.CT / 8; g += 2) {  // 8-column steps
+    for (int g = part; g < p.CT / 8; g += kBwXfWarps / 4) {  // 8-column steps
       float G[4][8];
       dw_acc_read8(tl, p.CT, g * 8, p.merged, G);
       if (d < p.D && g * 8 < p.C) {
@@ -360,38 +382,44 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const bool row_ok = lane < 16 && n < t_end;
       __half *drow = p.dx + n * row_elems;
       for (int g = 0; g < groups; ++g) {
-        uint32_t y0[16], y2[16], y1r[16], y1i[16];
-        const uint32_t col = tl + g * 16;
-        // the TMEM loads are warp-collective: reconverge after the wait and the
-        // per-lane stores of the previous group
-        __syncwarp();
-        tmem_ld16(col, y0);
-        tmem_ld16(col + p.BD, y2);
-        tmem_ld16(col + 2 * p.BD, y1r);
-        tmem_ld16(col + 3 * p.BD, y1i);
-        tmem_ld_wait();
-        if (g == groups - 1) {
-          tc_fence_before();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // 8 columns at a time keeps registers low
+          uint32_t y0[8], y2[8], y1r[8], y1i[8];
+          const uint32_t col = tl + g * 16 + h * 8;
+          // the TMEM loads are warp-collective: reconverge after the wait and the
+          // per-lane stores of the previous step
           __syncwarp();
-          if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
-        }
-        uint32_t packed[32];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
+          tmem_ld8(col, y0);
+          tmem_ld8(col + p.BD, y2);
+          tmem_ld8(col + 2 * p.BD, y1r);
+          tmem_ld8(col + 3 * p.BD, y1i);
+          tmem_ld_wait();
+          if (h == 1 && g == groups - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
+          }
+          // bin 2 of token 16q + l sits in lane l + 16 (the V2 rows of the merged MMA)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-          const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-          const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
-          packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-          packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
-        }
-        // C is even, so channels go out in 16-byte pairs
-        const int c0 = g * 16;
-        if (row_ok) {
+          for (int i = 0; i < 8; ++i) y2[i] = __shfl_down_sync(0xffffffffu, y2[i], 16);
+          uint32_t packed[16];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (c0 + 2 * j + 2 <= p.C)
-              *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
-                  packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          for (int i = 0; i < 8; ++i) {
+            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
+            const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
+            packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
+            packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+          }
+          // C is even, so channels go out in 16-byte pairs
+          const int c0 = g * 16 + h * 8;
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              if (c0 + 2 * j + 2 <= p.C)
+                *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
+                    packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
         }
       }
     }
