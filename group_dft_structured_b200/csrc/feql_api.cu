@@ -292,16 +292,19 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     while (p.stages > 2 && tc_dw_smem(p).total > budget) --p.stages;
     if (tc_dw_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
     const int smem = tc_dw_smem(p).total + 1024;
-    // one load per operand and chunk when the channels form whole boxes, else
-    // one 2-D load per 16-channel box
+    // Chunks of 16 tokens make 2 KB boxes, and issuing one TMA load per box
+    // then limits the kernel: such chunks take one load per operand when the
+    // channels form whole boxes.  Larger chunks keep one 2-D load per box
+    // (measured faster there).
     CUtensorMap tm_dy, tm_x;
-    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB,
-                                     p.nqd_max) == FEQL_OK;
+    const bool small = p.TB <= 16;
+    p.stack_dy = small && make_tmap_f16_boxes(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT,
+                                              p.TB, p.nqd_max) == FEQL_OK;
     int st = FEQL_OK;
     if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, p.N, static_cast<int64_t>(p.D) * kT, p.TB);
     if (st != FEQL_OK) return st;
-    p.stack_x = make_tmap_f16_boxes(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB,
-                                    p.nqc_max) == FEQL_OK;
+    p.stack_x = small && make_tmap_f16_boxes(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB,
+                                             p.nqc_max) == FEQL_OK;
     if (!p.stack_x) st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, p.TB);
     if (st != FEQL_OK) return st;
     if (cudaFuncSetAttribute(tc_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -310,10 +313,9 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     const int grid = p.tiles_d * p.tiles_c * p.splits;
     tc_dw_kernel<<<grid, kDwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  const RedPlan rp = make_red_plan(p.C, p.D, dev.sms);
-  if (rp.blocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-  dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
-      p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs, rp.q, rp.wblocks);
+  if (launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs,
+                          dev.sms, stream) != 0)
+    return FEQL_ERR_UNSUPPORTED;
   return launch_status();
 }
 
@@ -377,10 +379,8 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
       cudaSuccess)
     return FEQL_ERR_CUDA;
   tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, p);
-  const RedPlan rp = make_red_plan(p.C, p.D, dev.sms);
-  if (rp.blocks > INT32_MAX) return FEQL_ERR_UNSUPPORTED;
-  dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
-      p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs, rp.q, rp.wblocks);
+  if (launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs, dev.sms, stream) != 0)
+    return FEQL_ERR_UNSUPPORTED;
   return launch_status();
 }
 

@@ -353,6 +353,67 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
   }
 }
 
+// Small outputs (a few thousand (d, c) pairs, where the vector kernel below
+// has too few blocks): a block takes 32 consecutive (d, c) outputs (the last
+// blocks take db); its 16 warps each sum every 16th split, then warp 0 adds the
+// 16 partial sums in warp order — the same grouping on every run.
+constexpr int kRedOut = 32, kRedGroups = 16;
+constexpr int64_t kRedScalarMaxOut = 8192;  // D * C up to which the scalar kernel runs
+
+__global__ void __launch_bounds__(kRedOut * kRedGroups)
+dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
+                    __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
+                    int Cs) {
+  __shared__ float part[kRedGroups][4][kRedOut];
+  const int64_t plane = static_cast<int64_t>(D) * Cs;
+  const int64_t n = static_cast<int64_t>(D) * C;
+  const int64_t nblk_w = cdiv(n, kRedOut);
+  const int lo = threadIdx.x % kRedOut, grp = threadIdx.x / kRedOut;
+  if (blockIdx.x < nblk_w) {
+    const int64_t e = blockIdx.x * static_cast<int64_t>(kRedOut) + lo;
+    float g[4] = {0.f, 0.f, 0.f, 0.f};
+    if (e < n) {
+      const float *src = ws + (e / C) * Cs + (e % C);
+      for (int s = grp; s < splits; s += kRedGroups) {
+        const float *q = src + static_cast<int64_t>(s) * 4 * plane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) g[k] += q[k * plane];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) part[grp][k][lo] = g[k];
+    __syncthreads();
+    if (grp == 0 && e < n) {
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < kRedGroups; ++q)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) t[k] += part[q][k][lo];
+      const float ev = 0.25f * (t[0] + t[1]), od = 0.25f * (t[0] - t[1]);
+      uint2 pk;
+      pk.x = pack_half2(ev + 0.5f * t[2], od - 0.5f * t[3]);
+      pk.y = pack_half2(ev - 0.5f * t[2], od + 0.5f * t[3]);
+      *reinterpret_cast<uint2 *>(dW + e * kT) = pk;
+    }
+  } else if (db != nullptr) {
+    const int64_t d = (blockIdx.x - nblk_w) * kRedOut + lo;
+    float sdb = 0.f;
+    if (d < D)
+      for (int s = grp; s < splits; s += kRedGroups) sdb += ws_db[static_cast<int64_t>(s) * D + d];
+    part[grp][0][lo] = sdb;
+    __syncthreads();
+    if (grp == 0 && d < D) {
+      float t = 0.f;
+      for (int q = 0; q < kRedGroups; ++q) t += part[q][0][lo];
+      db[d] = __float2half_rn(t);
+    }
+  }
+}
+
+// Blocks for dw_tc_reduce_scalar_kernel: the dW outputs, then the db outputs.
+__host__ __device__ inline int64_t dw_reduce_scalar_blocks(int C, int D) {
+  return cdiv(static_cast<int64_t>(D) * C, kRedOut) + cdiv(D, kRedOut);
+}
+
 // Sum of the split partials in a fixed order, inverse rDFT, fp16 cast:
 //   dW[d][c][u] = (G0 + (-1)^u G2)/4 + Re(G1 i^u)/2,   db[d] = sum of partials.
 // A dW block owns `q` quads (one d, four consecutive c, all four bins: 16
@@ -450,6 +511,23 @@ dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
     __syncthreads();
     if (grp == 0 && d < D) db[d] = __float2half_rn(red[0][t]);
   }
+}
+
+// Launches the split reduce that suits the output size (both sum the splits in
+// a fixed order).
+inline int launch_dw_tc_reduce(const float *ws, const float *ws_db, __half *dW, __half *db,
+                               int splits, int C, int D, int Cs, int sms, cudaStream_t stream) {
+  if (static_cast<int64_t>(D) * C <= kRedScalarMaxOut) {
+    dw_tc_reduce_scalar_kernel<<<static_cast<unsigned>(dw_reduce_scalar_blocks(C, D)),
+                                 kRedOut * kRedGroups, 0, stream>>>(ws, ws_db, dW, db, splits, C,
+                                                                    D, Cs);
+  } else {
+    const RedPlan rp = make_red_plan(C, D, sms);
+    if (rp.blocks > 0x7fffffff) return 1;
+    dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
+        ws, ws_db, dW, db, splits, C, D, Cs, rp.q, rp.wblocks);
+  }
+  return 0;
 }
 
 }  // namespace feql
