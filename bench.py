@@ -121,17 +121,27 @@ def layer_macs(w):
     return fourier * w.N * w.C * w.D, w.T * w.T * w.N * w.C * w.D
 
 
+def strip_comments(src: str) -> str:
+    """C/CUDA source without // and /* */ comments, trailing blanks and empty lines
+    (the sources contain no string literal with a comment marker)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash():
-    """Hash of the CUDA sources; DRAM counters in profiles/traffic.json are only
-    reported while it matches the hash they were taken with."""
+    """Hash of the CUDA sources' code (comments excluded); DRAM counters in
+    profiles/traffic.json are only reported while it matches the hash they were
+    taken with."""
     import hashlib
     d = os.path.join(ROOT, "group_dft_structured_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
         if f.endswith((".cu", ".cuh")):
             h.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(d, f), encoding="utf-8") as fh:
+                h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,7 +7,7 @@
 //   dX[n,:] = irDFT_4( per-bin dY_k[n,:] . conj(What_k) )          (forward of conj(What)^T)
 //   G_k[d,c] += sum_{n in split} dY_k[n,d] conj(X_k[n,c])          (split-K partials of dW)
 //   db[d]    += sum_{n in split} dY_0[n,d]
-// and dw_tc_reduce_kernel finishes dW/db as for feql_backward_dw.
+// and the split reduce of tc_dw.cuh finishes dW/db as for feql_backward_dw.
 //
 // One CTA per token split (a multiple of 64 tokens); shapes with C <= 64 and
 // D <= 128 (one dW tile, one dX output tile).  Per stage of 64 tokens:

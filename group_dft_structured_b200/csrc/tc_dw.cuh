@@ -21,8 +21,11 @@
 //   warp 1      TMEM allocator + MMA issuer: per 16 tokens six M=128 x N=CT
 //               MMAs, one of them through the B-negate bit
 // After the last chunk warps 2..9 read the four fp32 accumulators out of
-// TMEM and write them to the workspace; dw_tc_reduce_kernel sums the splits
-// in a fixed order (bit-identical run to run) and applies the inverse rDFT.
+// TMEM and write them to the workspace; the split reduce (below: a scalar
+// kernel for small outputs, a vectorised one for large) sums the splits in a
+// fixed order (bit-identical run to run) and applies the inverse rDFT.
+// TMA: one 2-D load per 16-channel box, or with 16-token chunks one 3-D
+// "box stack" load per operand (see make_tmap_f16_boxes).
 #pragma once
 
 #include <cuda_fp16.h>
