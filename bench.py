@@ -7,7 +7,11 @@ and weight gradient (feql_backward_dw), all through the C ABI, fp16 data with
 fp32 accumulation, on the Swin stage-1-like forward+backward workload
 N = 128 x 3136 tokens, C = 24, D = 96 (96 -> 384 unrolled).  Inputs are
 resident in HBM; each pass reads/writes ~385 MB, more than the 126 MB L2, so
-no flush is needed between steps.
+no flush is needed between steps.  The same line carries "per_config": every
+layer configuration (1: fp32 256x16x16, 2: ViT fc1 12608x48x192, 3: square
+65536x192x192 in fp16 and fp32, 4: backward 32768x256x256, 5: the Swin stream)
+at full size, each pass timed over 50 reps with the L2 flushed before each,
+median and min, with its roofline fractions.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -59,6 +63,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--separate-backward", action="store_true",
                     help="run dX and dW as two passes instead of the fused backward")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-configuration table (configurations 1-5, L2 flushed)")
+    ap.add_argument("--config-reps", type=int, default=50,
+                    help="timed reps per pass in the per-configuration table")
     return ap.parse_args()
 
 
@@ -283,44 +291,61 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------- ours
 def setup_layer(args, w, rank, s, F, torch):
-    """Buffers and calls of the EQ-Linear layer workloads (p4 and C_8)."""
+    """Buffers and calls of the EQ-Linear layer workloads (p4, C_8, p4m)."""
     from group_dft_structured_b200.workloads import make_inputs
     mode = F.FEQL_FP16 if w.dtype == "fp16" else F.FEQL_FP32
     N, C, D, T = w.N, w.C, w.D, w.T
     elt = 2 if w.dtype == "fp16" else 4
     inp = make_inputs(rank_seed_id(w.wid, rank), N, C, D, w.dtype, T=T)
-    dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
-    x, W, b, dy = dev["x"], dev["W"], dev["b"], dev["dy"]
     p4m = w.group == "p4m"
     wbytes = (F.feql_p4m_weight_fft_bytes(C, D, mode) if p4m
               else F.feql_ct_weight_fft_bytes(T, C, D, mode))
-    What = torch.empty(wbytes, dtype=torch.uint8, device="cuda")
-    y = torch.empty((N, D, T), dtype=x.dtype, device="cuda")
-    dx = torch.empty((N, C, T), dtype=x.dtype, device="cuda")
-    dW = torch.empty((D, C, T), dtype=x.dtype, device="cuda")
-    db = torch.empty((D,), dtype=x.dtype, device="cuda")
     wsb = (F.feql_p4m_backward_dw_workspace_bytes(N, C, D, mode) if p4m
            else F.feql_ct_backward_dw_workspace_bytes(T, N, C, D, mode))
-    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
-    # One step = every row of the path: weight rDFT, forward, and the backward
-    # (dX and dW/db, fused into one pass over dy for p4 unless --separate-backward).
-    if p4m:
-        calls = {
-            "wfft": lambda: F.feql_p4m_weight_fft(W, What, C, D, mode, s),
-            "fwd": lambda: F.feql_p4m_forward(x, What, b, y, N, C, D, mode, s),
-            "dx": lambda: F.feql_p4m_backward_dx(dy, What, dx, N, C, D, mode, s),
-            "dw": lambda: F.feql_p4m_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
-        }
-    else:
-        calls = {
-            "wfft": lambda: F.feql_ct_weight_fft(T, W, What, C, D, mode, s),
-            "fwd": lambda: F.feql_ct_forward(T, x, What, b, y, N, C, D, mode, s),
-            "dx": lambda: F.feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, s),
+
+    def buffers(first=None):
+        """One set of device buffers: inputs (copied from the host arrays for the
+        first set, left uninitialised for the e2e run's second set), outputs,
+        the Fourier weights and the dW workspace."""
+        if first is None:
+            B = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+        else:
+            B = {k: torch.empty_like(first[k]) for k in inp}
+        dt = B["x"].dtype
+        B["What"] = torch.empty(wbytes, dtype=torch.uint8, device="cuda")
+        B["y"] = torch.empty((N, D, T), dtype=dt, device="cuda")
+        B["dx"] = torch.empty((N, C, T), dtype=dt, device="cuda")
+        B["dW"] = torch.empty((D, C, T), dtype=dt, device="cuda")
+        B["db"] = torch.empty((D,), dtype=dt, device="cuda")
+        B["ws"] = torch.empty(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        return B
+
+    def calls_for(B, st):
+        """The passes of one step on buffer set B, enqueued on stream handle st.
+        One step = every row of the path: weight rDFT, forward, and the backward
+        (dX and dW/db, fused into one pass over dy for p4 unless
+        --separate-backward)."""
+        x, W, b, dy, What, ws = B["x"], B["W"], B["b"], B["dy"], B["What"], B["ws"]
+        y, dx, dW, db = B["y"], B["dx"], B["dW"], B["db"]
+        if p4m:
+            return {
+                "wfft": lambda: F.feql_p4m_weight_fft(W, What, C, D, mode, st),
+                "fwd": lambda: F.feql_p4m_forward(x, What, b, y, N, C, D, mode, st),
+                "dx": lambda: F.feql_p4m_backward_dx(dy, What, dx, N, C, D, mode, st),
+                "dw": lambda: F.feql_p4m_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D,
+                                                     mode, st),
+            }
+        return {
+            "wfft": lambda: F.feql_ct_weight_fft(T, W, What, C, D, mode, st),
+            "fwd": lambda: F.feql_ct_forward(T, x, What, b, y, N, C, D, mode, st),
+            "dx": lambda: F.feql_ct_backward_dx(T, dy, What, dx, N, C, D, mode, st),
             "dw": lambda: F.feql_ct_backward_dw(T, x, dy, dW, db, ws, ws.numel(), N, C, D, mode,
-                                                s),
-            "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D, mode,
-                                           s),
+                                                st),
+            "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D,
+                                           mode, st),
         }
+
+    B0 = buffers()
     passes = ["wfft"] + (["fwd"] if "fwd" in w.passes else [])
     if "dx" in w.passes and "dw" in w.passes and not args.separate_backward and T == 4 and not p4m:
         passes.append("bwd")
@@ -330,19 +355,18 @@ def setup_layer(args, w, rank, s, F, torch):
     gemms = {"wfft": 0, "fwd": 1, "dx": 1, "dw": 1, "bwd": 2}  # layer contractions per pass
     has_bwd = any(p in passes for p in ("dx", "dw", "bwd"))
     ins = ["x", "W", "b"] + (["dy"] if has_bwd else [])
-    src = {"y": y, "dx": dx, "dW": dW, "db": db}
     outs = [k for k in ("y", "dx", "dW", "db")
             if (k == "y" and "fwd" in passes)
             or (k == "dx" and ("dx" in passes or "bwd" in passes))
             or (k in ("dW", "db") and ("dw" in passes or "bwd" in passes))]
     return {
-        "calls": calls, "passes": passes, "tokens": N, "elt": elt,
+        "calls": calls_for(B0, s), "calls_for": calls_for, "buffers": buffers, "B0": B0,
+        "passes": passes, "tokens": N, "elt": elt,
         "launches": {"wfft": 1, "fwd": 1, "dx": 1, "dw": 2, "bwd": 2},
         "bytes": workload_bytes(w, elt),
         "flops": {p: (2 * macs * gemms[p], 2 * dense_macs * gemms[p]) for p in passes},
-        "host": {k: inp[k] for k in ins}, "dev": {k: dev[k] for k in ins},
-        "outs": {k: src[k] for k in outs},
-        "allreduce": (lambda: dp_allreduce_grads(dW, db)) if has_bwd else None,
+        "host": {k: inp[k] for k in ins}, "ins": ins, "outs": outs,
+        "allreduce": (lambda B: dp_allreduce_grads(B["dW"], B["db"])) if has_bwd else None,
         "config": {"N": N, "C": C, "D": D, "T": T, "group": "p4m (D4)" if p4m else f"C_{T}"},
         "extra": {},
     }
@@ -356,15 +380,27 @@ def setup_mlp(args, w, rank, s, F, torch):
     mode = F.FEQL_FP16
     N, C, H, Co = w.N, w.C, w.D, w.C
     inp = make_mlp_inputs(rank_seed_id(w.wid, rank), N, C, H, Co, w.dtype)
-    dev = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
-    x, W1, b1, W2, b2 = (dev[k] for k in ("x", "W1", "b1", "W2", "b2"))
-    What = torch.empty(F.feql_mlp_weight_fft_bytes(C, H, Co, mode), dtype=torch.uint8,
-                       device="cuda")
-    y = torch.empty((N, Co, 4), dtype=x.dtype, device="cuda")
-    calls = {
-        "wfft": lambda: F.feql_mlp_weight_fft(W1, W2, What, C, H, Co, mode, s),
-        "mlp": lambda: F.feql_mlp_forward(x, What, b1, b2, y, N, C, H, Co, mode, s),
-    }
+    wbytes = F.feql_mlp_weight_fft_bytes(C, H, Co, mode)
+
+    def buffers(first=None):
+        if first is None:
+            B = {k: torch.from_numpy(v).cuda() for k, v in inp.items()}
+        else:
+            B = {k: torch.empty_like(first[k]) for k in inp}
+        B["What"] = torch.empty(wbytes, dtype=torch.uint8, device="cuda")
+        B["y"] = torch.empty((N, Co, 4), dtype=B["x"].dtype, device="cuda")
+        return B
+
+    def calls_for(B, st):
+        return {
+            "wfft": lambda: F.feql_mlp_weight_fft(B["W1"], B["W2"], B["What"], C, H, Co, mode,
+                                                  st),
+            "mlp": lambda: F.feql_mlp_forward(B["x"], B["What"], B["b1"], B["b2"], B["y"], N, C,
+                                              H, Co, mode, st),
+        }
+
+    B0 = buffers()
+    x, W1, b1, W2, b2, y = (B0[k] for k in ("x", "W1", "b1", "W2", "b2", "y"))
     macs = 6 * N * H * (C + Co)
     # context: the same block as three launches with the hidden activation in HBM
     W1hat = torch.empty(F.feql_weight_fft_bytes(C, H, mode), dtype=torch.uint8, device="cuda")
@@ -391,18 +427,145 @@ def setup_mlp(args, w, rank, s, F, torch):
         torch.cuda.synchronize()
         return a.elapsed_time(z) / reps
 
+    ins = ["x", "W1", "b1", "W2", "b2"]
     return {
-        "calls": calls, "passes": ["wfft", "mlp"], "tokens": N, "elt": 2,
+        "calls": calls_for(B0, s), "calls_for": calls_for, "buffers": buffers, "B0": B0,
+        "passes": ["wfft", "mlp"], "tokens": N, "elt": 2,
         "launches": {"wfft": 1, "mlp": 1},
         "bytes": mlp_bytes(w, 2),
         "flops": {"wfft": (0, 0), "mlp": (2 * macs, 2 * 16 * N * H * (C + Co))},
-        "host": {k: inp[k] for k in ("x", "W1", "b1", "W2", "b2")},
-        "dev": {k: dev[k] for k in ("x", "W1", "b1", "W2", "b2")},
-        "outs": {"y": y},
+        "host": {k: inp[k] for k in ins}, "ins": ins, "outs": ["y"],
         "allreduce": None,
         "config": {"N": N, "C": C, "H": H, "Co": Co, "T": 4, "gelu": "tanh form, fp16"},
         "extra": {"unfused": unfused},
     }
+
+
+# ------------------------------------------------------------- per config
+# Peaks for the per-config rooflines.  Nominal B200 figures (dense): HBM3e
+# 8.0 TB/s, fp16 tensor 2.25 PFLOP/s, fp32 FMA on CUDA cores 148 SMs x 128 lanes
+# x 2 FLOP x 1.965 GHz = 74.4 TFLOP/s.  The measured HBM and tensor figures come
+# from MEASURED_PEAKS.json (copy bandwidth; cuBLAS bf16, the same tensor rate as
+# fp16); the CUDA-core fp32 peak has no measurement and uses the nominal count.
+NOMINAL = {"hbm_gbs": 8000.0, "tensor_tflops": 2250.0, "fp32_fma_tflops": 74.4}
+
+# The five layer configurations, each with the passes its throughput is quoted
+# on (SURVEY of the method's workloads: forward for 1-3, dX and dW for 4,
+# forward and both gradients for 5; 3 also in fp32).
+CONFIG_RUNS = [(1, "fp32", ("fwd",)), (2, "fp16", ("fwd",)), (3, "fp16", ("fwd",)),
+               (3, "fp32", ("fwd",)), (4, "fp16", ("dx", "dw")),
+               (5, "fp16", ("fwd", "dx", "dw", "bwd"))]
+
+
+def peak_table():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    meas = None
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        meas = {"hbm_gbs": float(d["hbm_gbs"]), "tensor_tflops": float(d["bf16_tflops"]),
+                "fp32_fma_tflops": NOMINAL["fp32_fma_tflops"]}
+    return meas, NOMINAL
+
+
+def roofline_us(nbytes, flops, dtype, peaks):
+    """Roofline time (us) and its bound: the slower of the algorithmic bytes at
+    HBM bandwidth and the algorithmic FLOPs at the mode's arithmetic peak."""
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
+    fpeak = peaks["tensor_tflops"] if dtype == "fp16" else peaks["fp32_fma_tflops"]
+    t_cmp = flops / (fpeak * 1e12) * 1e6
+    return (t_mem, "hbm") if t_mem >= t_cmp else (t_cmp, "tensor" if dtype == "fp16" else "alu")
+
+
+def per_config_report(F, torch, stream, reps):
+    """Every layer configuration at full size: median and min over `reps` CUDA-event
+    timings of each pass, the L2 flushed before every rep by reading a buffer of
+    twice its size (that leaves the L2 holding clean lines of the flush buffer,
+    so neither the pass's inputs nor dirty lines of earlier writes remain)."""
+    import numpy as np
+
+    from group_dft_structured_b200 import layer as Lyr
+    from group_dft_structured_b200.workloads import WORKLOADS, workload_inputs
+    meas, nom = peak_table()
+    s = stream.cuda_stream
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    flush = torch.ones(2 * l2 // 4, dtype=torch.float32, device="cuda")
+    out = {}
+    for wid, dtype, passes in CONFIG_RUNS:
+        w = WORKLOADS[wid]
+        N, C, D = w.N, w.C, w.D
+        mode = F.FEQL_FP16 if dtype == "fp16" else F.FEQL_FP32
+        elt = 2 if dtype == "fp16" else 4
+        inp = workload_inputs(wid, dtype=dtype)
+        B = {k: torch.from_numpy(v).cuda() for k, v in inp.items()
+             if k in (("x", "W", "b") + (("dy",) if set(passes) - {"fwd"} else ()))}
+        What = torch.empty(F.feql_weight_fft_bytes(C, D, mode), dtype=torch.uint8, device="cuda")
+        dt = B["x"].dtype
+        y = torch.empty((N, D, 4), dtype=dt, device="cuda")
+        dx = torch.empty((N, C, 4), dtype=dt, device="cuda")
+        dW = torch.empty((D, C, 4), dtype=dt, device="cuda")
+        db = torch.empty((D,), dtype=dt, device="cuda")
+        ws = Lyr.dw_workspace(N, C, D, mode, "cuda")
+        x, W, b, dy = B["x"], B["W"], B["b"], B.get("dy")
+        calls = {
+            "wfft": lambda: F.feql_weight_fft(W, What, C, D, mode, s),
+            "fwd": lambda: F.feql_forward(x, What, b, y, N, C, D, mode, s),
+            "dx": lambda: F.feql_backward_dx(dy, What, dx, N, C, D, mode, s),
+            "dw": lambda: F.feql_backward_dw(x, dy, dW, db, ws, ws.numel(), N, C, D, mode, s),
+            "bwd": lambda: F.feql_backward(x, dy, What, dx, dW, db, ws, ws.numel(), N, C, D,
+                                           mode, s),
+        }
+        nbytes = workload_bytes(w, elt)
+        macs = 6 * N * C * D
+        flops = {"wfft": 0, "fwd": 2 * macs, "dx": 2 * macs, "dw": 2 * macs, "bwd": 4 * macs}
+        calls["wfft"]()
+        res = {}
+        for p in ("wfft",) + tuple(passes):
+            for _ in range(3):
+                calls[p]()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(reps)]
+            for a, z in ev:
+                flush.sum()
+                a.record(stream)
+                calls[p]()
+                z.record(stream)
+            torch.cuda.synchronize()
+            us = sorted(a.elapsed_time(z) * 1e3 for a, z in ev)
+            med, mn = float(np.median(us)), us[0]
+            r = {"median_us": round(med, 3), "min_us": round(mn, 3), "reps": reps,
+                 "algorithmic_bytes": nbytes[p],
+                 "GB_s": round(nbytes[p] / (med * 1e-6) / 1e9, 1)}
+            if flops[p]:
+                r["tokens_per_s"] = round(N / (med * 1e-6), 1)
+                r["alg_TFLOP_s"] = round(flops[p] / (med * 1e-6) / 1e12, 3)
+                r["dense_equiv_TFLOP_s"] = round(flops[p] * 16 / 6 / (med * 1e-6) / 1e12, 3)
+                for tag, pk in (("measured", meas), ("nominal", nom)):
+                    if pk is None:
+                        continue
+                    t_roof, bound = roofline_us(nbytes[p], flops[p], dtype, pk)
+                    r[f"roofline_us_{tag}"] = round(t_roof, 3)
+                    r[f"pct_roofline_{tag}"] = round(100 * t_roof / med, 2)
+                    r["bound"] = bound
+            res[p] = r
+        if F.feql_device_status(s) != F.FEQL_OK:
+            raise RuntimeError(f"device-side timeout in workload {wid}")
+        key = f"{wid}_{dtype}"
+        entry = {"workload": w.name, "N": N, "C": C, "D": D, "dtype": dtype,
+                 "l2": f"flushed before every rep (read of a {2 * l2 >> 20} MiB buffer)",
+                 "passes": res}
+        t = {p: res[p]["median_us"] for p in res}
+        if passes == ("fwd",):
+            entry["tokens_per_s"] = round(N / (t["fwd"] * 1e-6), 1)
+        elif passes == ("dx", "dw"):
+            entry["tokens_per_s"] = round(N / ((t["dx"] + t["dw"]) * 1e-6), 1)
+        else:
+            entry["tokens_per_s"] = round(N / ((t["fwd"] + t["dx"] + t["dw"]) * 1e-6), 1)
+            entry["tokens_per_s_fused_backward"] = round(N / ((t["fwd"] + t["bwd"]) * 1e-6), 1)
+        out[key] = entry
+        del B, x, W, b, dy, y, dx, dW, db, ws, What, calls
+        torch.cuda.empty_cache()
+    return out
 
 
 def main():
@@ -432,6 +595,7 @@ def main():
     s = stream.cuda_stream
     job = (setup_mlp if "mlp" in w.passes else setup_layer)(args, w, rank, s, F, torch)
     calls, passes, N = job["calls"], job["passes"], job["tokens"]
+    B0 = job["B0"]
 
     def step(ev=None):
         if ev is not None:
@@ -441,7 +605,7 @@ def main():
             if ev is not None:
                 ev[i + 1].record(stream)
         if world > 1 and job["allreduce"] is not None:
-            job["allreduce"]()
+            job["allreduce"](B0)
 
     def barrier():
         if world > 1:
@@ -477,26 +641,54 @@ def main():
         raise RuntimeError("device-side timeout during timing")
 
     # ---------------------------------------------------------- e2e (host buffers)
+    # Every step copies its inputs from pinned host memory and its results back.
+    # Two device buffer sets alternate between steps, and the copies run on their
+    # own streams, so that step k+1's host-to-device copy overlaps step k's compute
+    # and device-to-host copy (PCIe moves both directions at once).
     e2e = None
     if not args.no_e2e:
         hin = {k: torch.from_numpy(v).pin_memory() for k, v in job["host"].items()}
-        hout = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in job["outs"].items()}
+        sets = [B0, job["buffers"](B0)]
+        hout = {k: torch.empty_like(B0[k], device="cpu").pin_memory() for k in job["outs"]}
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        set_calls = [job["calls_for"](B, s) for B in sets]
+        in_done = [torch.cuda.Event() for _ in sets]
+        comp_done = [torch.cuda.Event() for _ in sets]
+        out_done = [torch.cuda.Event() for _ in sets]
 
-        def e2e_step():
-            for k, t in hin.items():
-                job["dev"][k].copy_(t, non_blocking=True)
-            step()
-            for k, t in hout.items():
-                t.copy_(job["outs"][k], non_blocking=True)
+        def e2e_run(nsteps):
+            for k in range(nsteps):
+                i = k % 2
+                B = sets[i]
+                if k >= 2:
+                    s_in.wait_event(comp_done[i])  # step k-2 has read this set's inputs
+                with torch.cuda.stream(s_in):
+                    for name, t in hin.items():
+                        B[name].copy_(t, non_blocking=True)
+                in_done[i].record(s_in)
+                stream.wait_event(in_done[i])
+                if k >= 2:
+                    stream.wait_event(out_done[i])  # step k-2's results are on the host
+                for p in passes:
+                    set_calls[i][p]()
+                if world > 1 and job["allreduce"] is not None:
+                    job["allreduce"](B)
+                comp_done[i].record(stream)
+                s_out.wait_event(comp_done[i])
+                with torch.cuda.stream(s_out):
+                    for name, t in hout.items():
+                        t.copy_(B[name], non_blocking=True)
+                out_done[i].record(s_out)
 
-        e2e_step()
+        e2e_run(2)
         barrier()
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        s_in.wait_stream(stream)
+        e2e_run(args.e2e_steps)
+        stream.wait_stream(s_out)
         z.record(stream)
         barrier()
         e_ms = a.elapsed_time(z)
@@ -504,7 +696,10 @@ def main():
             e_ms = max_over_ranks(e_ms, "cuda")
         e2e = {"value": N * world * args.e2e_steps / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps}
+               "steps": args.e2e_steps,
+               "copies": "pinned host buffers; H2D, compute and D2H on three streams, two "
+                         "device buffer sets alternating between steps"}
+        del sets, set_calls
     extra = {}
     if rank == 0 and "unfused" in job["extra"]:
         extra["unfused_ms"] = round(job["extra"]["unfused"](), 5)
@@ -519,18 +714,20 @@ def main():
     value = N * world * args.steps / (ms * 1e-3)
     peak, peak_src = measured_peaks()
     nbytes = job["bytes"]
-    mean_ms = {p: float(np.mean(v)) for p, v in per_pass.items()}
+    med_ms = {p: float(np.median(v)) for p, v in per_pass.items()}
     pass_report = {}
     for p in passes:
-        gbs = nbytes[p] / (mean_ms[p] * 1e-3) / 1e9
-        pass_report[p] = {"ms": round(mean_ms[p], 5), "GB_s": round(gbs, 1),
-                          "frac_hbm": round(gbs / peak, 4), "algorithmic_bytes": nbytes[p]}
+        gbs = nbytes[p] / (med_ms[p] * 1e-3) / 1e9
+        pass_report[p] = {"median_ms": round(med_ms[p], 5), "min_ms": round(min(per_pass[p]), 5),
+                          "mean_ms": round(float(np.mean(per_pass[p])), 5),
+                          "GB_s": round(gbs, 1), "frac_hbm": round(gbs / peak, 4),
+                          "algorithmic_bytes": nbytes[p]}
         alg, dense = job["flops"][p]
         if alg:
-            pass_report[p]["alg_TFLOP_s"] = round(alg / (mean_ms[p] * 1e-3) / 1e12, 2)
-            pass_report[p]["dense_equiv_TFLOP_s"] = round(dense / (mean_ms[p] * 1e-3) / 1e12, 2)
-    dom = max((p for p in passes if p != "wfft"), key=lambda p: mean_ms[p])
-    achieved = nbytes[dom] / (mean_ms[dom] * 1e-3) / 1e9
+            pass_report[p]["alg_TFLOP_s"] = round(alg / (med_ms[p] * 1e-3) / 1e12, 2)
+            pass_report[p]["dense_equiv_TFLOP_s"] = round(dense / (med_ms[p] * 1e-3) / 1e12, 2)
+    dom = max((p for p in passes if p != "wfft"), key=lambda p: med_ms[p])
+    achieved = nbytes[dom] / (med_ms[dom] * 1e-3) / 1e9
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -547,7 +744,10 @@ def main():
         "dtype": "f16" if w.dtype == "fp16" else "f32",
         "data": "synthetic",
         "config": dict({"workload": w.name}, **job["config"],
-                       passes=passes, accumulate="f32", l2="inputs larger than L2, no flush",
+                       passes=passes, accumulate="f32",
+                       l2="no flush: every pass streams more than twice the 126 MB L2"
+                       if sum(nbytes[p] for p in passes if p != "wfft") > 2 * 126e6
+                       else "no flush (inputs smaller than L2: warm)",
                        global_tokens=N * world,
                        parallelism=f"dp{world}" if world > 1 else "single"),
         "effective_TFLOP_s": round(sum(job["flops"][p][1] for p in passes) * world
@@ -556,13 +756,16 @@ def main():
                                    / peak, 2),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "peak_source": peak_src},
+                     "traffic": traffic, "peak_source": peak_src,
+                     "duration": "median of the pass's CUDA-event times in the timed loop"},
         "passes": pass_report,
         "gpu_launches": nkern * args.steps,
         "clocks": clk,
         "e2e": e2e,
     }
     line.update(extra)
+    if not args.no_per_config and args.workload == WORKLOAD_ID and args.dtype is None:
+        line["per_config"] = per_config_report(F, torch, stream, args.config_reps)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))

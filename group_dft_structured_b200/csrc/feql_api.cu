@@ -1181,6 +1181,8 @@ extern "C" int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW,
     p.split_len = align_up(cdiv(N > 0 ? N : 1, max_splits), p.TB);
     p.splits = static_cast<int>(cdiv(N > 0 ? N : 1, p.split_len));
   }
+  // the kernels index the array by split: never launch a plan that outgrows it
+  if (tc_dw_ws_floats(p) > cap) return FEQL_ERR_UNSUPPORTED;
   void *scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != FEQL_OK) return st;

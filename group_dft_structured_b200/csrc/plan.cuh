@@ -54,7 +54,7 @@ __host__ __device__ inline int sw32_offset(int row, int k) {
 
 // Layout of the opaque What buffer.
 //   fp16 tensor-core modes: [fwd chunks][dx chunks], each direction laid out
-//       [tile j][chunk kc][rows 0..5BD) with rows
+//       [tile j][chunk kc][rows 0..5BD) with rows (every bin divided by 4)
 //       [0,BD) What0 | [BD,2BD) What2 | [2BD,3BD) Re1 | [3BD,4BD) Im1 | [4BD,5BD) -Re1
 //   so that rows [2BD,4BD) = (Re1 ; Im1) multiply Re X1 and the overlapping
 //   window [3BD,5BD) = (Im1 ; -Re1) multiplies the stored -Im X1 plane.

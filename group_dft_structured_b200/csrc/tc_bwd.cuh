@@ -14,7 +14,8 @@
 //   warp 0      TMA: every 16-channel box of dy and x for the 64 tokens
 //   warps 2..17 4-point rDFT of every (token, channel) fibre, in place, one
 //               fibre row per thread: each 8 KB box becomes four 2 KB planes
-//               (V0, V2, Re V1, -Im V1), rows = tokens, 32-byte swizzle; in a
+//               (V0, V2, Re V1, -Im V1, each divided by 4 as in tc_fwd.cuh),
+//               rows = tokens, 32-byte swizzle; in a
 //               dy box the first 4 KB hold V0 and V2 interleaved in blocks of
 //               16 token rows (V0 of tokens 16j.., then V2 of the same
 //               tokens); db sums in registers
@@ -286,7 +287,7 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint4 v = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-            rdft4_pair(v, pl[k][0][q], pl[k][1][q], pl[k][2][q], pl[k][3][q]);
+            rdft4_pair_q(v, pl[k][0][q], pl[k][1][q], pl[k][2][q], pl[k][3][q]);
           }
         }
       }
@@ -407,9 +408,10 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           for (int i = 0; i < 8; ++i) {
             const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
             const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-            const float e = 0.25f * (Y0 + Y2), o = 0.25f * (Y0 - Y2);
-            packed[2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-            packed[2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+            // dy planes and weights are both stored divided by 4 (Y = 16 * acc)
+            const float e = 4.f * (Y0 + Y2), o = 4.f * (Y0 - Y2);
+            packed[2 * i] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
+            packed[2 * i + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
           }
           // C is even, so channels go out in 16-byte pairs
           const int c0 = g * 16 + h * 8;

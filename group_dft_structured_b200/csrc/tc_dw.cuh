@@ -15,7 +15,8 @@
 //   warp 0      TMA: the d-tile's dy boxes and the c-tile's x boxes (16
 //               channels x 4 group elements x TB tokens each) into a raw ring
 //   warps 2..9  4-point rDFT (packed fp16 pairs) of every (token, channel)
-//               fibre into planes X0, X2, Re X1, -Im X1 laid out MN-major
+//               fibre into planes X0, X2, Re X1, -Im X1 (each divided by 4,
+//               as in tc_fwd.cuh) laid out MN-major
 //               (channel contiguous, token = K), 32-byte swizzle; one
 //               (16-channel box, token) item per thread; db partial sums
 //   warp 1      TMEM allocator + MMA issuer: per 16 tokens six M=128 x N=CT
@@ -275,7 +276,7 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const uint4 v = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-          rdft4_pair(v, pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+          rdft4_pair_q(v, pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
         }
         uint8_t *dst = is_dy ? planes + b * chunk_plane : planes + x_off + (b - nqd) * chunk_plane;
         const int pstride = is_dy ? 8 * chunk_plane : p.nqc_max * chunk_plane;
@@ -391,10 +392,10 @@ dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict
       for (int q = 0; q < kRedGroups; ++q)
 #pragma unroll
         for (int k = 0; k < 4; ++k) t[k] += part[q][k][lo];
-      const float ev = 0.25f * (t[0] + t[1]), od = 0.25f * (t[0] - t[1]);
+      const float ev = 4.f * (t[0] + t[1]), od = 4.f * (t[0] - t[1]);
       uint2 pk;
-      pk.x = pack_half2(ev + 0.5f * t[2], od - 0.5f * t[3]);
-      pk.y = pack_half2(ev - 0.5f * t[2], od + 0.5f * t[3]);
+      pk.x = pack_half2(ev + 8.f * t[2], od - 8.f * t[3]);
+      pk.y = pack_half2(ev - 8.f * t[2], od + 8.f * t[3]);
       *reinterpret_cast<uint2 *>(dW + e * kT) = pk;
     }
   } else if (db != nullptr) {
@@ -407,7 +408,7 @@ dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict
     if (grp == 0 && d < D) {
       float t = 0.f;
       for (int q = 0; q < kRedGroups; ++q) t += part[q][0][lo];
-      db[d] = __float2half_rn(t);
+      db[d] = __float2half_rn(4.f * t);
     }
   }
 }
@@ -419,6 +420,8 @@ __host__ __device__ inline int64_t dw_reduce_scalar_blocks(int C, int D) {
 
 // Sum of the split partials in a fixed order, inverse rDFT, fp16 cast:
 //   dW[d][c][u] = (G0 + (-1)^u G2)/4 + Re(G1 i^u)/2,   db[d] = sum of partials.
+// The partials come from planes divided by 4 on both sides (G/16, and db/4),
+// so the constants applied are 4, 8 and 4.
 // A dW block owns `q` quads (one d, four consecutive c, all four bins: 16
 // floats) and 256/q split groups; thread (group g, quad) adds splits g, g +
 // groups, ... with 16-byte loads, then the groups are folded pairwise in a fixed
@@ -491,10 +494,10 @@ dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
         const int c = c0 + i;
         if (c >= C) break;
         const float g0 = red[i][t], g2 = red[4 + i][t], gr = red[8 + i][t], gi = red[12 + i][t];
-        const float ev = 0.25f * (g0 + g2), od = 0.25f * (g0 - g2);
+        const float ev = 4.f * (g0 + g2), od = 4.f * (g0 - g2);
         uint2 pk;
-        pk.x = pack_half2(ev + 0.5f * gr, od - 0.5f * gi);
-        pk.y = pack_half2(ev - 0.5f * gr, od + 0.5f * gi);
+        pk.x = pack_half2(ev + 8.f * gr, od - 8.f * gi);
+        pk.y = pack_half2(ev - 8.f * gr, od + 8.f * gi);
         *reinterpret_cast<uint2 *>(dW + (static_cast<int64_t>(d) * C + c) * kT) = pk;
       }
     }
@@ -512,7 +515,7 @@ dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
       if (grp < h) red[0][t] += red[0][t + h * kRedDbItems];
     }
     __syncthreads();
-    if (grp == 0 && d < D) db[d] = __float2half_rn(red[0][t]);
+    if (grp == 0 && d < D) db[d] = __float2half_rn(4.f * red[0][t]);
   }
 }
 

@@ -16,7 +16,8 @@
 //   warps 2-4, 6-8, 10, 11
 //                transform, two 4-warp teams taking alternate chunks: 4-point
 //                rDFT of the chunk (packed fp16 pairs), in place, into four
-//                K-major operand planes (X0, X2, Re X1, -Im X1)
+//                K-major operand planes (X0, X2, Re X1, -Im X1), each divided
+//                by 4 so that any finite fp16 input has finite bins
 //   warps 12..19 epilogue, two 4-warp teams: tcgen05.ld of the four fp32
 //                accumulators, inverse rDFT + bias, fp16 pack, swizzled smem
 //                staging; each warp owns 32 token rows and issues its own TMA
@@ -284,7 +285,7 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
           raw[q] = *reinterpret_cast<const uint4 *>(st + r * 128 + ((q ^ (r & 7)) << 4));
         uint32_t pl[4][8];  // [plane][channel pair] packed half2: V0, V2, Re V1, -Im V1
 #pragma unroll
-        for (int q = 0; q < 8; ++q) rdft4_pair(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+        for (int q = 0; q < 8; ++q) rdft4_pair_q(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
         named_bar_sync(2 + team, 128);  // every row read before the planes overwrite it
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
@@ -353,9 +354,11 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
             const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
             const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
             const float bv = sbias[d0 + h * 8 + i];
-            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
-            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+            // planes and weights are both stored divided by 4: Y = 16 * acc, so the
+            // inverse's 1/4 and 1/2 become 4 and 8
+            const float e = fmaf(4.f, Y0 + Y2, bv), o = fmaf(4.f, Y0 - Y2, bv);
+            packed[16 * h + 2 * i] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
+            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
           }
         }
         if (d0 >= p.Do) continue;  // whole group is padding

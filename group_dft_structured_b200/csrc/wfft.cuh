@@ -37,6 +37,8 @@ __device__ __forceinline__ void weight_bins(const T *__restrict__ W, int C, int 
 }
 
 // Tensor-core layout (fp16): one thread per element of the tiled buffer.
+// The bins are stored divided by 4 (exact), so that every bin of a finite fp16
+// weight is finite; the passes' epilogues undo the scale in fp32.
 __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict__ What,
                                WhatLayout L, int C) {
   const int64_t n_fwd = L.fwd.bytes / 2, n_dx = L.dx.bytes / 2;
@@ -65,7 +67,7 @@ __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict
       else v = -b1r;
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
-    *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);
+    *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(0.25f * v);
   }
 }
 

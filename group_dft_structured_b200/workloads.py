@@ -129,3 +129,30 @@ def make_mlp_inputs(wid: int, N: int, C: int, H: int, Co: int, dtype: str) -> di
             "b1": _normal(base + 2, (H,), 0.02, dtype),
             "W2": _normal(base + 4, (Co, H, 4), 1.0 / np.sqrt(4 * H), dtype),
             "b2": _normal(base + 5, (Co,), 0.02, dtype)}
+
+
+def _magnitude(seed: int, shape, lo: float, hi: float, dtype: str) -> np.ndarray:
+    """Values with |v| uniform in [lo, hi] and a random sign (seeded)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    mag = rng.uniform(lo, hi, size=shape)
+    sign = np.where(rng.integers(0, 2, size=shape) == 1, 1.0, -1.0)
+    return (sign * mag).astype(np_dtype(dtype))
+
+
+def make_range_inputs(wid: int, N: int, C: int, D: int, x_range, dy_range,
+                      w_std: float, b_std: float = 0.02, T: int = 4) -> dict:
+    """fp16 inputs at the edges of the half-precision range.
+
+    x and dy have magnitudes uniform in x_range / dy_range (pairs (lo, hi)) with
+    random signs; W ~ N(0, w_std^2), b ~ N(0, b_std^2).  Used to check that the
+    fp16 path handles every finite fp16 input (large ones whose group-axis sums
+    leave the fp16 range, and small ones near the subnormals) as long as the
+    outputs themselves are representable: the caller picks w_std and the other
+    operand's range so that y, dx and dW stay finite.
+    Seeds: 20260000 + 100 * wid + {x: 0, W: 1, b: 2, dy: 3}.
+    """
+    base = 20260000 + 100 * wid
+    return {"x": _magnitude(base + 0, (N, C, T), *x_range, "fp16"),
+            "W": _normal(base + 1, (D, C, T), w_std, "fp16"),
+            "b": _normal(base + 2, (D,), b_std, "fp16"),
+            "dy": _magnitude(base + 3, (N, D, T), *dy_range, "fp16")}

@@ -39,6 +39,10 @@ def _inputs(wid, N, C, D):
 
 def test_noalloc_matches_workspace_version_on_consecutive_calls():
     lib = F.load()
+    # the 256 x 256 case needs more than the 16 MiB array with the regular
+    # split count, so it runs the reduced-split plan; fail loudly if a planner
+    # or device change ever stops exercising that path
+    assert F.feql_backward_dw_workspace_bytes(3000, 256, 256, F.FEQL_FP16) > 16 << 20
     # two calls in a row on different shapes: the second must not see the
     # first one's leftovers in the shared scratch array
     for wid, (N, C, D) in [(11, (20000, 24, 96)), (12, (3000, 256, 256)), (13, (517, 48, 192))]:
