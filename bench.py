@@ -477,6 +477,13 @@ def roofline_us(nbytes, flops, dtype, peaks):
     return (t_mem, "hbm") if t_mem >= t_cmp else (t_cmp, "tensor" if dtype == "fp16" else "alu")
 
 
+def hold_gpu(torch, ms=20.0):
+    """Keeps the current stream busy for about `ms` milliseconds (a spin kernel),
+    so that the host enqueues the launches that follow before the GPU reaches
+    them: the CUDA-event times then hold no host-side launch gaps."""
+    torch.cuda._sleep(int(ms * 1e-3 * 1.965e9))
+
+
 def per_config_report(F, torch, stream, reps):
     """Every layer configuration at full size: median and min over `reps` CUDA-event
     timings of each pass, the L2 flushed before every rep by reading a buffer of
@@ -525,6 +532,7 @@ def per_config_report(F, torch, stream, reps):
                 calls[p]()
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(reps)]
+            hold_gpu(torch)  # the reps queue up behind it: no host gaps between them
             for a, z in ev:
                 flush.sum()
                 a.record(stream)
@@ -626,6 +634,7 @@ def main():
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
+    hold_gpu(torch)  # before the timed region: the host runs ahead of the GPU
     t_start.record(stream)
     for k in range(args.steps):
         step(evs[k])

@@ -313,9 +313,11 @@ int launch_tc_dw(TcDwParams p, const void *x, const void *dy, __half *dW, __half
     const int grid = p.tiles_d * p.tiles_c * p.splits;
     tc_dw_kernel<<<grid, kDwThreads, smem, stream>>>(tm_dy, tm_x, p);
   }
-  if (launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D, p.Cs,
-                          dev.sms, stream) != 0)
-    return FEQL_ERR_UNSUPPORTED;
+  {
+    const int r = launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.N > 0 ? p.splits : 0, p.C, p.D,
+                                      p.Cs, dev.sms, stream);
+    if (r != 0) return r == 1 ? FEQL_ERR_UNSUPPORTED : FEQL_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -375,12 +377,19 @@ int launch_tc_bwd(TcBwdParams p, const void *x, const void *dy, const uint8_t *w
                                   p.nqc) == FEQL_OK;
   if (!p.stack_x) st = make_tmap_f16(&tm_x, x, p.N, static_cast<int64_t>(p.C) * kT, kBwTB);
   if (st != FEQL_OK) return st;
-  if (cudaFuncSetAttribute(tc_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  // db from the dW bin-0 MMA when the last x box has a padding channel
+  auto kernel = (p.C % 16) != 0 ? tc_bwd_kernel<true> : tc_bwd_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FEQL_ERR_CUDA;
-  tc_bwd_kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, p);
-  if (launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs, dev.sms, stream) != 0)
-    return FEQL_ERR_UNSUPPORTED;
+  kernel<<<p.splits, kBwThreads, smem, stream>>>(tm_dy, tm_x, p);
+  if (cudaGetLastError() != cudaSuccess) return FEQL_ERR_CUDA;
+  // the split reduce as the kernel's programmatic dependent (see tc_dw.cuh)
+  {
+    const int r =
+        launch_dw_tc_reduce(p.ws, p.ws_db, dW, db, p.splits, p.C, p.D, p.Cs, dev.sms, stream);
+    if (r != 0) return r == 1 ? FEQL_ERR_UNSUPPORTED : FEQL_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -824,7 +833,8 @@ size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
   if (!valid_dtype(dtype) || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
-  if (is_tc(resolve(dtype))) return static_cast<size_t>(tc_dw_ws_floats(make_tc_dw_plan(N, C, D, dev.sms))) * 4;
+  if (is_tc(resolve(dtype)))
+    return static_cast<size_t>(tc_dw_ws_floats(make_tc_dw_plan(N, C, D, dev.sms))) * 4;
   return static_cast<size_t>(make_dw_plan(N, C, D, dev.sms).ws_floats) * 4;
 }
 

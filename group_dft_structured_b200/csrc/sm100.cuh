@@ -113,6 +113,21 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch
+// ----------------------------------------------------------------------------
+// A kernel launched after this one with programmatic stream serialization may
+// be scheduled once every CTA of this grid has signalled (or exited); its
+// launch latency then overlaps this kernel's tail.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the preceding grid (when this one was launched as its
+// programmatic dependent) has completed and its memory operations are visible.
+// A no-op for a grid launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------
 // TMA and bulk copies
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
@@ -276,6 +291,16 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                  "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// Warp-wide, 16 TMEM lanes from taddr's lane: thread t gets columns 2(t%4) and
+// 2(t%4)+1 of lane t/4 (r[0], r[1]) and of lane t/4 + 8 (r[2], r[3]).  Four
+// threads share a row, so a row's eight columns land in four neighbouring
+// threads (the layout that lets each four lanes store one row's 64 bytes).
+__device__ __forceinline__ void tmem_ld16x256(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(taddr));
 }
 

@@ -15,29 +15,31 @@
 //   warps 2..17 4-point rDFT of every (token, channel) fibre, in place, one
 //               fibre row per thread: each 8 KB box becomes four 2 KB planes
 //               (V0, V2, Re V1, -Im V1, each divided by 4 as in tc_fwd.cuh),
-//               rows = tokens, 32-byte swizzle; in a
-//               dy box the first 4 KB hold V0 and V2 interleaved in blocks of
-//               16 token rows (V0 of tokens 16j.., then V2 of the same
-//               tokens); db sums in registers
+//               rows = tokens, 32-byte swizzle; in a dy box the first 4 KB
+//               hold V0 and V2 interleaved in blocks of 16 token rows (V0 of
+//               tokens 16j.., then V2 of the same tokens) and the second 4 KB
+//               Re V1 and -Im V1 the same way; db sums in registers
 //   warp 1      TMEM allocator + MMA issuer:
 //                 dW: per 16 tokens six M=128 (d) x N=CT (c) MMAs, both
 //                     operands MN-major (the planes read column-wise)
 //                 dX: per 16-channel d chunk, against the resident
 //                     conj(What)^T tiles, K-major (the same planes read
-//                     row-wise), into a double-buffered accumulator: bins 0
-//                     and 2 as one M=128 MMA over the interleaved V0/V2 rows
-//                     with N = 2 BD (What0 | What2; the cross products in the
-//                     other halves are not read), bin 1 as two M=64 MMAs
+//                     row-wise), into a double-buffered accumulator, two
+//                     M=128 MMAs: bins 0 and 2 over the interleaved V0/V2
+//                     rows with N = 2 BD (What0 | What2; the cross products
+//                     in the other halves are not read), and bin 1 over the
+//                     interleaved Re V1 / -Im V1 rows against the window
+//                     (Re1 ; Im1), whose four products the epilogue combines
 //   warps 18..21 dX epilogue: warp q's TMEM lane quadrant holds tokens
-//               16q..16q+15: in lanes 0..15 for bin 0 and for the M=64 bin-1
-//               accumulator (lanes (m mod 16) + 32 * (m / 16)), in lanes
-//               16..31 for bin 2 (moved down by a shuffle); inverse rDFT,
-//               fp16, direct 16-byte stores
-//               (each lane writes whole channels of its own token row), which
-//               leaves the shared memory to the stages (three fit for C = 24,
-//               D = 96)
+//               16q..16q+15 in lanes 0..15 (V0 and Re V1 rows) and 16..31
+//               (V2 and -Im V1 rows); 16x256b TMEM loads give each thread two
+//               channels of two tokens from both halves, so the inverse rDFT
+//               needs no shuffle and each four lanes store one token's 64
+//               contiguous bytes (fp16, direct stores), which leaves the
+//               shared memory to the stages (three fit for C = 24, D = 96)
 // After the last stage warps 2..17 write the dW partials and db to the
-// workspace.  Every wait is bounded.
+// workspace; the split reduce of tc_dw.cuh, launched as this kernel's
+// programmatic dependent, finishes dW and db.  Every wait is bounded.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -79,11 +81,11 @@ struct TcBwdParams {
 };
 
 // Byte offset of token row r of plane pp (0..3) inside a transformed dy box:
-// V0 and V2 interleaved in 16-row blocks (a 128-row K-major operand for the
-// merged bins-0/2 dX MMA, one 512-byte block per 16-token dW step), then the
-// Re V1 and -Im V1 planes.
+// V0 and V2 interleaved in 16-row blocks in the first 4 KB, Re V1 and -Im V1
+// the same way in the second (each half a 128-row K-major operand for one
+// merged dX MMA; one 512-byte block per plane and 16-token dW step).
 __device__ __forceinline__ int bw_dy_row(int pp, int r) {
-  return pp < 2 ? ((r >> 4) << 10) + (pp << 9) + ((r & 15) << 5) : pp * kBwPlane + (r << 5);
+  return ((pp >> 1) << 12) + ((r >> 4) << 10) + ((pp & 1) << 9) + ((r & 15) << 5);
 }
 
 struct BwSmem {
@@ -103,6 +105,12 @@ __host__ __device__ inline BwSmem tc_bwd_smem(const TcBwdParams &p) {
 // 22 warps over the 4 SM sub-partitions put 6 warps on one 16K-register slice:
 // 6 x 32 x 80 = 15,360 (88 would not fit).  The transform is latency-bound, so
 // it gets many warps with one item each rather than few with several.
+// kDbCol: C is not a multiple of 16, so the last x box has a padding channel
+// (p.C itself, zero in the loaded data).  The transform sets that channel's
+// bin-0 plane value to 1/4, so the dW bin-0 MMA produces
+//   G0[d][C] = sum_n (dY0[n,d] / 4) * (1/4) = db[d] / 16
+// in the padding column and db needs no accumulation in registers.
+template <bool kDbCol>
 __global__ void __maxnreg__(80)
 tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
               const TcBwdParams p) {
@@ -192,9 +200,9 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       // dW: planes hold -Im of bin 1 for dy and x alike (see tc_dw.cuh)
       const uint32_t id_w = instr_desc(128, p.CT, 0, 0, 1, 1);
       const uint32_t id_wneg = instr_desc(128, p.CT, 0, 0, 1, 1, 1);
-      // dX: M = 64 tokens, K-major operands
-      const uint32_t id_x02 = instr_desc(128, 2 * p.BD, 0, 0);  // bins 0 and 2, interleaved rows
-      const uint32_t id_x2 = instr_desc(64, 2 * p.BD, 0, 0);
+      // dX: K-major operands, M = 128 interleaved rows (bins 0 and 2, or Re and
+      // -Im of bin 1, of 64 tokens)
+      const uint32_t id_x = instr_desc(128, 2 * p.BD, 0, 0);
       const uint32_t acc0 = tmem_base, acc2 = tmem_base + p.CT;
       const uint32_t acc1r = tmem_base + 2 * p.CT, acc1i = tmem_base + 3 * p.CT;
       const uint32_t acca = tmem_base + 2 * p.CT, accb = tmem_base + 4 * p.CT;
@@ -225,11 +233,11 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
         if (ok) {
 #pragma unroll
           for (int k = 0; k < kBwTB / 16; ++k) {
-            // dy planes: d chunks 8 KB apart, V0/V2 blocks of 16 tokens interleaved
-            // (1 KB per step), Re/-Im V1 planes 2 KB each; x planes: plane-major,
-            // c chunks 2 KB apart; 16 tokens = 512 B
+            // dy planes: d chunks 8 KB apart, V0/V2 and Re/-Im V1 blocks of 16
+            // tokens interleaved (1 KB per step, the bin-1 pair 4 KB in); x
+            // planes: plane-major, c chunks 2 KB apart; 16 tokens = 512 B
             const uint32_t A0 = mn + k * 64, A1 = A0 + 32;
-            const uint32_t A2 = mn + 2 * (kBwPlane >> 4) + k * 32, A3 = A2 + (kBwPlane >> 4);
+            const uint32_t A2 = A0 + 256, A3 = A2 + 32;
             const uint32_t B0 = mx + k * 32, B1 = B0 + xb16;
             const uint32_t B2 = B1 + xb16, B3 = B2 + xb16;
             const uint32_t first = (ch == 0 && k == 0) ? 0u : 1u;
@@ -251,9 +259,8 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           uint32_t ab = kl, wb = wl;  // running box and weight-chunk descriptor words
           for (int q = 0; q < p.nqd; ++q, ab += kBwBox >> 4, wb += chunk16) {
             const uint32_t in = q > 0 ? 1u : 0u;
-            mma_f16_lo(acc, ab, wb, dhi, id_x02, in);
-            mma_f16_lo(acc + 2 * p.BD, ab + 2 * (kBwPlane >> 4), wb + 2 * w1, dhi, id_x2, in);
-            mma_f16_lo(acc + 2 * p.BD, ab + 3 * (kBwPlane >> 4), wb + 3 * w1, dhi, id_x2, 1u);
+            mma_f16_lo(acc, ab, wb, dhi, id_x, in);
+            mma_f16_lo(acc + 2 * p.BD, ab + 256, wb + 2 * w1, dhi, id_x, in);
           }
           mma_commit(&dxfull[b]);
           mma_commit(&empty[s]);
@@ -267,11 +274,12 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
     // ---------------------------------------------------------- transform
     const int t = threadIdx.x - 64;
     constexpr int kPer = kBwMaxItems / (kBwXfWarps * 32);  // items per thread (1)
-    float db_acc[kPer][16];
+    constexpr int kDbRegs = kDbCol ? 1 : 16;                 // db accumulators per item
+    float db_acc[kPer][kDbRegs];
 #pragma unroll
     for (int k = 0; k < kPer; ++k)
 #pragma unroll
-      for (int c = 0; c < 16; ++c) db_acc[k][c] = 0.f;
+      for (int c = 0; c < kDbRegs; ++c) db_acc[k][c] = 0.f;
     int s = 0;
     uint32_t ph = 0;
     for (int ch = 0; ch < nst; ++ch) {
@@ -300,12 +308,20 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           // dy box: its four planes in place (bw_dy_row); x box q: plane pp at
           // x + (pp * nqc + q) planes
           const bool is_dy = b < p.nqd;
+          if (kDbCol && b == p.nqd + p.C / 16) {
+            // the padding channel C of this x box: bin 0 = 1 (stored as 1/4)
+            const int cq = (p.C % 16) >> 1;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (q == cq) pl[k][0][q] = (p.C & 1) ? (pl[k][0][q] & 0xFFFFu) | 0x34000000u
+                                                  : (pl[k][0][q] & 0xFFFF0000u) | 0x3400u;
+          }
           uint8_t *base = is_dy ? st + b * kBwBox : st + p.nqd * kBwBox + (b - p.nqd) * kBwPlane;
           // planes 0, 1 and 2, 3 are each one stride apart
           const int o01 = is_dy ? bw_dy_row(0, r) : r * 32;
           const int s01 = is_dy ? 512 : p.nqc * kBwPlane;
           const int o23 = is_dy ? bw_dy_row(2, r) : 2 * p.nqc * kBwPlane + r * 32;
-          const int s23 = is_dy ? kBwPlane : p.nqc * kBwPlane;
+          const int s23 = s01;
 #pragma unroll
           for (int pp = 0; pp < 4; ++pp) {
             uint8_t *row = base + (pp < 2 ? o01 + pp * s01 : o23 + (pp - 2) * s23);
@@ -315,12 +331,12 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
                   make_uint4(pl[k][pp][4 * hh + 0], pl[k][pp][4 * hh + 1], pl[k][pp][4 * hh + 2],
                              pl[k][pp][4 * hh + 3]);
           }
-          if (b < p.nqd) {
+          if (!kDbCol && b < p.nqd) {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float2 f = __half22float2(as_h2(pl[k][0][q]));
-              db_acc[k][2 * q] += f.x;
-              db_acc[k][2 * q + 1] += f.y;
+              db_acc[k][2 * q % kDbRegs] += f.x;
+              db_acc[k][(2 * q + 1) % kDbRegs] += f.y;
             }
           }
         }
@@ -350,8 +366,18 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
           o[1] = make_float4(G[bin][4], G[bin][5], G[bin][6], G[bin][7]);
         }
       }
+      if (kDbCol && d < p.D && g == p.C / 8) {
+        // db partial in the padding column; the reduce expects sum of dY0 / 4
+        const int j = p.C % 8;
+        float v = G[0][0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i)
+          if (i == j) v = G[0][i];
+        p.ws_db[static_cast<int64_t>(split) * p.D + d] = 4.f * v;
+      }
     }
     tc_fence_before();
+    if (!kDbCol) {
     // db: fixed-order reduction of the per-thread partials through shared memory
     named_bar_sync(3, kBwXfWarps * 32);  // stages are free: every chunk has been consumed
     float *sdb = reinterpret_cast<float *>(smem + L.stage0);  // [kBwMaxItems][16]
@@ -367,61 +393,65 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
       const int dd = bb * 16 + c;
       if (dd < p.D) p.ws_db[static_cast<int64_t>(split) * p.D + dd] = sum;
     }
+    }
   } else {
     // ------------------------------------------------------- dX epilogue
+    // Per 8-channel block six 16x256b loads: thread t holds channels
+    // c0 + 2(t%4) and c0 + 2(t%4) + 1 of tokens 16q + t/4 and 16q + t/4 + 8:
+    //   bin 0 (lanes 0..15, columns [0, BD)), bin 2 (lanes 16..31, [BD, 2BD)),
+    //   bin 1: Re rows (lanes 0..15) and -Im rows (16..31) against (Re1 ; Im1)
+    //   (columns [2BD, 4BD)): Re Y1 = a_r + b_i, Im Y1 = a_i - b_r.
     const int quad = warp & 3;
-    const int groups = p.BD / 16;
     const int64_t row_elems = static_cast<int64_t>(p.C) * kT;
+    const int nblk = (p.C + 7) / 8;    // 8-channel blocks holding real channels
+    const int tc = 2 * (lane & 3);     // first channel of this thread's pair in a block
     int b = 0;
     uint32_t bph = 0;
     for (int ch = 0; ch < nst; ++ch, b = b + 1 == p.ndx ? 0 : b + 1, bph ^= (b == 0)) {
       if (ok) ok = mbar_wait(&dxfull[b], bph);
       tc_fence_after();
-      const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + dx0 + b * 4 * p.BD;
-      // lanes 0..15 hold this warp's 16 tokens
-      const int64_t n = t_begin + static_cast<int64_t>(ch) * kBwTB + quad * 16 + lane;
-      const bool row_ok = lane < 16 && n < t_end;
-      __half *drow = p.dx + n * row_elems;
-      for (int g = 0; g < groups; ++g) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 8 columns at a time keeps registers low
-          uint32_t y0[8], y2[8], y1r[8], y1i[8];
-          const uint32_t col = tl + g * 16 + h * 8;
-          // the TMEM loads are warp-collective: reconverge after the wait and the
-          // per-lane stores of the previous step
+      const uint32_t lo = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + dx0 + b * 4 * p.BD;
+      const uint32_t hi = lo + (16u << 16);
+      const int64_t n0 = t_begin + static_cast<int64_t>(ch) * kBwTB + quad * 16 + (lane >> 2);
+      __half *row0 = p.dx + n0 * row_elems, *row1 = row0 + 8 * row_elems;
+      for (int g = 0; g < nblk; ++g) {
+        const int c0 = 8 * g;
+        uint32_t y0[4], y2[4], ar[4], ai[4], br[4], bi[4];
+        // the TMEM loads are warp-collective: reconverge after the wait and the
+        // per-lane stores of the previous block
+        __syncwarp();
+        tmem_ld16x256(lo + c0, y0);
+        tmem_ld16x256(hi + p.BD + c0, y2);
+        tmem_ld16x256(lo + 2 * p.BD + c0, ar);
+        tmem_ld16x256(lo + 3 * p.BD + c0, ai);
+        tmem_ld16x256(hi + 2 * p.BD + c0, br);
+        tmem_ld16x256(hi + 3 * p.BD + c0, bi);
+        tmem_ld_wait();
+        if (g == nblk - 1) {
+          tc_fence_before();
           __syncwarp();
-          tmem_ld8(col, y0);
-          tmem_ld8(col + p.BD, y2);
-          tmem_ld8(col + 2 * p.BD, y1r);
-          tmem_ld8(col + 3 * p.BD, y1i);
-          tmem_ld_wait();
-          if (h == 1 && g == groups - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
-          }
-          // bin 2 of token 16q + l sits in lane l + 16 (the V2 rows of the merged MMA)
+          if (lane == 0 && ok) mbar_arrive(&dxempty[b]);
+        }
+        // dy planes and weights are both stored divided by 4 (Y = 16 * acc);
+        // out[i] = (u0, u1) and (u2, u3) of register i's (token, channel)
+        uint32_t out[4][2];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) y2[i] = __shfl_down_sync(0xffffffffu, y2[i], 16);
-          uint32_t packed[16];  // channel i: packed[2i] = (y0, y1), packed[2i+1] = (y2, y3)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-            // dy planes and weights are both stored divided by 4 (Y = 16 * acc)
-            const float e = 4.f * (Y0 + Y2), o = 4.f * (Y0 - Y2);
-            packed[2 * i] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
-            packed[2 * i + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
-          }
-          // C is even, so channels go out in 16-byte pairs
-          const int c0 = g * 16 + h * 8;
-          if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (c0 + 2 * j + 2 <= p.C)
-                *reinterpret_cast<uint4 *>(drow + (c0 + 2 * j) * kT) = make_uint4(
-                    packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
+        for (int i = 0; i < 4; ++i) {
+          const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
+          const float Yr = __uint_as_float(ar[i]) + __uint_as_float(bi[i]);
+          const float Yi = __uint_as_float(ai[i]) - __uint_as_float(br[i]);
+          const float e = 4.f * (Y0 + Y2), o = 4.f * (Y0 - Y2);
+          out[i][0] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
+          out[i][1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
+        }
+        // C is even: a thread's channel pair is either whole or past the end
+        if (c0 + tc + 2 <= p.C) {
+          if (n0 < t_end)
+            *reinterpret_cast<uint4 *>(row0 + (c0 + tc) * kT) =
+                make_uint4(out[0][0], out[0][1], out[1][0], out[1][1]);
+          if (n0 + 8 < t_end)
+            *reinterpret_cast<uint4 *>(row1 + (c0 + tc) * kT) =
+                make_uint4(out[2][0], out[2][1], out[3][0], out[3][1]);
         }
       }
     }
@@ -429,6 +459,9 @@ tc_bwd_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__
 
   tc_fence_before();
   __syncthreads();
+  // the partial sums are written: the split reduce (launched as this grid's
+  // programmatic dependent) may be scheduled as the CTAs exit
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);

@@ -351,6 +351,9 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
 
   tc_fence_before();
   __syncthreads();
+  // the partial sums are written: the split reduce (launched as this grid's
+  // programmatic dependent) may be scheduled as the CTAs exit
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
@@ -358,10 +361,12 @@ tc_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ 
 }
 
 // Small outputs (a few thousand (d, c) pairs, where the vector kernel below
-// has too few blocks): a block takes 32 consecutive (d, c) outputs (the last
-// blocks take db); its 16 warps each sum every 16th split, then warp 0 adds the
-// 16 partial sums in warp order — the same grouping on every run.
-constexpr int kRedOut = 32, kRedGroups = 16;
+// has too few blocks): a block takes 16 consecutive (d, c) outputs (the last
+// blocks take db); its 32 thread groups each sum every 32nd split, then the
+// first group adds the 32 partial sums in group order — the same grouping on
+// every run.  Both reduce kernels may be launched as programmatic dependents
+// of the kernel that writes the partials (pdl_wait before the first read).
+constexpr int kRedOut = 16, kRedGroups = 32;
 constexpr int64_t kRedScalarMaxOut = 8192;  // D * C up to which the scalar kernel runs
 
 __global__ void __launch_bounds__(kRedOut * kRedGroups)
@@ -369,6 +374,7 @@ dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict
                     __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
                     int Cs) {
   __shared__ float part[kRedGroups][4][kRedOut];
+  pdl_wait();
   const int64_t plane = static_cast<int64_t>(D) * Cs;
   const int64_t n = static_cast<int64_t>(D) * C;
   const int64_t nblk_w = cdiv(n, kRedOut);
@@ -378,6 +384,7 @@ dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict
     float g[4] = {0.f, 0.f, 0.f, 0.f};
     if (e < n) {
       const float *src = ws + (e / C) * Cs + (e % C);
+#pragma unroll 4
       for (int s = grp; s < splits; s += kRedGroups) {
         const float *q = src + static_cast<int64_t>(s) * 4 * plane;
 #pragma unroll
@@ -402,6 +409,7 @@ dw_tc_reduce_scalar_kernel(const float *__restrict__ ws, const float *__restrict
     const int64_t d = (blockIdx.x - nblk_w) * kRedOut + lo;
     float sdb = 0.f;
     if (d < D)
+#pragma unroll 4
       for (int s = grp; s < splits; s += kRedGroups) sdb += ws_db[static_cast<int64_t>(s) * D + d];
     part[grp][0][lo] = sdb;
     __syncthreads();
@@ -452,6 +460,7 @@ dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
                     __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
                     int Cs, int q, int64_t wblocks) {
   __shared__ float red[16][kRedThreads];
+  pdl_wait();
   const int t = threadIdx.x;
   if (blockIdx.x < wblocks) {
     const int groups = kRedThreads / q;
@@ -520,20 +529,33 @@ dw_tc_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
 }
 
 // Launches the split reduce that suits the output size (both sum the splits in
-// a fixed order).
+// a fixed order) as a programmatic dependent of the kernel before it on the
+// stream: its blocks take the SMs as that kernel's CTAs exit and wait there
+// (pdl_wait) for its partial sums, so no launch gap separates the two.
 inline int launch_dw_tc_reduce(const float *ws, const float *ws_db, __half *dW, __half *db,
                                int splits, int C, int D, int Cs, int sms, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.stream = stream;
+  cfg.dynamicSmemBytes = 0;
+  cudaError_t e;
   if (static_cast<int64_t>(D) * C <= kRedScalarMaxOut) {
-    dw_tc_reduce_scalar_kernel<<<static_cast<unsigned>(dw_reduce_scalar_blocks(C, D)),
-                                 kRedOut * kRedGroups, 0, stream>>>(ws, ws_db, dW, db, splits, C,
-                                                                    D, Cs);
+    cfg.gridDim = dim3(static_cast<unsigned>(dw_reduce_scalar_blocks(C, D)));
+    cfg.blockDim = dim3(kRedOut * kRedGroups);
+    e = cudaLaunchKernelEx(&cfg, dw_tc_reduce_scalar_kernel, ws, ws_db, dW, db, splits, C, D, Cs);
   } else {
     const RedPlan rp = make_red_plan(C, D, sms);
     if (rp.blocks > 0x7fffffff) return 1;
-    dw_tc_reduce_kernel<<<static_cast<unsigned>(rp.blocks), kRedThreads, 0, stream>>>(
-        ws, ws_db, dW, db, splits, C, D, Cs, rp.q, rp.wblocks);
+    cfg.gridDim = dim3(static_cast<unsigned>(rp.blocks));
+    cfg.blockDim = dim3(kRedThreads);
+    e = cudaLaunchKernelEx(&cfg, dw_tc_reduce_kernel, ws, ws_db, dW, db, splits, C, D, Cs, rp.q,
+                           rp.wblocks);
   }
-  return 0;
+  return e == cudaSuccess ? 0 : 2;
 }
 
 }  // namespace feql
