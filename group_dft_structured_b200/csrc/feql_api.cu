@@ -165,6 +165,7 @@ int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __h
   p.nacc = (4 * P.BD <= 256) ? 2 : 1;
   p.acc_stride = p.nacc == 2 ? 256 : 0;
   p.bias_floats = P.nD * P.BD;
+  p.out = static_cast<__half *>(out);
   const int budget = dev.smem_optin - 1024;  // 1 KB for aligning the base
   // Resident weights when the CTA's slice fits beside >= 4 input stages and
   // there are enough CTAs for one fixed output tile each.
@@ -190,15 +191,13 @@ int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __h
     grid = p.n_units < dev.sms ? p.n_units : dev.sms;
   }
 
-  CUtensorMap tm_in, tm_out;
+  CUtensorMap tm_in;
   st = make_tmap_f16(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT);
-  if (st != FEQL_OK) return st;
-  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT, kOutRows);
   if (st != FEQL_OK) return st;
   if (cudaFuncSetAttribute(tc_fourier_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return FEQL_ERR_CUDA;
-  tc_fourier_gemm_kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, tm_out, p);
+  tc_fourier_gemm_kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, p);
   return launch_status();
 }
 

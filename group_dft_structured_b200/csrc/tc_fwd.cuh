@@ -19,9 +19,9 @@
 //                K-major operand planes (X0, X2, Re X1, -Im X1), each divided
 //                by 4 so that any finite fp16 input has finite bins
 //   warps 12..19 epilogue, two 4-warp teams: tcgen05.ld of the four fp32
-//                accumulators, inverse rDFT + bias, fp16 pack, swizzled smem
-//                staging; each warp owns 32 token rows and issues its own TMA
-//                stores
+//                accumulators, inverse rDFT + bias, fp16 pack, direct 16-byte
+//                global stores (each four lanes write one token row's 64
+//                contiguous bytes of an 8-channel block)
 // Per chunk the MMA warp issues four M=128 x K=16 MMAs:
 //   acc[0, BD)    += X0  * What0^T                (N = BD)
 //   acc[BD, 2BD)  += X2  * What2^T                (N = BD)
@@ -58,9 +58,6 @@ __device__ __forceinline__ int tc_xf_ordinal(int w) {
 }
 constexpr int kXChunkBytes = kBM * kCK * kT * 2;  // 16 KB: 128 rows x 128 B
 constexpr int kPlaneBytes = kBM * kCK * 2;        // 4 KB: 128 rows x 32 B
-constexpr int kOutRows = 32;                      // rows per epilogue TMA store (one warp)
-constexpr int kOutBoxBytes = kOutRows * 64 * 2;   // 4 KB: 32 rows x (16 ch x 4) fp16
-constexpr int kNumOut = 2;                        // staging buffers per epilogue warp
 constexpr int kTmemCols = 512;
 
 struct TcFwdParams {
@@ -76,19 +73,19 @@ struct TcFwdParams {
   int stages;
   int stage_bytes;      // 16 KB input chunk (+ weight chunk unless resident), 1 KB aligned
   int bias_floats;      // nD * BD
+  __half *out;          // [N][Do][4]
 };
 
 struct TcSmem {
   // offsets (bytes) from the 1024-aligned dynamic smem base
-  int wres, stage0, out0, bias, bars, total;
+  int wres, stage0, bias, bars, total;
 };
 
 __host__ __device__ inline TcSmem tc_fwd_smem(const TcFwdParams &p) {
   TcSmem s;
   s.wres = 0;
   s.stage0 = p.resident ? p.wres_bytes : 0;
-  s.out0 = s.stage0 + p.stages * p.stage_bytes;
-  s.bias = s.out0 + 4 * kTeams * kNumOut * kOutBoxBytes;
+  s.bias = s.stage0 + p.stages * p.stage_bytes;
   s.bars = s.bias + static_cast<int>(align_up(p.bias_floats * 4, 16));
   // full, tready, empty per stage; acc_full, acc_empty per acc buffer; final; wfull; tmem slot
   s.total = s.bars + (3 * p.stages + 2 * 2 + 2) * 8 + 16;
@@ -133,8 +130,7 @@ struct TcUnits {
 // 20 warps over the 4 SM sub-partitions put 5 warps on each 16K-register
 // slice: 5 x 32 x 96 = 15,360 registers fits, 104 would not.
 __global__ void __maxnreg__(96)
-tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
-                       const __grid_constant__ CUtensorMap tm_out, const TcFwdParams p) {
+tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -182,7 +178,6 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       tma_prefetch_desc(&tm_in);
-      tma_prefetch_desc(&tm_out);
       TcUnits U(p);
       if (p.resident && U.valid) {
         mbar_arrive_expect_tx(wfull, p.nK * p.chunk_bytes);
@@ -307,17 +302,19 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
     // kTeams teams of 4 warps.  With double-buffered accumulators each team
     // owns one TMEM buffer (alternate tiles); with a single buffer the teams
     // split each tile's 16-column groups.  Each warp owns one TMEM lane
-    // quadrant (32 token rows) and stores its rows with its own TMA stores.
+    // quadrant (32 token rows).  It reads them with 16x256b loads (four lanes
+    // per token row, two channels each) and stores each row's 64-byte channel
+    // blocks straight to global memory: every store instruction writes 8 rows
+    // x 64 contiguous bytes, and no shared memory goes to output staging.
     const int ew = warp - kTcEpi0;           // epilogue warp index
     const int eteam = ew / 4;
     const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-    uint8_t *obase = smem + L.out0 + ew * kNumOut * kOutBoxBytes;
     const int groups = p.BD / 16;
     const bool split = p.nacc == 1;
     const int g0 = split ? eteam : 0, gstep = split ? kTeams : 1;
     int last_g = -1;
     for (int g = g0; g < groups; g += gstep) last_g = g;
-    int oi = 0, it = 0;
+    int it = 0;
     for (TcUnits U(p); U.valid; U.next(), ++it) {
       const int m = U.m, j = U.j;
       if (!split && it % kTeams != eteam) continue;
@@ -332,53 +329,59 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in,
         if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
       }
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
+      // thread t: rows r0 = 32 quad + 16 half + t/4 (and r0 + 8), channels
+      // c + 2(t%4) and c + 2(t%4) + 1 of each 8-channel block c
+      const int tcp = 2 * (lane & 3);
+      const int64_t row0 = static_cast<int64_t>(m) * kBM + quad * 32 + (lane >> 2);
+      const int64_t row_elems = static_cast<int64_t>(p.Do) * kT;
       for (int g = g0; g < groups; g += gstep) {
-        const int d0 = j * p.BD + g * 16;
-        uint32_t packed[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 8 columns at a time keeps registers low
-          uint32_t y0[8], y2[8], y1r[8], y1i[8];
-          const uint32_t col = tl + g * 16 + h * 8;
-          tmem_ld8(col, y0);
-          tmem_ld8(col + p.BD, y2);
-          tmem_ld8(col + 2 * p.BD, y1r);
-          tmem_ld8(col + 3 * p.BD, y1i);
+        for (int h = 0; h < 2; ++h) {
+          const int c = g * 16 + h * 8;
+          uint32_t y0[2][4], y2[2][4], yr[2][4], yi[2][4];
+          __syncwarp();  // the TMEM loads are warp-collective
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t col = tl + (static_cast<uint32_t>(16 * hf) << 16) + c;
+            tmem_ld16x256(col, y0[hf]);
+            tmem_ld16x256(col + p.BD, y2[hf]);
+            tmem_ld16x256(col + 2 * p.BD, yr[hf]);
+            tmem_ld16x256(col + 3 * p.BD, yi[hf]);
+          }
           tmem_ld_wait();
           if (h == 1 && g == last_g) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
           }
+          const int d = j * p.BD + c + tcp;  // this thread's first output channel
+          if (d + 2 > p.Do) continue;        // Do is even: the pair is whole or padding
+          const float b0 = sbias[d], b1 = sbias[d + 1];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
-            const float Yr = __uint_as_float(y1r[i]), Yi = __uint_as_float(y1i[i]);
-            const float bv = sbias[d0 + h * 8 + i];
-            // planes and weights are both stored divided by 4: Y = 16 * acc, so the
-            // inverse's 1/4 and 1/2 become 4 and 8
-            const float e = fmaf(4.f, Y0 + Y2, bv), o = fmaf(4.f, Y0 - Y2, bv);
-            packed[16 * h + 2 * i] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
-            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
+          for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {  // rows r0 and r0 + 8
+              uint32_t w[4];
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const int i = 2 * rr + cc;
+                const float Y0 = __uint_as_float(y0[hf][i]), Y2 = __uint_as_float(y2[hf][i]);
+                const float Yr = __uint_as_float(yr[hf][i]), Yi = __uint_as_float(yi[hf][i]);
+                const float bv = cc ? b1 : b0;
+                // planes and weights are both stored divided by 4 (Y = 16 * acc)
+                const float e = fmaf(4.f, Y0 + Y2, bv), o = fmaf(4.f, Y0 - Y2, bv);
+                w[2 * cc] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
+                w[2 * cc + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
+              }
+              const int64_t row = row0 + 16 * hf + 8 * rr;
+              if (row < p.N)
+                *reinterpret_cast<uint4 *>(p.out + row * row_elems + static_cast<int64_t>(d) * kT) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
-        if (d0 >= p.Do) continue;  // whole group is padding
-        uint8_t *ob = obase + (oi % kNumOut) * kOutBoxBytes;
-        if (lane == 0) bulk_wait_read<kNumOut - 1>();  // this buffer's last store has read it
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4 *>(ob + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tm_out, d0 * kT, m * kBM + quad * 32, ob);
-          bulk_commit();
-        }
-        ++oi;
       }
     }
-    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
