@@ -16,6 +16,11 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfeql.so")
+# Failure-detection test build: a 20 ms bound on every device-side wait and one
+# accumulator-release arrive left out of the forward kernel, so that a bounded
+# wait runs out (tests/test_wait_timeout_gpu.py).  Not for use outside tests.
+TIMEOUT_LIB = os.path.join(PKG, "libfeql_waittest.so")
+TIMEOUT_FLAGS = ["-DFEQL_WAIT_LIMIT_NS=20000000ull", "-DFEQL_TEST_SKIP_FIRST_RELEASE=1"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -45,17 +50,18 @@ def deps() -> list[str]:
     return out
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-o", LIB + ".tmp", *sources()]
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          lib: str = LIB) -> str:
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-o", lib + ".tmp", *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
@@ -64,8 +70,13 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose:
         print(r.stdout + r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
+
+
+def build_waittest(force: bool = False) -> str:
+    """The failure-detection test library (see TIMEOUT_LIB)."""
+    return build(force=force, extra=TIMEOUT_FLAGS, lib=TIMEOUT_LIB)
 
 
 if __name__ == "__main__":

@@ -44,6 +44,18 @@
 namespace feql {
 
 constexpr int kTeams = 2;                         // transform teams and epilogue teams
+
+// Failure-detection test builds (FEQL_TEST_SKIP_FIRST_RELEASE, compiled into a
+// separate library with a short FEQL_WAIT_LIMIT_NS) leave out one arrive: the
+// first epilogue warp never releases the first accumulator it drains.  The MMA
+// thread's bounded wait for that buffer then runs out, the kernel winds down
+// (every role stops waiting once its own wait has run out; loads already
+// issued are still awaited, TMEM is freed) and FEQL_ERR_TIMEOUT is reported.
+#ifdef FEQL_TEST_SKIP_FIRST_RELEASE
+constexpr bool kSkipFirstRelease = true;
+#else
+constexpr bool kSkipFirstRelease = false;
+#endif
 // Warp w runs on SM sub-partition w % 4.  Sub-partition 1 holds the MMA issuer
 // (warp 1), so warps 5 and 9 stay idle and the transform warps sit on the other
 // three sub-partitions: warps 2-4, 6-8, 10-11 transform, 12-19 epilogue.
@@ -352,7 +364,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
           if (h == 1 && g == last_g) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
+            if (lane == 0 && ok && !(kSkipFirstRelease && ew == 0 && it == 0))
+              mbar_arrive(&acc_empty[a]);
           }
           const int d = j * p.BD + c + tcp;  // this thread's first output channel
           if (d + 2 > p.Do) continue;        // Do is even: the pair is whole or padding
