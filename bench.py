@@ -67,6 +67,8 @@ def parse():
                     help="skip the per-configuration table (configurations 1-5, L2 flushed)")
     ap.add_argument("--config-reps", type=int, default=50,
                     help="timed reps per pass in the per-configuration table")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -495,6 +497,13 @@ def per_config_report(F, torch, stream, reps):
     from group_dft_structured_b200.workloads import WORKLOADS, workload_inputs
     meas, nom = peak_table()
     s = stream.cuda_stream
+    traffic = {}
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        if tj.get("source_hash") == kernel_source_hash():
+            traffic = tj
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
     flush = torch.ones(2 * l2 // 4, dtype=torch.float32, device="cuda")
     out = {}
@@ -543,7 +552,8 @@ def per_config_report(F, torch, stream, reps):
             med, mn = float(np.median(us)), us[0]
             r = {"median_us": round(med, 3), "min_us": round(mn, 3), "reps": reps,
                  "algorithmic_bytes": nbytes[p],
-                 "GB_s": round(nbytes[p] / (med * 1e-6) / 1e9, 1)}
+                 "GB_s": round(nbytes[p] / (med * 1e-6) / 1e9, 1),
+                 "traffic": traffic.get(w.name, {}).get(p)}
             if flops[p]:
                 r["tokens_per_s"] = round(N / (med * 1e-6), 1)
                 r["alg_TFLOP_s"] = round(flops[p] / (med * 1e-6) / 1e12, 3)
@@ -590,9 +600,9 @@ def main():
     from group_dft_structured_b200.workloads import WORKLOADS
 
     w = WORKLOADS[args.workload]
-    if args.dtype is not None:
+    if args.dtype is not None or args.tokens is not None:
         import dataclasses
-        w = dataclasses.replace(w, dtype=args.dtype)
+        w = dataclasses.replace(w, dtype=args.dtype or w.dtype, N=args.tokens or w.N)
     torch.cuda.set_device(local_rank)
     if world > 1:
         from datetime import timedelta
@@ -773,7 +783,8 @@ def main():
         "e2e": e2e,
     }
     line.update(extra)
-    if not args.no_per_config and args.workload == WORKLOAD_ID and args.dtype is None:
+    if (not args.no_per_config and args.workload == WORKLOAD_ID and args.dtype is None
+            and args.tokens is None):
         line["per_config"] = per_config_report(F, torch, stream, args.config_reps)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
