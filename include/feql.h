@@ -32,6 +32,14 @@
  *    enqueued (FEQL_ERR_CUDA: a launch failed; see feql_status_string).
  *  - N == 0 is a valid no-op (for feql_backward_dw it zeroes dW and db); the
  *    token-indexed pointers (x, y, dy, dx) may then be NULL.
+ *  - Value range (FEQL_FP16): every finite fp16 x, dy and W is accepted.  The
+ *    group-axis sums of the transform reach 4 max|v|, so the fp16 operand
+ *    planes and Fourier weights hold every bin divided by 4 (an exact power
+ *    of two that the fp32 epilogues undo); results are within the fp16 mode's
+ *    tolerance whenever the outputs y, dx, dW and db themselves are finite in
+ *    fp16 (an output beyond 65504 becomes inf, as in any fp16 layer).  A bin
+ *    whose quarter falls among the fp16 subnormals (|bin| < 2^-12) is rounded
+ *    to the subnormal spacing: an absolute error of at most 2^-23 per bin.
  */
 #ifndef FEQL_H
 #define FEQL_H
