@@ -449,14 +449,17 @@ def setup_mlp(args, w, rank, s, F, torch):
 # x 2 FLOP x 1.965 GHz = 74.4 TFLOP/s.  The measured HBM and tensor figures come
 # from MEASURED_PEAKS.json (copy bandwidth; cuBLAS bf16, the same tensor rate as
 # fp16); the CUDA-core fp32 peak has no measurement and uses the nominal count.
-NOMINAL = {"hbm_gbs": 8000.0, "tensor_tflops": 2250.0, "fp32_fma_tflops": 74.4}
+NOMINAL = {"hbm_gbs": 8000.0, "tensor_tflops": 2250.0, "fp32_fma_tflops": 74.4,
+           "tf32_tflops": 1125.0}
 
 # The five layer configurations, each with the passes its throughput is quoted
 # on (SURVEY of the method's workloads: forward for 1-3, dX and dW for 4,
 # forward and both gradients for 5; 3 also in fp32).
-CONFIG_RUNS = [(1, "fp32", ("fwd",)), (2, "fp16", ("fwd",)), (3, "fp16", ("fwd",)),
-               (3, "fp32", ("fwd",)), (4, "fp16", ("dx", "dw")),
-               (5, "fp16", ("fwd", "dx", "dw", "bwd"))]
+# fp32 runs in both fp32 modes: CUDA cores ("fp32") and split TF32 on the tensor
+# cores ("fp32_3xtf32", three tf32 products per product).
+CONFIG_RUNS = [(1, "fp32", ("fwd",)), (1, "fp32_3xtf32", ("fwd",)), (2, "fp16", ("fwd",)),
+               (3, "fp16", ("fwd",)), (3, "fp32", ("fwd",)), (3, "fp32_3xtf32", ("fwd",)),
+               (4, "fp16", ("dx", "dw")), (5, "fp16", ("fwd", "dx", "dw", "bwd"))]
 
 
 def peak_table():
@@ -466,17 +469,24 @@ def peak_table():
         with open(p) as f:
             d = json.load(f)
         meas = {"hbm_gbs": float(d["hbm_gbs"]), "tensor_tflops": float(d["bf16_tflops"]),
-                "fp32_fma_tflops": NOMINAL["fp32_fma_tflops"]}
+                "fp32_fma_tflops": NOMINAL["fp32_fma_tflops"],
+                # tf32 runs at half the bf16 rate per FLOP (the nominal 1.125 vs 2.25 PF)
+                "tf32_tflops": float(d["bf16_tflops"]) / 2}
     return meas, NOMINAL
 
 
 def roofline_us(nbytes, flops, dtype, peaks):
     """Roofline time (us) and its bound: the slower of the algorithmic bytes at
-    HBM bandwidth and the algorithmic FLOPs at the mode's arithmetic peak."""
+    HBM bandwidth and the algorithmic FLOPs at the mode's arithmetic peak (split
+    TF32 issues three tf32 products per product)."""
     t_mem = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e6
-    fpeak = peaks["tensor_tflops"] if dtype == "fp16" else peaks["fp32_fma_tflops"]
-    t_cmp = flops / (fpeak * 1e12) * 1e6
-    return (t_mem, "hbm") if t_mem >= t_cmp else (t_cmp, "tensor" if dtype == "fp16" else "alu")
+    if dtype == "fp16":
+        t_cmp, bound = flops / (peaks["tensor_tflops"] * 1e12) * 1e6, "tensor"
+    elif dtype == "fp32_3xtf32":
+        t_cmp, bound = 3 * flops / (peaks["tf32_tflops"] * 1e12) * 1e6, "tensor"
+    else:
+        t_cmp, bound = flops / (peaks["fp32_fma_tflops"] * 1e12) * 1e6, "alu"
+    return (t_mem, "hbm") if t_mem >= t_cmp else (t_cmp, bound)
 
 
 def hold_gpu(torch, ms=20.0):
@@ -510,9 +520,10 @@ def per_config_report(F, torch, stream, reps):
     for wid, dtype, passes in CONFIG_RUNS:
         w = WORKLOADS[wid]
         N, C, D = w.N, w.C, w.D
-        mode = F.FEQL_FP16 if dtype == "fp16" else F.FEQL_FP32
+        mode = {"fp16": F.FEQL_FP16, "fp32": F.FEQL_FP32_SIMT,
+                "fp32_3xtf32": F.FEQL_FP32_3XTF32}[dtype]
         elt = 2 if dtype == "fp16" else 4
-        inp = workload_inputs(wid, dtype=dtype)
+        inp = workload_inputs(wid, dtype="fp16" if dtype == "fp16" else "fp32")
         B = {k: torch.from_numpy(v).cuda() for k, v in inp.items()
              if k in (("x", "W", "b") + (("dy",) if set(passes) - {"fwd"} else ()))}
         What = torch.empty(F.feql_weight_fft_bytes(C, D, mode), dtype=torch.uint8, device="cuda")

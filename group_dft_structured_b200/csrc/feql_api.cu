@@ -114,6 +114,24 @@ int make_tmap_f16_boxes(CUtensorMap *m, const void *base, int64_t rows, int64_t 
   return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
 }
 
+// Row-major fp32 matrix [rows][cols] viewed as a 2-D tensor; box = 32 cols (128
+// bytes) x box_rows rows, 128-byte swizzle, zero fill out of range: the same
+// shared-memory image as make_tmap_f16's box, with 8 channels x 4 group
+// elements of fp32 per row.
+int make_tmap_f32(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                  int box_rows = kBM) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return FEQL_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  cuuint32_t box[2] = {32, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_dtype(int dt) { return dt >= FEQL_FP16 && dt <= FEQL_FP16_SIMT; }
@@ -121,7 +139,20 @@ bool valid_dtype(int dt) { return dt >= FEQL_FP16 && dt <= FEQL_FP16_SIMT; }
 // Resolves FEQL_FP32 to the library's fp32 algorithm.
 int resolve(int dt) { return dt == FEQL_FP32 ? FEQL_FP32_SIMT : dt; }
 
+// The p4 layer's FEQL_FP32: split TF32 on the tensor cores up to 512 channels on
+// either side (measured within the fp32 bound at that contraction depth per
+// bin), fp32 FMA on CUDA cores beyond.  Depends on (C, D) only, so the weight
+// transform and the passes agree on the Fourier buffer's layout.
+constexpr int kTf32MaxChannels = 512;
+int resolve(int dt, int C, int D) {
+  if (dt != FEQL_FP32) return dt;
+  return (C <= kTf32MaxChannels && D <= kTf32MaxChannels) ? FEQL_FP32_3XTF32 : FEQL_FP32_SIMT;
+}
+
 bool is_tc(int dt) { return dt == FEQL_FP16; }
+bool is_tf32(int dt) { return dt == FEQL_FP32_3XTF32; }
+// Layout kind of the Fourier-weight buffer of a (resolved) mode.
+int what_kind(int dt) { return is_tc(dt) ? kWhatF16 : (is_tf32(dt) ? kWhatTF32 : kWhatSimt); }
 bool is_half(int dt) { return dt == FEQL_FP16 || dt == FEQL_FP16_SIMT; }
 
 int check_shape(int C, int D) {
@@ -142,8 +173,9 @@ int grid_for(int64_t work, int threads, int sms) {
 }
 
 // ---------------------------------------------------------------- tc launch
-int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __half *bias,
-                   void *out, int64_t N, cudaStream_t stream) {
+// tf32: fp32 data in the split-TF32 mode (FEQL_FP32_3XTF32), else fp16.
+int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const void *bias,
+                   void *out, int64_t N, cudaStream_t stream, bool tf32 = false) {
   DeviceInfo dev;
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
@@ -165,19 +197,20 @@ int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __h
   p.nacc = (4 * P.BD <= 256) ? 2 : 1;
   p.acc_stride = p.nacc == 2 ? 256 : 0;
   p.bias_floats = P.nD * P.BD;
-  p.out = static_cast<__half *>(out);
+  p.out = out;
+  const int slot = tf32 ? 2 * kXChunkBytes : kXChunkBytes;  // input chunk / its planes
   const int budget = dev.smem_optin - 1024;  // 1 KB for aligning the base
   // Resident weights when the CTA's slice fits beside >= 4 input stages and
   // there are enough CTAs for one fixed output tile each.
   p.resident = 1;
   p.wres_bytes = static_cast<int>(align_up(static_cast<int64_t>(P.nK) * P.chunk_bytes, 1024));
-  p.stage_bytes = kXChunkBytes;
+  p.stage_bytes = slot;
   p.stages = 8;
   while (p.stages > 4 && tc_fwd_smem(p).total > budget) --p.stages;
   if (tc_fwd_smem(p).total > budget || dev.sms < P.nD) {
     p.resident = 0;
     p.wres_bytes = 0;
-    p.stage_bytes = kXChunkBytes + static_cast<int>(align_up(P.chunk_bytes, 1024));
+    p.stage_bytes = slot + static_cast<int>(align_up(P.chunk_bytes, 1024));
     p.stages = 8;
     while (p.stages > 2 && tc_fwd_smem(p).total > budget) --p.stages;
     if (tc_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
@@ -192,12 +225,13 @@ int launch_tc_gemm(const void *in, const uint8_t *wt, const TcPlan &P, const __h
   }
 
   CUtensorMap tm_in;
-  st = make_tmap_f16(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT);
+  st = tf32 ? make_tmap_f32(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT)
+            : make_tmap_f16(&tm_in, in, N, static_cast<int64_t>(P.Ci) * kT);
   if (st != FEQL_OK) return st;
-  if (cudaFuncSetAttribute(tc_fourier_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
+  auto kernel = tf32 ? tc_fourier_gemm_kernel<true> : tc_fourier_gemm_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return FEQL_ERR_CUDA;
-  tc_fourier_gemm_kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, p);
+  kernel<<<grid, kTcThreads, smem, stream>>>(tm_in, p);
   return launch_status();
 }
 
@@ -763,24 +797,25 @@ extern "C" {
 
 size_t feql_weight_fft_bytes(int C, int D, int dtype) {
   if (!valid_dtype(dtype) || check_shape(C, D) != FEQL_OK) return 0;
-  const int dt = resolve(dtype);
-  if (dt == FEQL_FP32_3XTF32) return 0;
-  return static_cast<size_t>(make_what_layout(C, D, is_tc(dt)).bytes);
+  return static_cast<size_t>(make_what_layout(C, D, what_kind(resolve(dtype, C, D))).bytes);
 }
 
 int feql_weight_fft(const void *W, void *What, int C, int D, int dtype, feql_stream stream) {
   if (!valid_dtype(dtype) || W == nullptr || What == nullptr) return FEQL_ERR_INVALID_ARG;
   if (check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
-  const int dt = resolve(dtype);
-  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  const int dt = resolve(dtype, C, D);
   if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
   DeviceInfo dev;
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const WhatLayout L = make_what_layout(C, D, is_tc(dt));
-  if (is_tc(dt)) {
+  const WhatLayout L = make_what_layout(C, D, what_kind(dt));
+  if (is_tf32(dt)) {
+    const int64_t words = (L.fwd.bytes + L.dx.bytes) / 4;
+    wfft_tf32_kernel<<<grid_for(words, 256, dev.sms), 256, 0, s>>>(
+        static_cast<const float *>(W), static_cast<uint8_t *>(What), L, C);
+  } else if (is_tc(dt)) {
     const int64_t elems = (L.fwd.bytes + L.dx.bytes) / 2;
     wfft_tc_kernel<<<grid_for(elems, 256, dev.sms), 256, 0, s>>>(
         static_cast<const __half *>(W), static_cast<uint8_t *>(What), L, C);
@@ -801,17 +836,19 @@ static int pass_common(const void *in, const void *What, const void *bias, void 
   if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
   if (bias != nullptr && !aligned16(bias)) return FEQL_ERR_INVALID_ARG;
-  const int dt = resolve(dtype);
-  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  const int dt = resolve(dtype, C, D);
   if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
   if (N == 0) return FEQL_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const WhatLayout L = make_what_layout(C, D, is_tc(dt));
+  const WhatLayout L = make_what_layout(C, D, what_kind(dt));
   const int Ci = dir == 0 ? C : D, Do = dir == 0 ? D : C;
+  if (is_tf32(dt)) {
+    const uint8_t *wt = static_cast<const uint8_t *>(What) + (dir == 0 ? L.off_fwd : L.off_dx);
+    return launch_tc_gemm(in, wt, dir == 0 ? L.fwd : L.dx, bias, out, N, s, true);
+  }
   if (is_tc(dt)) {
     const uint8_t *wt = static_cast<const uint8_t *>(What) + (dir == 0 ? L.off_fwd : L.off_dx);
-    return launch_tc_gemm(in, wt, dir == 0 ? L.fwd : L.dx, static_cast<const __half *>(bias), out,
-                          N, s);
+    return launch_tc_gemm(in, wt, dir == 0 ? L.fwd : L.dx, bias, out, N, s);
   }
   const float *Wp = static_cast<const float *>(What) + (dir == 0 ? L.off_fwd : L.off_dx) / 4;
   if (is_half(dt)) return launch_simt_fwd<__half>(in, Wp, bias, out, N, Ci, Do, s);
@@ -832,7 +869,7 @@ size_t feql_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
   if (!valid_dtype(dtype) || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
-  if (is_tc(resolve(dtype)))
+  if (is_tc(resolve(dtype, C, D)))
     return static_cast<size_t>(tc_dw_ws_floats(make_tc_dw_plan(N, C, D, dev.sms))) * 4;
   return static_cast<size_t>(make_dw_plan(N, C, D, dev.sms).ws_floats) * 4;
 }
@@ -847,8 +884,7 @@ int feql_backward(const void *x, const void *dy, const void *What, void *dx, voi
   if (!aligned16(x) || !aligned16(dy) || !aligned16(What) || !aligned16(dx) || !aligned16(dW) ||
       !aligned16(ws) || (db != nullptr && !aligned16(db)))
     return FEQL_ERR_INVALID_ARG;
-  const int dt = resolve(dtype);
-  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  const int dt = resolve(dtype, C, D);
   if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
   DeviceInfo dev;
   int st = device_info(&dev);
@@ -879,8 +915,8 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws
   if (!aligned16(x) || !aligned16(dy) || !aligned16(dW) || !aligned16(ws))
     return FEQL_ERR_INVALID_ARG;
   if (db != nullptr && !aligned16(db)) return FEQL_ERR_INVALID_ARG;
-  const int dt = resolve(dtype);
-  if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
+  // split-TF32 mode: the weight gradient runs on the fp32 CUDA-core kernels
+  const int dt = resolve(dtype, C, D);
   if (is_tc(dt) && ((C | D) & 1)) return FEQL_ERR_UNSUPPORTED;
   DeviceInfo dev;
   int st = device_info(&dev);

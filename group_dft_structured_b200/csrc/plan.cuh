@@ -14,6 +14,7 @@ namespace feql {
 constexpr int kT = 4;            // group order (p4)
 constexpr int kBM = 128;         // tokens per tile = tcgen05 M
 constexpr int kCK = 16;          // channels per K-chunk (one K=16 fp16 MMA step)
+constexpr int kCK32 = 8;         // channels per K-chunk in split-TF32 mode (one K=8 tf32 step)
 constexpr int kMaxBD = 128;      // largest output-channel tile (complex bin N = 2*BD <= 256)
 
 __host__ __device__ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -45,11 +46,32 @@ __host__ __device__ inline TcPlan make_tc_plan(int Ci, int Do) {
   return p;
 }
 
+// Split-TF32 direction plan (fp32 data, FEQL_FP32_3XTF32): chunks of 8
+// channels (a K-major row of 8 tf32 values is 32 bytes, the fp16 row's size),
+// the same output tiles, and per (tile, chunk) two 5-plane weight tiles: the
+// tf32-rounded bins (hi) and the tf32-rounded remainders (lo).
+__host__ __device__ inline TcPlan make_tc_plan_tf32(int Ci, int Do) {
+  TcPlan p;
+  p.Ci = Ci;
+  p.Do = Do;
+  p.nK = static_cast<int>(cdiv(Ci, kCK32));
+  p.nD = static_cast<int>(cdiv(Do, Ci <= 4 * kCK ? kMaxBD / 2 : kMaxBD));
+  p.BD = static_cast<int>(align_up(cdiv(Do, p.nD), 16));
+  p.chunk_bytes = 2 * 5 * p.BD * 32;
+  p.bytes = static_cast<int64_t>(p.nD) * p.nK * p.chunk_bytes;
+  return p;
+}
+
 // Byte offset of element (row, k) inside one weight chunk: K-major rows of
 // 16 fp16 (32 B) with the 32-byte swizzle (16-byte half-row index XOR bit 2
 // of the row), i.e. exactly the shared-memory image the MMA reads.
 __host__ __device__ inline int sw32_offset(int row, int k) {
   return row * 32 + ((((k >> 3) ^ (row >> 2)) & 1) << 4) + (k & 7) * 2;
+}
+
+// The same for 32-bit elements (8 per row): tf32 tiles.
+__host__ __device__ inline int sw32_offset4(int row, int k) {
+  return row * 32 + ((((k >> 2) ^ (row >> 2)) & 1) << 4) + (k & 3) * 4;
 }
 
 // Layout of the opaque What buffer.
@@ -59,17 +81,23 @@ __host__ __device__ inline int sw32_offset(int row, int k) {
 //   so that rows [2BD,4BD) = (Re1 ; Im1) multiply Re X1 and the overlapping
 //   window [3BD,5BD) = (Im1 ; -Re1) multiplies the stored -Im X1 plane.
 //   SIMT modes: fp32 planes [dir][bin p][Do][Ci], p = (0, 2, Re 1, Im 1).
+//   Split-TF32 mode: [fwd chunks][dx chunks] of make_tc_plan_tf32 tiles, each
+//       chunk the hi tile (rows as above, tf32 in 32-bit words, 32-byte
+//       swizzle) followed by the lo tile; bins not scaled.
+enum WhatKind { kWhatSimt = 0, kWhatF16 = 1, kWhatTF32 = 2 };
+
 struct WhatLayout {
   bool tc;
   TcPlan fwd, dx;
   int64_t off_fwd, off_dx, bytes;
 };
 
-__host__ __device__ inline WhatLayout make_what_layout(int C, int D, bool tc) {
+__host__ __device__ inline WhatLayout make_what_layout(int C, int D, int kind) {
   WhatLayout L;
+  const bool tc = kind != kWhatSimt;
   L.tc = tc;
-  L.fwd = make_tc_plan(C, D);
-  L.dx = make_tc_plan(D, C);
+  L.fwd = kind == kWhatTF32 ? make_tc_plan_tf32(C, D) : make_tc_plan(C, D);
+  L.dx = kind == kWhatTF32 ? make_tc_plan_tf32(D, C) : make_tc_plan(D, C);
   if (tc) {
     L.off_fwd = 0;
     L.off_dx = align_up(L.fwd.bytes, 1024);

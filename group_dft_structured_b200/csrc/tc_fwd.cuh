@@ -74,7 +74,7 @@ constexpr int kTmemCols = 512;
 
 struct TcFwdParams {
   const uint8_t *wt;    // weight chunks of this direction
-  const __half *bias;   // [Do] or nullptr
+  const void *bias;     // [Do] (fp16, or fp32 in split-TF32 mode) or nullptr
   int64_t N;
   int Ci, Do, BD, nD, nK, chunk_bytes;
   int nM;               // token tiles: ceil(N / 128)
@@ -83,9 +83,10 @@ struct TcFwdParams {
   int resident;         // 1: the CTA's weight slice is loaded once (fixed D tile per CTA)
   int wres_bytes;       // resident weight buffer: nK * chunk_bytes (1 KB aligned)
   int stages;
-  int stage_bytes;      // 16 KB input chunk (+ weight chunk unless resident), 1 KB aligned
+  int stage_bytes;      // input chunk slot (16 KB; 32 KB of planes in split-TF32 mode)
+                        // + weight chunk unless resident, 1 KB aligned
   int bias_floats;      // nD * BD
-  __half *out;          // [N][Do][4]
+  void *out;            // [N][Do][4], fp16 (fp32 in split-TF32 mode)
 };
 
 struct TcSmem {
@@ -141,6 +142,16 @@ struct TcUnits {
 
 // 20 warps over the 4 SM sub-partitions put 5 warps on each 16K-register
 // slice: 5 x 32 x 96 = 15,360 registers fits, 104 would not.
+//
+// kTF32: the split-TF32 mode of fp32 data (FEQL_FP32_3XTF32).  A chunk is 8
+// channels (the same 16 KB TMA box: 128 rows x 128 bytes of fp32), transformed
+// in fp32 into eight 4 KB planes (the four bins rounded to tf32, hi, and the
+// tf32-rounded remainders, lo) that overwrite the 32 KB slot; per chunk the
+// MMA thread issues three kind::tf32 MMAs (K = 8) per bin product,
+// A_hi B_hi + A_hi B_lo + A_lo B_hi (the lo x lo term, ~2^-22 of the product,
+// is dropped: Ootomo and Yokota's split-TF32 scheme), and the epilogue stores
+// fp32 rows.  Bins are not scaled (fp32 has the range).
+template <bool kTF32>
 __global__ void __maxnreg__(96)
 tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -174,8 +185,13 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
     mbar_init(wfull, 1);
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < p.bias_floats; i += blockDim.x)
-    sbias[i] = (p.bias != nullptr && i < p.Do) ? __half2float(p.bias[i]) : 0.f;
+  for (int i = threadIdx.x; i < p.bias_floats; i += blockDim.x) {
+    float bv = 0.f;
+    if (p.bias != nullptr && i < p.Do)
+      bv = kTF32 ? static_cast<const float *>(p.bias)[i]
+                 : __half2float(static_cast<const __half *>(p.bias)[i]);
+    sbias[i] = bv;
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -206,11 +222,11 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
             uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
             if (p.resident) {
               mbar_arrive_expect_tx(&full[s], kXChunkBytes);
-              tma_load_2d(st, &tm_in, kc * (kCK * kT), m * kBM, &full[s]);
+              tma_load_2d(st, &tm_in, kc * (kTF32 ? kCK32 * kT : kCK * kT), m * kBM, &full[s]);
             } else {
               mbar_arrive_expect_tx(&full[s], kXChunkBytes + p.chunk_bytes);
-              tma_load_2d(st, &tm_in, kc * (kCK * kT), m * kBM, &full[s]);
-              bulk_load(st + kXChunkBytes,
+              tma_load_2d(st, &tm_in, kc * (kTF32 ? kCK32 * kT : kCK * kT), m * kBM, &full[s]);
+              bulk_load(st + (kTF32 ? 2 * kXChunkBytes : kXChunkBytes),
                         p.wt + (static_cast<int64_t>(j) * p.nK + kc) * p.chunk_bytes,
                         p.chunk_bytes, &full[s]);
             }
@@ -222,8 +238,9 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
-      const uint32_t id_bd = instr_desc(kBM, p.BD, 0, 0);
-      const uint32_t id_2bd = instr_desc(kBM, 2 * p.BD, 0, 0);
+      const uint32_t fmt = kTF32 ? 2u : 0u;  // operand format: tf32 or f16
+      const uint32_t id_bd = instr_desc(kBM, p.BD, fmt, fmt);
+      const uint32_t id_2bd = instr_desc(kBM, 2 * p.BD, fmt, fmt);
       const uint32_t wrow = 32;  // bytes per weight row (16 fp16)
       const uint64_t dsw32 = smem_desc(0, 16, 256, kSw32);  // K-major, 32-byte swizzle
       const uint32_t stage_base = smem_u32(smem + L.stage0), wres_base = smem_u32(smem + L.wres);
@@ -252,12 +269,27 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
           tc_fence_after();
           if (ok) {
             const uint32_t xd = x0 + s * stage16;
-            const uint32_t wd = p.resident ? wr : xd + (kXChunkBytes >> 4);
+            const uint32_t wd =
+                p.resident ? wr : xd + ((kTF32 ? 2 * kXChunkBytes : kXChunkBytes) >> 4);
             const uint32_t acc_in = kc > 0 ? 1u : 0u;
-            mma_f16_lo(acc, xd, wd, dhi, id_bd, acc_in);
-            mma_f16_lo(acc + p.BD, xd + pl16, wd + w16, dhi, id_bd, acc_in);
-            mma_f16_lo(acc + 2 * p.BD, xd + 2 * pl16, wd + 2 * w16, dhi, id_2bd, acc_in);
-            mma_f16_lo(acc + 2 * p.BD, xd + 3 * pl16, wd + 3 * w16, dhi, id_2bd, 1u);
+            if constexpr (kTF32) {
+              // planes 0..3 hi, 4..7 lo; the lo weight tile 5 BD rows after the hi one
+              const uint32_t lo_x = 4 * pl16, lo_w = 5 * w16;
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t dcol = acc + (b < 2 ? b : 2) * p.BD;
+                const uint32_t id = b < 2 ? id_bd : id_2bd;
+                const uint32_t in = (b == 3) ? 1u : acc_in;  // window b adds onto window a
+                mma_tf32_lo(dcol, xd + b * pl16, wd + b * w16, dhi, id, in);
+                mma_tf32_lo(dcol, xd + b * pl16, wd + b * w16 + lo_w, dhi, id, 1u);
+                mma_tf32_lo(dcol, xd + b * pl16 + lo_x, wd + b * w16, dhi, id, 1u);
+              }
+            } else {
+              mma_f16_lo(acc, xd, wd, dhi, id_bd, acc_in);
+              mma_f16_lo(acc + p.BD, xd + pl16, wd + w16, dhi, id_bd, acc_in);
+              mma_f16_lo(acc + 2 * p.BD, xd + 2 * pl16, wd + 2 * w16, dhi, id_2bd, acc_in);
+              mma_f16_lo(acc + 2 * p.BD, xd + 3 * pl16, wd + 3 * w16, dhi, id_2bd, 1u);
+            }
             mma_commit(&empty[s]);
           }
           if (++s == p.stages) { s = 0; ph ^= 1; }
@@ -285,23 +317,52 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
         }
         if (ok) ok = mbar_wait(&full[s], ph);
         uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
-        // row r: 8 x 16 B, logical chunk q = channels 2q, 2q+1 (x 4 group elements)
+        // row r: 8 x 16 B; fp16: logical chunk q = channels 2q, 2q+1 (x 4 group
+        // elements); fp32: chunk q = channel q's four group elements
         uint4 raw[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           raw[q] = *reinterpret_cast<const uint4 *>(st + r * 128 + ((q ^ (r & 7)) << 4));
-        uint32_t pl[4][8];  // [plane][channel pair] packed half2: V0, V2, Re V1, -Im V1
+        if constexpr (kTF32) {
+          named_bar_sync(2 + team, 128);  // every row read before the planes overwrite it
+          // per half row (channels 4h..4h+3): the four bins in fp32, each split into
+          // its tf32 rounding (planes 0..3) and the rounded remainder (planes 4..7)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) rdft4_pair_q(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
-        named_bar_sync(2 + team, 128);  // every row read before the planes overwrite it
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pl[8][4];
 #pragma unroll
-        for (int pp = 0; pp < 4; ++pp) {
-          uint8_t *plane = st + pp * kPlaneBytes + r * 32;
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = raw[4 * h + q];
+              const float v0 = __uint_as_float(u.x), v1 = __uint_as_float(u.y);
+              const float v2 = __uint_as_float(u.z), v3 = __uint_as_float(u.w);
+              const float a = v0 + v2, b = v1 + v3;
+              const float bins[4] = {a + b, a - b, v0 - v2, v1 - v3};  // V0, V2, Re V1, -Im V1
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-            *reinterpret_cast<uint4 *>(plane + (((h ^ (r >> 2)) & 1) << 4)) =
-                make_uint4(pl[pp][4 * h + 0], pl[pp][4 * h + 1], pl[pp][4 * h + 2],
-                           pl[pp][4 * h + 3]);
+              for (int k = 0; k < 4; ++k) {
+                pl[k][q] = tf32_rna(bins[k]);
+                pl[4 + k][q] = tf32_rna(bins[k] - __uint_as_float(pl[k][q]));
+              }
+            }
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp)
+              *reinterpret_cast<uint4 *>(st + pp * kPlaneBytes + r * 32 +
+                                         (((h ^ (r >> 2)) & 1) << 4)) =
+                  make_uint4(pl[pp][0], pl[pp][1], pl[pp][2], pl[pp][3]);
+          }
+        } else {
+          uint32_t pl[4][8];  // [plane][channel pair] packed half2: V0, V2, Re V1, -Im V1
+#pragma unroll
+          for (int q = 0; q < 8; ++q) rdft4_pair_q(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+          named_bar_sync(2 + team, 128);  // every row read before the planes overwrite it
+#pragma unroll
+          for (int pp = 0; pp < 4; ++pp) {
+            uint8_t *plane = st + pp * kPlaneBytes + r * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              *reinterpret_cast<uint4 *>(plane + (((h ^ (r >> 2)) & 1) << 4)) =
+                  make_uint4(pl[pp][4 * h + 0], pl[pp][4 * h + 1], pl[pp][4 * h + 2],
+                             pl[pp][4 * h + 3]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -368,6 +429,30 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
               mbar_arrive(&acc_empty[a]);
           }
           const int d = j * p.BD + c + tcp;  // this thread's first output channel
+          if constexpr (kTF32) {
+            // fp32 rows: channel d and d + 1 (each checked: Do may be odd), 16 bytes each
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+              for (int rr = 0; rr < 2; ++rr) {
+                const int64_t row = row0 + 16 * hf + 8 * rr;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                  const int i = 2 * rr + cc;
+                  const float Y0 = __uint_as_float(y0[hf][i]), Y2 = __uint_as_float(y2[hf][i]);
+                  const float Yr = __uint_as_float(yr[hf][i]), Yi = __uint_as_float(yi[hf][i]);
+                  const float bv = d + cc < p.Do ? sbias[d + cc] : 0.f;
+                  const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
+                  if (row < p.N && d + cc < p.Do)
+                    *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + row * row_elems +
+                                                static_cast<int64_t>(d + cc) * kT) =
+                        make_float4(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o), fmaf(-0.5f, Yr, e),
+                                    fmaf(0.5f, Yi, o));
+                }
+              }
+            }
+            continue;
+          }
           if (d + 2 > p.Do) continue;        // Do is even: the pair is whole or padding
           const float b0 = sbias[d], b1 = sbias[d + 1];
 #pragma unroll
@@ -388,7 +473,8 @@ tc_fourier_gemm_kernel(const __grid_constant__ CUtensorMap tm_in, const TcFwdPar
               }
               const int64_t row = row0 + 16 * hf + 8 * rr;
               if (row < p.N)
-                *reinterpret_cast<uint4 *>(p.out + row * row_elems + static_cast<int64_t>(d) * kT) =
+                *reinterpret_cast<uint4 *>(static_cast<__half *>(p.out) + row * row_elems +
+                                           static_cast<int64_t>(d) * kT) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
           }

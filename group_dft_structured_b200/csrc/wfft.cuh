@@ -10,6 +10,7 @@
 #include <cuda_fp16.h>
 
 #include "plan.cuh"
+#include "sm100.cuh"
 
 namespace feql {
 
@@ -68,6 +69,44 @@ __global__ void wfft_tc_kernel(const __half *__restrict__ W, uint8_t *__restrict
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(0.25f * v);
+  }
+}
+
+// Split-TF32 layout: per (tile, chunk of 8 input channels) the hi tile (the
+// bins rounded to tf32) then the lo tile (the remainders rounded to tf32),
+// each 5*BD rows of 8 words with the 32-byte swizzle.  One thread per word.
+__global__ void wfft_tf32_kernel(const float *__restrict__ W, uint8_t *__restrict__ What,
+                                 WhatLayout L, int C) {
+  const int64_t n_fwd = L.fwd.bytes / 4, n_dx = L.dx.bytes / 4;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n_fwd + n_dx;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int dir = e < n_fwd ? 0 : 1;
+    const TcPlan &P = dir == 0 ? L.fwd : L.dx;
+    const int64_t le = dir == 0 ? e : e - n_fwd;
+    const int rows = 5 * P.BD;
+    const int64_t chunk = le / (2 * rows * kCK32);
+    const int rem = static_cast<int>(le % (2 * rows * kCK32));
+    const int half = rem / (rows * kCK32);  // 0: hi tile, 1: lo tile
+    const int row = (rem % (rows * kCK32)) / kCK32, k = rem % kCK32;
+    const int j = static_cast<int>(chunk / P.nK), kc = static_cast<int>(chunk % P.nK);
+    const int sub = row / P.BD;
+    const int o = j * P.BD + row % P.BD;
+    const int i = kc * kCK32 + k;
+    float v = 0.f;
+    if (o < P.Do && i < P.Ci) {
+      float b0, b2, b1r, b1i;
+      weight_bins(W, C, dir, o, i, b0, b2, b1r, b1i);
+      if (sub == 0) v = b0;
+      else if (sub == 1) v = b2;
+      else if (sub == 2) v = b1r;
+      else if (sub == 3) v = b1i;
+      else v = -b1r;
+    }
+    const uint32_t hi = tf32_rna(v);
+    const uint32_t word = half == 0 ? hi : tf32_rna(v - __uint_as_float(hi));
+    const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes +
+                         half * (rows * 32);
+    *reinterpret_cast<uint32_t *>(What + base + sw32_offset4(row, k)) = word;
   }
 }
 

@@ -57,9 +57,14 @@ typedef struct CUstream_st *feql_stream;
 /* Arithmetic mode. */
 typedef enum {
   FEQL_FP16 = 0,        /* fp16 data, fp32 accumulate, tcgen05 tensor cores */
-  FEQL_FP32 = 1,        /* fp32 data; the library picks FEQL_FP32_SIMT or FEQL_FP32_3XTF32 */
+  FEQL_FP32 = 1,        /* fp32 data; the p4 layer takes FEQL_FP32_3XTF32 when C, D <= 512,
+                           else FEQL_FP32_SIMT (every other entry point: FEQL_FP32_SIMT) */
   FEQL_FP32_SIMT = 2,   /* fp32 data, fp32 FMA on CUDA cores */
-  FEQL_FP32_3XTF32 = 3, /* fp32 data, split-TF32 (hi*hi + hi*lo + lo*hi) on tensor cores */
+  FEQL_FP32_3XTF32 = 3, /* fp32 data, split TF32 on the tensor cores: each operand is its
+                           tf32 rounding (hi) plus the rounded remainder (lo), three tf32
+                           products hi*hi + hi*lo + lo*hi per product (Ootomo and Yokota),
+                           fp32 accumulation; forward and dX of the p4 layer (dW and db run
+                           on the fp32 CUDA-core kernels) */
   FEQL_FP16_SIMT = 4    /* fp16 data, fp32 FMA on CUDA cores (cross-check path) */
 } feql_dtype;
 

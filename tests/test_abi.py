@@ -69,15 +69,30 @@ def _tc_plan(Ci, Do):
     return nD, BD, nK, nD * nK * 5 * BD * 16 * 2
 
 
-@pytest.mark.parametrize("C,D", [(16, 16), (48, 192), (192, 192), (256, 256), (24, 96), (6, 40)])
+def _tf32_plan(Ci, Do):
+    """Split-TF32 direction: chunks of 8 channels, the fp16 tiling of outputs
+    (BD <= 64 when the contraction is at most 64 channels), hi and lo tiles."""
+    nK = -(-Ci // 8)
+    nD = -(-Do // (64 if Ci <= 64 else 128))
+    BD = -(-(-(-Do // nD)) // 16) * 16
+    return nD, BD, nK, nD * nK * 2 * 5 * BD * 32
+
+
+@pytest.mark.parametrize("C,D", [(16, 16), (48, 192), (192, 192), (256, 256), (24, 96), (6, 40),
+                                 (3, 5), (600, 16)])
 def test_weight_buffer_sizes(lib, C, D):
     def al(v):
         return -(-v // 1024) * 1024
     tc = al(_tc_plan(C, D)[3]) + al(_tc_plan(D, C)[3])
-    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16) == tc
-    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32_SIMT) == 2 * 4 * C * D * 4
-    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32) == 2 * 4 * C * D * 4
-    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16_SIMT) == 2 * 4 * C * D * 4
+    tf32 = al(_tf32_plan(C, D)[3]) + al(_tf32_plan(D, C)[3])
+    simt = 2 * 4 * C * D * 4
+    if ((C | D) & 1) == 0:
+        assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16) == tc
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32_SIMT) == simt
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32_3XTF32) == tf32
+    # FEQL_FP32 is split TF32 up to 512 channels on either side, CUDA cores beyond
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP32) == (tf32 if max(C, D) <= 512 else simt)
+    assert F.feql_weight_fft_bytes(C, D, F.FEQL_FP16_SIMT) == simt
     assert F.feql_weight_fft_bytes(0, D, F.FEQL_FP16) == 0
 
 

@@ -17,9 +17,10 @@ from oracle import feql_oracle as O
 
 pytestmark = pytest.mark.gpu
 
-TOL = {F.FEQL_FP16: 5e-3, F.FEQL_FP16_SIMT: 5e-3, F.FEQL_FP32: 1e-5, F.FEQL_FP32_SIMT: 1e-5}
+TOL = {F.FEQL_FP16: 5e-3, F.FEQL_FP16_SIMT: 5e-3, F.FEQL_FP32: 1e-5, F.FEQL_FP32_SIMT: 1e-5,
+       F.FEQL_FP32_3XTF32: 1e-5}
 NAME = {F.FEQL_FP16: "fp16", F.FEQL_FP16_SIMT: "fp16", F.FEQL_FP32: "fp32",
-        F.FEQL_FP32_SIMT: "fp32"}
+        F.FEQL_FP32_SIMT: "fp32", F.FEQL_FP32_3XTF32: "fp32"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -76,7 +77,8 @@ SMALL = [(300, 16, 16), (1000, 48, 192), (517, 24, 96), (260, 192, 192), (257, 2
          (1, 24, 96), (129, 6, 40), (384, 2, 2), (128, 34, 130)]
 
 
-@pytest.mark.parametrize("mode", [F.FEQL_FP16, F.FEQL_FP16_SIMT, F.FEQL_FP32_SIMT])
+@pytest.mark.parametrize("mode", [F.FEQL_FP16, F.FEQL_FP16_SIMT, F.FEQL_FP32_SIMT,
+                                  F.FEQL_FP32_3XTF32])
 @pytest.mark.parametrize("N,C,D", SMALL)
 def test_small_shapes_all_passes(mode, N, C, D):
     inp = make_inputs(9, N, C, D, NAME[mode])
@@ -89,10 +91,19 @@ def test_forward_without_bias(mode):
     check(run_all(inp, mode, passes=("fwd",), with_bias=False), inp, mode, with_bias=False)
 
 
-@pytest.mark.parametrize("C,D", [(3, 5), (17, 9)])
-def test_fp32_odd_channels(C, D):
+@pytest.mark.parametrize("mode", [F.FEQL_FP32, F.FEQL_FP32_3XTF32])
+@pytest.mark.parametrize("C,D", [(3, 5), (17, 9), (1, 1), (33, 130)])
+def test_fp32_odd_channels(mode, C, D):
     inp = make_inputs(7, 200, C, D, "fp32")
-    check(run_all(inp, F.FEQL_FP32), inp, F.FEQL_FP32)
+    check(run_all(inp, mode), inp, mode)
+
+
+def test_split_tf32_deep_contraction():
+    """Split TF32 keeps the fp32 bound over a 512-channel contraction per bin (the
+    unrolled layer is 2048 deep), where a single tf32 product (about 2^-11
+    relative) would miss it by an order of magnitude."""
+    inp = make_inputs(17, 640, 512, 64, "fp32")
+    check(run_all(inp, F.FEQL_FP32_3XTF32, passes=("fwd", "dx")), inp, F.FEQL_FP32_3XTF32)
 
 
 def test_zero_tokens_is_a_noop_and_zeroes_dw():
@@ -207,7 +218,8 @@ def test_fused_backward_is_deterministic_and_stays_in_bounds():
 # ---------------------------------------------------------------- full sizes
 
 @pytest.mark.parametrize("wid,mode", [(1, F.FEQL_FP32), (2, F.FEQL_FP16), (3, F.FEQL_FP16),
-                                      (3, F.FEQL_FP32), (4, F.FEQL_FP16), (5, F.FEQL_FP16)])
+                                      (3, F.FEQL_FP32), (4, F.FEQL_FP16), (5, F.FEQL_FP16),
+                                      (1, F.FEQL_FP32_3XTF32), (3, F.FEQL_FP32_3XTF32)])
 def test_workload_full_size(wid, mode):
     w = WORKLOADS[wid]
     inp = workload_inputs(wid, dtype=NAME[mode])
