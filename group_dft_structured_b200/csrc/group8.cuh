@@ -104,15 +104,22 @@ struct Cyclic8 {
     o[7] = g - b2;
   }
 
-  // The same for two channels at once on packed fp16 pairs: v[t] = (channel q,
-  // channel q+1) at group element t; o[p] packs plane p (three to four
-  // roundings per output).
+  // The same for two channels at once on packed fp16 pairs, every plane divided
+  // by 8: v[t] = (channel q, channel q+1) at group element t; o[p] packs plane
+  // p / 8 (three to four roundings per output).  Bin 0 sums eight values, so
+  // the unscaled planes of inputs above 65504 / 8 would overflow fp16; the
+  // first butterfly stage takes the 1/8 (exact outside the subnormals).
   __device__ static void planes_h2(const __half2 (&v)[8], __half2 (&o)[8]) {
-    const __half2 c = __float2half2_rn(kC8);
-    const __half2 a0 = __hadd2(v[0], v[4]), a1 = __hadd2(v[1], v[5]);
-    const __half2 a2 = __hadd2(v[2], v[6]), a3 = __hadd2(v[3], v[7]);
-    const __half2 b0 = __hsub2(v[0], v[4]), b1 = __hsub2(v[1], v[5]);
-    const __half2 b2 = __hsub2(v[2], v[6]), b3 = __hsub2(v[3], v[7]);
+    const __half2 c = __float2half2_rn(kC8), q = __float2half2_rn(0.125f);
+    __half2 a[4], b[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __half2 u = __hmul2(v[t + 4], q);
+      a[t] = __hfma2(v[t], q, u);
+      b[t] = __hfma2(v[t], q, __hneg2(u));
+    }
+    const __half2 a0 = a[0], a1 = a[1], a2 = a[2], a3 = a[3];
+    const __half2 b0 = b[0], b1 = b[1], b2 = b[2], b3 = b[3];
     const __half2 e02 = __hadd2(a0, a2), e13 = __hadd2(a1, a3);
     const __half2 h = __hmul2(c, __hsub2(b1, b3)), g = __hmul2(c, __hadd2(b1, b3));
     o[0] = __hadd2(e02, e13);
@@ -125,19 +132,21 @@ struct Cyclic8 {
     o[7] = __hsub2(g, b2);
   }
 
-  // Group values from the accumulator blocks Y0, Y4, Re Y1, Im Y1, ..., Im Y3.
-  __device__ static void inverse(const float (&F)[8], float (&y)[8]) {
+  // Group values, times s, from the accumulator blocks Y0, Y4, Re Y1, Im Y1,
+  // ..., Im Y3 (s undoes the scale of the fp16 planes and weights).
+  __device__ static void inverse(const float (&F)[8], float (&y)[8], float s) {
     const float r1 = F[2], i1 = F[3], r2 = F[4], i2 = F[5], r3 = F[6], i3 = F[7];
-    const float P = 0.125f * (F[0] + F[1]), Q = 0.125f * (F[0] - F[1]);
+    const float e = 0.125f * s, h = 0.25f * s;
+    const float P = e * (F[0] + F[1]), Q = e * (F[0] - F[1]);
     const float u = kC8 * (r1 - r3), w = kC8 * (i1 + i3);  // the +-c terms of bins 1 and 3
-    y[0] = P + 0.25f * (r1 + r2 + r3);
-    y[1] = Q + 0.25f * (u - w - i2);
-    y[2] = P + 0.25f * (i3 - i1 - r2);
-    y[3] = Q + 0.25f * (i2 - u - w);
-    y[4] = P + 0.25f * (r2 - r1 - r3);
-    y[5] = Q + 0.25f * (w - u - i2);
-    y[6] = P + 0.25f * (i1 - r2 - i3);
-    y[7] = Q + 0.25f * (u + w + i2);
+    y[0] = P + h * (r1 + r2 + r3);
+    y[1] = Q + h * (u - w - i2);
+    y[2] = P + h * (i3 - i1 - r2);
+    y[3] = Q + h * (i2 - u - w);
+    y[4] = P + h * (r2 - r1 - r3);
+    y[5] = Q + h * (w - u - i2);
+    y[6] = P + h * (i1 - r2 - i3);
+    y[7] = Q + h * (u + w + i2);
   }
 
   // Weight rows of one fibre W[d][c][0..7] for pass direction dir (0: forward,
@@ -219,11 +228,15 @@ struct Dihedral4 {
     o[7] = Ca - Cb;  // E11
   }
 
+  // Packed fp16 pairs, every plane divided by 8 in the first stage (as for C8).
   __device__ static void planes_h2(const __half2 (&v)[8], __half2 (&o)[8]) {
-    const __half2 Pa = __hadd2(v[0], v[2]), Qa = __hadd2(v[1], v[3]);
-    const __half2 Ca = __hsub2(v[0], v[2]), Sa = __hsub2(v[1], v[3]);
-    const __half2 Pb = __hadd2(v[4], v[6]), Qb = __hadd2(v[5], v[7]);
-    const __half2 Cb = __hsub2(v[4], v[6]), Sb = __hsub2(v[5], v[7]);
+    const __half2 q = __float2half2_rn(0.125f);
+    const __half2 u2 = __hmul2(v[2], q), u3 = __hmul2(v[3], q);
+    const __half2 u6 = __hmul2(v[6], q), u7 = __hmul2(v[7], q);
+    const __half2 Pa = __hfma2(v[0], q, u2), Qa = __hfma2(v[1], q, u3);
+    const __half2 Ca = __hfma2(v[0], q, __hneg2(u2)), Sa = __hfma2(v[1], q, __hneg2(u3));
+    const __half2 Pb = __hfma2(v[4], q, u6), Qb = __hfma2(v[5], q, u7);
+    const __half2 Cb = __hfma2(v[4], q, __hneg2(u6)), Sb = __hfma2(v[5], q, __hneg2(u7));
     const __half2 sa = __hadd2(Pa, Qa), da = __hsub2(Pa, Qa);
     const __half2 sb = __hadd2(Pb, Qb), db = __hsub2(Pb, Qb);
     o[0] = __hadd2(sa, sb);
@@ -239,12 +252,14 @@ struct Dihedral4 {
   // x(r, 0) = (A1 + A2 + (-1)^r (B1 + B2)) / 8 + (c_r (E00 + E11) + s_r (E10 - E01)) / 4
   // x(r, 1) = (A1 - A2 + (-1)^r (B1 - B2)) / 8 + (c_r (E00 - E11) + s_r (E01 + E10)) / 4
   // with (c_r, s_r) = (1, 0), (0, 1), (-1, 0), (0, -1).
-  __device__ static void inverse(const float (&F)[8], float (&y)[8]) {
+  // (times s, as for C8)
+  __device__ static void inverse(const float (&F)[8], float (&y)[8], float s) {
     const float s12 = F[0] + F[1], d12 = F[0] - F[1], s34 = F[2] + F[3], d34 = F[2] - F[3];
-    const float Pp = 0.125f * (s12 + s34), Pm = 0.125f * (s12 - s34);
-    const float Qp = 0.125f * (d12 + d34), Qm = 0.125f * (d12 - d34);
-    const float c0 = 0.25f * (F[4] + F[7]), s0 = 0.25f * (F[6] - F[5]);
-    const float c1 = 0.25f * (F[4] - F[7]), s1 = 0.25f * (F[5] + F[6]);
+    const float e = 0.125f * s, h = 0.25f * s;
+    const float Pp = e * (s12 + s34), Pm = e * (s12 - s34);
+    const float Qp = e * (d12 + d34), Qm = e * (d12 - d34);
+    const float c0 = h * (F[4] + F[7]), s0 = h * (F[6] - F[5]);
+    const float c1 = h * (F[4] - F[7]), s1 = h * (F[5] + F[6]);
     y[0] = Pp + c0;
     y[1] = Pm + s0;
     y[2] = Pp - c0;
@@ -368,7 +383,8 @@ __global__ void wfft_g8_kernel(const __half *__restrict__ W, uint8_t *__restrict
         if (r == sub) v = wr[r];
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
-    *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);
+    // every weight plane divided by 8 (as the operand planes): no fp16 overflow for any finite W
+    *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(0.125f * v);
   }
 }
 
@@ -618,7 +634,7 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
           float F[8], y[8];
 #pragma unroll
           for (int bk = 0; bk < 8; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
-          Gp::inverse(F, y);
+          Gp::inverse(F, y, 64.f);  // planes and weights both carry 1/8
           const float bv = sbias[d0 + i];
           *reinterpret_cast<uint4 *>(ob + lane * 128 + ((i ^ (lane & 7)) << 4)) =
               make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
@@ -649,7 +665,8 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
 // dW / db kernel
 // ---------------------------------------------------------------------------
 // G_k[d,c] = sum_n dY_k[n,d] conj(X_k[n,c]) for bins k = 0..4, dW = irDFT_8(G)
-// (cross-correlation theorem; the same inverse as the forward), db = sum dY_0.
+// (cross-correlation theorem; the same inverse as the forward), db = sum dY_0
+// (from the fp16 bin-0 planes, which carry dY_0 / 8).
 // One CTA per (128-row d tile, c tile of CT <= 32 columns, token split),
 // 10 warps: TMA, MMA, 8 transform warps that also read the accumulators at the
 // end.  Per chunk of 32 tokens the TMA warp loads the tile's dy boxes into box
@@ -819,6 +836,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
   } else {
     // ---------------------------------------------------------- transform
     const int t = threadIdx.x - 64;
+    const bool do_db = tj == 0;  // the tiles of the first c column produce db
     float db_acc[kG8DwMaxPer][8];
 #pragma unroll
     for (int k = 0; k < kG8DwMaxPer; ++k)
@@ -843,7 +861,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
             const uint4 r1 = *reinterpret_cast<const uint4 *>(src + (((q + 1) ^ (r & 7)) << 4));
             uint32_t o[8];
             g8_planes_pair<Gp>(r0, r1, o);
-            if (bi < nqd) {
+            if (do_db && bi < nqd) {  // bin 0 of the dy planes, as the MMAs see it
               const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&o[0]));
               db_acc[k][q] += f.x;
               db_acc[k][q + 1] += f.y;
@@ -912,7 +930,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
     }
     tc_fence_before();
     // db (tiles of the first c column only): fixed-order reduction through shared memory
-    if (tj == 0) {
+    if (do_db) {
       named_bar_sync(3, 256);  // the stages are free: every chunk has been consumed
       float *sdb = reinterpret_cast<float *>(smem + L.stage0);  // [kG8DwMaxPer * 256][8]
 #pragma unroll
@@ -979,7 +997,7 @@ g8_dw_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
 #pragma unroll
         for (int k = 0; k < kT8; ++k) t[k] += part[q][k][lo];
       float y[kT8];
-      Gp::inverse(t, y);
+      Gp::inverse(t, y, 64.f);  // x and dy planes both carry 1/8
       *reinterpret_cast<uint4 *>(dW + e * kT8) =
           make_uint4(pack_half2(y[0], y[1]), pack_half2(y[2], y[3]), pack_half2(y[4], y[5]),
                      pack_half2(y[6], y[7]));
@@ -994,7 +1012,7 @@ g8_dw_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_d
     if (grp == 0 && d < D) {
       float t = 0.f;
       for (int q = 0; q < kRed8Groups; ++q) t += part[q][0][lo];
-      db[d] = __float2half_rn(t);
+      db[d] = __float2half_rn(8.f * t);  // bin 0 of the dy planes carries 1/8
     }
   }
 }

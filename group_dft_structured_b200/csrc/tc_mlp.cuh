@@ -93,9 +93,11 @@ __host__ __device__ inline MlpPlan make_mlp_plan(int C, int H, int Co, int hs_ma
 }
 
 // Weight transform of both layers: one thread per fp16 element of the buffer.
-// fc1's bins carry the inverse transform's scales and the 1/2 of GELU: bins 0
-// and 2 are stored times 1/8, bin 1 times 1/4 (powers of two: exact), so its
-// accumulators give u_t = h_t / 2 with sums and differences alone.
+// fc1's bins carry the inverse transform's scales: bins 0 and 2 are stored
+// times 1/8, bin 1 times 1/4 (powers of two: exact); with x's planes divided by
+// 4 its accumulators give v_t = h_t / 8 with sums and differences alone.  fc2's
+// bins are divided by 4, like the hidden planes (GELU / 4) they multiply, so no
+// fp16 plane overflows for any finite x, W1, W2 or hidden activation.
 __global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__restrict__ W2,
                                 uint8_t *__restrict__ What, MlpPlan P) {
   const int64_t n1 = P.w1_bytes / 2, n2 = P.w2_bytes / 2;
@@ -126,7 +128,7 @@ __global__ void wfft_mlp_kernel(const __half *__restrict__ W1, const __half *__r
       float b0, b2, b1r, b1i;
       weight_bins(first ? W1 : W2, Ci, 0, o, i, b0, b2, b1r, b1i);
       v = sub == 0 ? b0 : sub == 1 ? b2 : sub == 2 ? b1r : sub == 3 ? b1i : -b1r;
-      if (first) v *= sub < 2 ? 0.125f : 0.25f;
+      v *= first ? (sub < 2 ? 0.125f : 0.25f) : 0.25f;
     }
     const int64_t base = first ? chunk * P.w1_chunk : P.off_w2 + chunk * P.w2_chunk;
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(v);
@@ -190,14 +192,17 @@ __device__ __forceinline__ uint32_t tanh_h2(uint32_t x) {
   return y;
 }
 
-// GELU (tanh form) of z = 2u for a packed fp16 pair u:
-//   GELU(2u) = u (1 + tanh(2 k0 u + 8 k1 u^3)),  k0 = sqrt(2/pi), k1 = 0.044715 k0.
-__device__ __forceinline__ uint32_t gelu_half_arg_h2(uint32_t uu) {
-  const __half2 u = as_h2(uu);
-  const __half2 c0 = __float2half2_rn(1.5957691216057308f);  // 2 sqrt(2/pi)
-  const __half2 c1 = __float2half2_rn(0.2854192650904008f);  // 8 * 0.044715 sqrt(2/pi)
-  const __half2 t = as_h2(tanh_h2(as_u32(__hmul2(u, __hfma2(c1, __hmul2(u, u), c0)))));
-  return as_u32(__hfma2(u, t, u));
+// A quarter of the GELU (tanh form) of z = 8v for a packed fp16 pair v:
+//   GELU(8v) / 4 = v (1 + tanh(8 k0 v + 512 k1 v^3)),  k0 = sqrt(2/pi), k1 = 0.044715 k0.
+// (z / 8 and GELU / 4 keep the fp16 operand planes around it in range; the
+// powers of two leave the rounding of every step as for z itself.  Where v^2
+// overflows, the tanh argument is +-inf and the result v (1 +- 1) is exact.)
+__device__ __forceinline__ uint32_t gelu_eighth_arg_h2(uint32_t vv) {
+  const __half2 v = as_h2(vv);
+  const __half2 c0 = __float2half2_rn(6.3830764864229232f);  // 8 sqrt(2/pi)
+  const __half2 c1 = __float2half2_rn(18.266832965785664f);  // 512 * 0.044715 sqrt(2/pi)
+  const __half2 t = as_h2(tanh_h2(as_u32(__hmul2(v, __hfma2(c1, __hmul2(v, v), c0)))));
+  return as_u32(__hfma2(v, t, v));
 }
 
 // 22 warps: six on the busiest 16K-register sub-partition, 80 registers each.
@@ -247,10 +252,10 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
     }
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < nS * hs / 2; i += blockDim.x) {  // b1 / 2, like fc1's accumulators
+  for (int i = threadIdx.x; i < nS * hs / 2; i += blockDim.x) {  // b1 / 8, like fc1's accumulators
     const int j = 2 * i;
-    const float v0 = (p.b1 != nullptr && j < P.H) ? 0.5f * __half2float(p.b1[j]) : 0.f;
-    const float v1 = (p.b1 != nullptr && j + 1 < P.H) ? 0.5f * __half2float(p.b1[j + 1]) : 0.f;
+    const float v0 = (p.b1 != nullptr && j < P.H) ? 0.125f * __half2float(p.b1[j]) : 0.f;
+    const float v1 = (p.b1 != nullptr && j + 1 < P.H) ? 0.125f * __half2float(p.b1[j + 1]) : 0.f;
     sb1[i] = pack_half2(v0, v1);
   }
   for (int i = threadIdx.x; i < P.BD2; i += blockDim.x)
@@ -428,7 +433,7 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
           raw[q] = *reinterpret_cast<const uint4 *>(st + r * 128 + ((q ^ (r & 7)) << 4));
         uint32_t pl[4][8];  // [plane][channel pair]: V0, V2, Re V1, -Im V1
 #pragma unroll
-        for (int q = 0; q < 8; ++q) rdft4_pair(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
+        for (int q = 0; q < 8; ++q) rdft4_pair_q(raw[q], pl[0][q], pl[1][q], pl[2][q], pl[3][q]);
         named_bar_sync(2, 128);  // every row read before the planes overwrite it
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
@@ -487,10 +492,11 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(&a1empty[b]);
           }
-          // Per channel pair (c, c+1), packed as fp16 pairs: half the group
-          // values u_t = h_t / 2 (inverse rDFT + b1 / 2, the scales folded into
-          // the weights), GELU, and the rDFT of the activations, whose four bins
-          // are fc2's operand planes (channel pairs are the planes' word layout).
+          // Per channel pair (c, c+1), packed as fp16 pairs: an eighth of the
+          // group values, v_t = h_t / 8 (inverse rDFT + b1 / 8, the scales
+          // folded into the weights and x's planes), GELU / 4, and the rDFT of
+          // those, whose four bins are fc2's operand planes (a quarter of the
+          // activations' bins; channel pairs are the planes' word layout).
           uint32_t pl[4][4];
 #pragma unroll
           for (int i2 = 0; i2 < 4; ++i2) {
@@ -500,10 +506,10 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             const __half2 ai = as_h2(pack_half2(__uint_as_float(yi[2 * i2]), __uint_as_float(yi[2 * i2 + 1])));
             const __half2 pb = __hadd2(a0, as_h2(bias[c8 * 4 + i2]));
             const __half2 e = __hadd2(pb, a2), o = __hsub2(pb, a2);
-            const __half2 g0 = as_h2(gelu_half_arg_h2(as_u32(__hadd2(e, ar))));
-            const __half2 g1 = as_h2(gelu_half_arg_h2(as_u32(__hsub2(o, ai))));
-            const __half2 g2 = as_h2(gelu_half_arg_h2(as_u32(__hsub2(e, ar))));
-            const __half2 g3 = as_h2(gelu_half_arg_h2(as_u32(__hadd2(o, ai))));
+            const __half2 g0 = as_h2(gelu_eighth_arg_h2(as_u32(__hadd2(e, ar))));
+            const __half2 g1 = as_h2(gelu_eighth_arg_h2(as_u32(__hsub2(o, ai))));
+            const __half2 g2 = as_h2(gelu_eighth_arg_h2(as_u32(__hsub2(e, ar))));
+            const __half2 g3 = as_h2(gelu_eighth_arg_h2(as_u32(__hadd2(o, ai))));
             const __half2 s02 = __hadd2(g0, g2), s13 = __hadd2(g1, g3);
             pl[0][i2] = as_u32(__hadd2(s02, s13));   // V0
             pl[1][i2] = as_u32(__hsub2(s02, s13));   // V2
@@ -557,9 +563,10 @@ tc_mlp_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__
             const float Y0 = __uint_as_float(y0[i]), Y2 = __uint_as_float(y2[i]);
             const float Yr = __uint_as_float(yr[i]), Yi = __uint_as_float(yi[i]);
             const float bv = sb2[d0 + h * 8 + i];
-            const float e = fmaf(0.25f, Y0 + Y2, bv), o = fmaf(0.25f, Y0 - Y2, bv);
-            packed[16 * h + 2 * i] = pack_half2(fmaf(0.5f, Yr, e), fmaf(-0.5f, Yi, o));
-            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-0.5f, Yr, e), fmaf(0.5f, Yi, o));
+            // the planes and fc2's weights each carry 1/4: the inverse's 1/4 and 1/2 times 16
+            const float e = fmaf(4.f, Y0 + Y2, bv), o = fmaf(4.f, Y0 - Y2, bv);
+            packed[16 * h + 2 * i] = pack_half2(fmaf(8.f, Yr, e), fmaf(-8.f, Yi, o));
+            packed[16 * h + 2 * i + 1] = pack_half2(fmaf(-8.f, Yr, e), fmaf(8.f, Yi, o));
           }
         }
         if (d0 >= P.Co) continue;  // whole group is padding

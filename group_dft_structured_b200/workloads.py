@@ -131,6 +131,29 @@ def make_mlp_inputs(wid: int, N: int, C: int, H: int, Co: int, dtype: str) -> di
             "b2": _normal(base + 5, (Co,), 0.02, dtype)}
 
 
+def make_mlp_range_inputs(wid: int, N: int, C: int, H: int, Co: int, x, W1, W2,
+                          b1_std: float = 0.02, b2_std: float = 0.02) -> dict:
+    """fp16 inputs of the MLP block at the edges of the half-precision range.
+
+    Each of x, W1, W2 is given either as a float s (normal values, N(0, s^2))
+    or as a pair (lo, hi) (magnitudes uniform in [lo, hi] with random signs);
+    b1 ~ N(0, b1_std^2), b2 ~ N(0, b2_std^2).
+    Seeds: 20260000 + 100 * wid + {x: 0, W1: 1, b1: 2, W2: 4, b2: 5}.
+    """
+    base = 20260000 + 100 * wid
+
+    def draw(seed, shape, spec):
+        if isinstance(spec, tuple):
+            return _magnitude(seed, shape, spec[0], spec[1], "fp16")
+        return _normal(seed, shape, spec, "fp16")
+
+    return {"x": draw(base + 0, (N, C, 4), x),
+            "W1": draw(base + 1, (H, C, 4), W1),
+            "b1": _normal(base + 2, (H,), b1_std, "fp16"),
+            "W2": draw(base + 4, (Co, H, 4), W2),
+            "b2": _normal(base + 5, (Co,), b2_std, "fp16")}
+
+
 def _magnitude(seed: int, shape, lo: float, hi: float, dtype: str) -> np.ndarray:
     """Values with |v| uniform in [lo, hi] and a random sign (seeded)."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -139,6 +139,49 @@ def test_fused_backward_with_large_inputs(large, N, C, D):
         assert O.rel_err(host(db), ref_db) <= TOL
 
 
+# signs along the group axis: the first-stage pairs (0, 2) and (1, 3) add equal
+# signs, so both double |dy|, while bin 0 (their sum) nearly cancels
+PATTERN = np.array([1, -1, 1, -1], dtype=np.float64)
+U16 = 2.0 ** -11  # unit roundoff of fp16
+
+
+def db_plane_bound(dy, ref_db):
+    """Error bound of db taken from the fp16 bin-0 planes: the two butterfly
+    stages round once each (unit roundoff u) at magnitudes of at most
+    sum_t |dy[n, d, t]| / 4, the 1/4 is exact and the fp32 sums add O(u^2), so
+    |db - ref| <= 2 u sum_n sum_t |dy[n, d, t]| + u |ref| (the final fp16 rounding)."""
+    return 2 * U16 * np.abs(dy).sum(axis=(0, 2)) + U16 * np.abs(ref_db) + 1e-6
+
+
+@pytest.mark.parametrize("N,C,D", [(16, 24, 96), (48, 256, 256)])
+def test_db_with_large_cancelling_dy(N, C, D):
+    """|dy| in [3.4e4, 3.6e4] with the sign pattern above: the unscaled
+    first-stage sums would overflow, yet dW (for small x) and db are ordinary
+    fp16 numbers.  dx and dW meet the parity bound; db, whose fibre sums cancel
+    to a few percent of sum |dy|, meets the bound of the fp16 bin-0 planes it
+    is computed from (db_plane_bound), in the separate and the fused backward."""
+    inp = make_range_inputs(49, N, C, D, (5e-3, 1.5e-2), (3.4e4, 3.6e4), 0.5 / np.sqrt(4 * D * 16))
+    dy = inp["dy"].astype(np.float64)
+    sign = np.sign(dy[..., :1])  # one random sign per (token, output channel)
+    inp["dy"] = (sign * PATTERN * np.abs(dy)).astype(np.float16)
+    assert overflows_unscaled(inp["dy"])
+    r = f64(inp)
+    ref_dx = O.backward_dx(r["dy"], r["W"])
+    ref_dW, ref_db = O.backward_dw(r["x"], r["dy"])
+    assert np.abs(ref_db).max() < FP16_MAX / 2 and np.abs(ref_dW).max() < FP16_MAX / 2
+    assert np.abs(ref_dx).max() < FP16_MAX / 2
+    What = Lyr.weight_fft(dev(inp["W"]), MODE)
+    bound = db_plane_bound(r["dy"], ref_db)
+    for dx, dW, db in ((None,) + Lyr.backward_dw(dev(inp["x"]), dev(inp["dy"]), MODE),
+                       Lyr.backward(dev(inp["x"]), dev(inp["dy"]), What, MODE)):
+        assert F.feql_device_status() == F.FEQL_OK
+        if dx is not None:
+            assert O.rel_err(host(dx), ref_dx) <= TOL
+        assert O.rel_err(host(dW), ref_dW) <= TOL
+        err = np.abs(host(db) - ref_db)
+        assert np.all(err <= bound), err.max()
+
+
 def test_large_weights():
     """Weights up to 3e4 (bin 0 of a fibre then exceeds the fp16 range) with small x."""
     N, C, D = 300, 24, 96
