@@ -10,8 +10,9 @@ resident in HBM; each pass reads/writes ~385 MB, more than the 126 MB L2, so
 no flush is needed between steps.  The same line carries "per_config": every
 layer configuration (1: fp32 256x16x16, 2: ViT fc1 12608x48x192, 3: square
 65536x192x192 in fp16 and fp32, 4: backward 32768x256x256, 5: the Swin stream)
-at full size, each pass timed over 50 reps with the L2 flushed before each,
-median and min, with its roofline fractions.
+and the widened workloads (C_8, p4m, C_6, the two MLP blocks) at full size,
+each pass timed over 50 reps with the L2 flushed before each, median and min,
+with its roofline fractions.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -593,6 +594,84 @@ def per_config_report(F, torch, stream, reps):
             entry["tokens_per_s_fused_backward"] = round(N / ((t["fwd"] + t["bwd"]) * 1e-6), 1)
         out[key] = entry
         del B, x, W, b, dy, y, dx, dW, db, ws, What, calls
+        torch.cuda.empty_cache()
+    out.update(widening_report(F, torch, stream, reps, meas, nom, flush))
+    return out
+
+
+# The widened rows at full size: the C_8 and p4m layers and the two MLP blocks
+# on the tensor cores, C_6 on the CUDA cores (fp32 arithmetic on fp16 data).
+WIDENING_RUNS = (6, 8, 10, 7, 9)
+# Nominal special-function throughput: 16 MUFU operations per SM per clock
+# (four per SM sub-partition), one tanh.approx.f16x2 (two values) per
+# operation, at the maximum SM clock.
+MUFU_OPS_PER_SM_CLK = 16
+SM_CLOCK_GHZ = 1.965
+
+
+def widening_report(F, torch, stream, reps, meas, nom, flush):
+    """The per-config measurement of the widened workloads: each pass over `reps`
+    CUDA-event timings with the L2 flushed before each, median and min, against
+    the slower of its algorithmic bytes at HBM bandwidth and its Fourier-route
+    FLOPs at the arithmetic peak of the units it runs on (tensor cores, or the
+    fp32 FMA pipes for C_6).  The MLP block also gets a special-function floor:
+    its GELU takes one tanh per two hidden values."""
+    import numpy as np
+
+    from group_dft_structured_b200.workloads import WORKLOADS
+    s = stream.cuda_stream
+    args = argparse.Namespace(separate_backward=True)
+    out = {}
+    for wid in WIDENING_RUNS:
+        w = WORKLOADS[wid]
+        mlp = "mlp" in w.passes
+        st = (setup_mlp if mlp else setup_layer)(args, w, 0, s, F, torch)
+        calls, res = st["calls"], {}
+        calls["wfft"]()
+        simt = w.T not in (4, 8)
+        for p in st["passes"]:
+            for _ in range(3):
+                calls[p]()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(reps)]
+            hold_gpu(torch)
+            for a, z in ev:
+                flush.sum()
+                a.record(stream)
+                calls[p]()
+                z.record(stream)
+            torch.cuda.synchronize()
+            us = sorted(a.elapsed_time(z) * 1e3 for a, z in ev)
+            med, mn = float(np.median(us)), us[0]
+            nbytes, (fl, dense_fl) = st["bytes"][p], st["flops"][p]
+            r = {"median_us": round(med, 3), "min_us": round(mn, 3), "reps": reps,
+                 "algorithmic_bytes": nbytes, "GB_s": round(nbytes / (med * 1e-6) / 1e9, 1)}
+            if fl:
+                r["tokens_per_s"] = round(w.N / (med * 1e-6), 1)
+                r["alg_TFLOP_s"] = round(fl / (med * 1e-6) / 1e12, 3)
+                r["dense_equiv_TFLOP_s"] = round(dense_fl / (med * 1e-6) / 1e12, 3)
+                for tag, pk in (("measured", meas), ("nominal", nom)):
+                    if pk is None:
+                        continue
+                    t_roof, bound = roofline_us(nbytes, fl, "fp32" if simt else "fp16", pk)
+                    r[f"roofline_us_{tag}"] = round(t_roof, 3)
+                    r[f"pct_roofline_{tag}"] = round(100 * t_roof / med, 2)
+                    r["bound"] = bound
+                if p == "mlp":
+                    mufu = w.N * 4 * w.D / 2  # tanh.approx.f16x2 per two hidden values
+                    t_xu = mufu / (MUFU_OPS_PER_SM_CLK * torch.cuda.get_device_properties(
+                        0).multi_processor_count * SM_CLOCK_GHZ * 1e9) * 1e6
+                    r["xu_floor_us_nominal"] = round(t_xu, 3)
+                    r["pct_xu_floor"] = round(100 * t_xu / med, 2)
+            res[p] = r
+        if F.feql_device_status(s) != F.FEQL_OK:
+            raise RuntimeError(f"device-side timeout in workload {wid}")
+        out[f"{wid}_{w.dtype}"] = {
+            "workload": w.name, "N": w.N, "C": w.C, "D": w.D, "T": w.T, "group": w.group,
+            "dtype": w.dtype, "units": "CUDA cores (fp32 arithmetic)" if simt else "tensor cores",
+            "l2": f"flushed before every rep (read of a {flush.numel() * 4 >> 20} MiB buffer)",
+            "passes": res}
+        del st, calls
         torch.cuda.empty_cache()
     return out
 
