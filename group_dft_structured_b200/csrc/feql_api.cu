@@ -454,9 +454,19 @@ int launch_g8_fwd(const void *in, const uint8_t *wt, const G8Plan &P, const __ha
   p.stage_bytes = kG8XChunk + static_cast<int>(align_up(p.chunk_bytes, 1024));
   p.bias_floats = p.nD * p.BD;
   const int budget = dev.smem_optin - 1024;
-  p.stages = 6;
-  while (p.stages > 2 && g8_fwd_smem(p).total > budget) --p.stages;
-  if (g8_fwd_smem(p).total > budget) return FEQL_ERR_UNSUPPORTED;
+  // two staging boxes per epilogue warp when a unit has few input chunks (its
+  // time goes to the epilogue) or when they cost no input stage; otherwise one
+  // box if that leaves room for more stages while two would leave fewer than four
+  int fit[3] = {0, 0, 0};
+  for (int nout = 1; nout <= kG8MaxOut; ++nout) {
+    p.nout = nout;
+    p.stages = 6;
+    while (p.stages > 2 && g8_fwd_smem(p).total > budget) --p.stages;
+    fit[nout] = g8_fwd_smem(p).total > budget ? 0 : p.stages;
+  }
+  p.nout = ((p.nK <= 2 && fit[2] >= 3) || fit[2] >= 4 || fit[2] >= fit[1]) ? 2 : 1;
+  p.stages = fit[p.nout];
+  if (p.stages == 0) return FEQL_ERR_UNSUPPORTED;
   CUtensorMap tm, tm_out;
   st = make_tmap_f16(&tm, in, N, static_cast<int64_t>(P.Ci) * kT8, kBM);
   if (st != FEQL_OK) return st;

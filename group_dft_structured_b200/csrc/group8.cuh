@@ -402,16 +402,19 @@ __global__ void wfft_g8_kernel(const __half *__restrict__ W, uint8_t *__restrict
 //   warps 2..9   transform: thread = (token row, box); the 8-point rDFT of its
 //                8 channel fibres on packed fp16 pairs, then, after a team barrier, the
 //                chunk rewritten in place as eight K-major planes of 4 KB
-//   warps 10..13 epilogue: warp q reads TMEM lane quadrant q (32 token rows);
+//   warps 10..17 epilogue, two teams of four taking alternate 8-channel groups
+//                of every unit: warp q reads TMEM lane quadrant q (32 token
+//                rows), four columns of each accumulator block at a time;
 //                inverse rDFT + bias in fp32; per 8 output channels each lane
 //                writes its row (128 B) into a 128-byte-swizzled staging box
 //                and the warp issues one 4 KB TMA store (two boxes per warp)
-constexpr int kG8Threads = 64 + 12 * 32;
+constexpr int kG8EpiWarps = 8;
+constexpr int kG8Threads = 64 + (8 + kG8EpiWarps) * 32;
 constexpr int kG8XChunk = kBM * kCK * kT8 * 2;  // 32 KB: 128 tokens x 16 channels x 8
 constexpr int kG8Box = kG8XChunk / 2;          // 16 KB: 8 channels
 constexpr int kG8Plane = kBM * kCK * 2;         // 4 KB: 128 tokens x 32 B
 constexpr int kG8OutBox = 32 * 128;             // 4 KB: 32 rows x 8 channels x 8
-constexpr int kG8NumOut = 2;                    // staging boxes per epilogue warp
+constexpr int kG8MaxOut = 2;                    // staging boxes per epilogue warp (at most)
 
 struct G8FwdParams {
   const uint8_t *wt;   // weight chunks of this direction, [j][kc]
@@ -422,6 +425,7 @@ struct G8FwdParams {
   int nM, n_units;
   int nacc, acc_stride;
   int stages, stage_bytes, bias_floats;
+  int nout;            // staging boxes per epilogue warp: 2, or 1 when that leaves room for a third stage
 };
 
 struct G8Smem {
@@ -432,7 +436,7 @@ __host__ __device__ inline G8Smem g8_fwd_smem(const G8FwdParams &p) {
   G8Smem s;
   s.stage0 = 0;
   s.out0 = p.stages * p.stage_bytes;
-  s.bias = s.out0 + 4 * kG8NumOut * kG8OutBox;
+  s.bias = s.out0 + kG8EpiWarps * p.nout * kG8OutBox;
   s.bars = s.bias + static_cast<int>(align_up(p.bias_floats * 4, 16));
   // full, tready, empty per stage; acc_full, acc_empty x2; final; tmem slot
   s.total = s.bars + (3 * p.stages + 4 + 1) * 8 + 16;
@@ -462,9 +466,10 @@ struct G8Units {
   }
 };
 
-// 14 warps over the 4 SM sub-partitions put 4 warps on one 16K-register slice.
+// 18 warps over the 4 SM sub-partitions put 5 warps on two 16K-register slices:
+// 5 x 32 x 96 = 15,360 registers fit, 104 would not.
 template <class Gp>
-__global__ void __maxnreg__(128)
+__global__ void __maxnreg__(96)
 tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ CUtensorMap tm_out,
                   const G8FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -490,7 +495,7 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], kG8EpiWarps);
     }
     mbar_init(final_bar, 1);
     fence_mbar_init();
@@ -603,43 +608,63 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    const int ew = warp - 10, team = ew / 4;
     const int quad = warp & 3;
     const int groups = p.BD / 8;
-    uint8_t *obase = smem + L.out0 + (warp - 10) * kG8NumOut * kG8OutBox;
+    int last_g = -1;  // this team's last 8-channel group of a unit
+    for (int g = team; g < groups; g += 2) last_g = g;
+    uint8_t *obase = smem + L.out0 + ew * p.nout * kG8OutBox;
     int a = 0, oi = 0;
     uint32_t aph = 0;
     for (G8Units U(p); U.valid; U.next()) {
       const int m = U.m, j = U.j;
       if (ok) ok = mbar_wait(&acc_full[a], aph);
       tc_fence_after();
-      const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
-      for (int g = 0; g < groups; ++g) {
-        uint32_t Y[8][8];  // [accumulator block][column], in the group's plane order
-        __syncwarp();      // the TMEM loads are warp-collective
-#pragma unroll
-        for (int bk = 0; bk < 8; ++bk) tmem_ld8(tl + g * 8 + bk * p.BD, Y[bk]);
-        tmem_ld_wait();
-        if (g == groups - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
-        }
-        const int d0 = j * p.BD + g * 8;
-        if (d0 >= p.Do) continue;  // whole group is padding
-        uint8_t *ob = obase + (oi % kG8NumOut) * kG8OutBox;
-        if (lane == 0) bulk_wait_read<kG8NumOut - 1>();  // this box's last store has read it
+      if (last_g < 0) {  // this team reads nothing of the unit
+        tc_fence_before();
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {  // 16-byte chunk i of the row = output channel d0 + i
-          float F[8], y[8];
-#pragma unroll
-          for (int bk = 0; bk < 8; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
-          Gp::inverse(F, y, 64.f);  // planes and weights both carry 1/8
-          const float bv = sbias[d0 + i];
-          *reinterpret_cast<uint4 *>(ob + lane * 128 + ((i ^ (lane & 7)) << 4)) =
-              make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
-                         pack_half2(y[4] + bv, y[5] + bv), pack_half2(y[6] + bv, y[7] + bv));
+        if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
+      }
+      const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
+      for (int g = team; g < groups; g += 2) {
+        const int d0 = j * p.BD + g * 8;
+        uint8_t *ob = obase + (p.nout == 2 ? (oi & 1) : 0) * kG8OutBox;
+        if (d0 < p.Do) {
+          if (lane == 0) {  // this box's last store has read it
+            if (p.nout == 2)
+              bulk_wait_read<1>();
+            else
+              bulk_wait_read<0>();
+          }
+          __syncwarp();
         }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // four output channels at a time
+          uint32_t Y[8][4];  // [accumulator block][column], in the group's plane order
+          __syncwarp();      // the TMEM loads are warp-collective
+#pragma unroll
+          for (int bk = 0; bk < 8; ++bk) tmem_ld4(tl + g * 8 + h * 4 + bk * p.BD, Y[bk]);
+          tmem_ld_wait();
+          if (h == 1 && g == last_g) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
+          }
+          if (d0 >= p.Do) continue;  // whole group is padding
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {  // 16-byte chunk 4h + i of the row = channel d0 + 4h + i
+            const int c = 4 * h + i;
+            float F[8], y[8];
+#pragma unroll
+            for (int bk = 0; bk < 8; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
+            Gp::inverse(F, y, 64.f);  // planes and weights both carry 1/8
+            const float bv = sbias[d0 + c];
+            *reinterpret_cast<uint4 *>(ob + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
+                           pack_half2(y[4] + bv, y[5] + bv), pack_half2(y[6] + bv, y[7] + bv));
+          }
+        }
+        if (d0 >= p.Do) continue;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {  // the store clips rows past N and channels past Do

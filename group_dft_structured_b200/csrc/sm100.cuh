@@ -305,6 +305,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
                : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+
 // Warp-wide, 16 TMEM lanes from taddr's lane: thread t gets columns 2(t%4) and
 // 2(t%4)+1 of lane t/4 (r[0], r[1]) and of lane t/4 + 8 (r[2], r[3]).  Four
 // threads share a row, so a row's eight columns land in four neighbouring
