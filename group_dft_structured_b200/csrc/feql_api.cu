@@ -80,16 +80,19 @@ EncodeTiledFn encode_fn() {
 
 // Row-major fp16 matrix [rows][cols] viewed as a 2-D tensor; box = 64 cols x box_rows
 // rows, 128-byte swizzle, zero fill out of range.
+// Box of box_cols x box_rows, 128-byte swizzle (64 columns: 128-byte rows), or
+// without swizzle for other widths (the 96-byte rows of 8 channels x 6).
 int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
-                  int box_rows = kBM) {
+                  int box_rows = kBM, int box_cols = 64) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return FEQL_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
 }
@@ -101,15 +104,19 @@ int make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
 // box_count 2-D loads.  Needs row_elems % 64 == 0 (else a box would run into
 // the next row).
 int make_tmap_f16_boxes(CUtensorMap *m, const void *base, int64_t rows, int64_t row_elems,
-                        int box_rows, int box_count) {
+                        int box_rows, int box_count, int box_cols = 64) {
   EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr || row_elems % 64 != 0) return FEQL_ERR_CUDA;
-  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(row_elems / 64)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_elems) * 2, 128};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_count)};
+  if (enc == nullptr || row_elems % box_cols != 0) return FEQL_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(box_cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(row_elems / box_cols)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_elems) * 2,
+                           static_cast<cuuint64_t>(box_cols) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(box_count)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FEQL_OK : FEQL_ERR_CUDA;
 }
@@ -449,9 +456,11 @@ int launch_g8_fwd(const void *in, const uint8_t *wt, const G8Plan &P, const __ha
   p.chunk_bytes = P.chunk_bytes;
   p.nM = static_cast<int>(cdiv(N, kBM));
   p.n_units = p.nM * p.nD;
-  p.nacc = 16 * p.BD <= 512 ? 2 : 1;
-  p.acc_stride = 8 * p.BD;
-  p.stage_bytes = kG8XChunk + static_cast<int>(align_up(p.chunk_bytes, 1024));
+  constexpr int T = Gp::kT;
+  p.nacc = 2 * T * p.BD <= 512 ? 2 : 1;
+  p.acc_stride = T * p.BD;
+  p.stage_bytes = g8_xchunk<T>() + static_cast<int>(align_up(p.chunk_bytes, 1024));
+  p.out_box = 32 * 16 * T;
   p.bias_floats = p.nD * p.BD;
   const int budget = dev.smem_optin - 1024;
   // two staging boxes per epilogue warp when a unit has few input chunks (its
@@ -468,9 +477,9 @@ int launch_g8_fwd(const void *in, const uint8_t *wt, const G8Plan &P, const __ha
   p.stages = fit[p.nout];
   if (p.stages == 0) return FEQL_ERR_UNSUPPORTED;
   CUtensorMap tm, tm_out;
-  st = make_tmap_f16(&tm, in, N, static_cast<int64_t>(P.Ci) * kT8, kBM);
+  st = make_tmap_f16(&tm, in, N, static_cast<int64_t>(P.Ci) * T, kBM, 8 * T);
   if (st != FEQL_OK) return st;
-  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * kT8, 32);
+  st = make_tmap_f16(&tm_out, out, N, static_cast<int64_t>(P.Do) * T, 32, 8 * T);
   if (st != FEQL_OK) return st;
   const int smem = g8_fwd_smem(p).total + 1024;
   if (cudaFuncSetAttribute(tc_g8_fwd_kernel<Gp>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -481,7 +490,7 @@ int launch_g8_fwd(const void *in, const uint8_t *wt, const G8Plan &P, const __ha
   return launch_status();
 }
 
-G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms) {
+G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms, int T) {
   G8DwParams p;
   p.N = N;
   p.C = C;
@@ -497,6 +506,7 @@ G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms) {
   p.split_len = N > 0 ? align_up(cdiv(N, s), kG8DwTB) : kG8DwTB;
   p.splits = N > 0 ? static_cast<int>(cdiv(N, p.split_len)) : 0;
   p.slot_boxes = kG8DwDySlots + 2 * (p.CT / 16);
+  p.box_bytes = kG8DwTB * 16 * T;
   p.stages = 1;
   p.stack_dy = 0;
   p.stack_x = 0;
@@ -506,8 +516,8 @@ G8DwParams make_g8_dw_plan(int64_t N, int C, int D, int sms) {
   return p;
 }
 
-int64_t g8_dw_ws_floats(const G8DwParams &p) {
-  return static_cast<int64_t>(p.splits) * (8ll * p.D * p.Cs + p.D);
+int64_t g8_dw_ws_floats(const G8DwParams &p, int T) {
+  return static_cast<int64_t>(p.splits) * (static_cast<int64_t>(T) * p.D * p.Cs + p.D);
 }
 
 template <class Gp>
@@ -517,10 +527,11 @@ int launch_g8_dw(const void *x, const void *dy, __half *dW, __half *db, float *w
   int st = device_info(&dev);
   if (st != FEQL_OK) return st;
   if (dev.cc_major != 10) return FEQL_ERR_UNSUPPORTED;
-  G8DwParams p = make_g8_dw_plan(N, C, D, dev.sms);
-  if (ws_bytes < static_cast<size_t>(g8_dw_ws_floats(p)) * 4) return FEQL_ERR_INVALID_ARG;
+  constexpr int T = Gp::kT;
+  G8DwParams p = make_g8_dw_plan(N, C, D, dev.sms, T);
+  if (ws_bytes < static_cast<size_t>(g8_dw_ws_floats(p, T)) * 4) return FEQL_ERR_INVALID_ARG;
   p.ws = ws;
-  p.ws_db = ws + static_cast<int64_t>(p.splits) * 8 * p.D * p.Cs;
+  p.ws_db = ws + static_cast<int64_t>(p.splits) * T * p.D * p.Cs;
   const int budget = dev.smem_optin - 1024;
   p.stages = 4;
   while (p.stages > 1 && g8_dw_smem(p).total > budget) --p.stages;
@@ -531,13 +542,14 @@ int launch_g8_dw(const void *x, const void *dy, __half *dW, __half *db, float *w
     // boxes (the dy stack spans the largest tile's boxes), else one per box
     const int dt0 = D < 128 ? D : 128;
     p.nqd_stack = 2 * static_cast<int>(cdiv(dt0, 16));
-    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB,
-                                     p.nqd_stack) == FEQL_OK;
-    if (!p.stack_dy) st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * kT8, kG8DwTB);
+    p.stack_dy = make_tmap_f16_boxes(&tm_dy, dy, N, static_cast<int64_t>(D) * T, kG8DwTB,
+                                     p.nqd_stack, 8 * T) == FEQL_OK;
+    if (!p.stack_dy)
+      st = make_tmap_f16(&tm_dy, dy, N, static_cast<int64_t>(D) * T, kG8DwTB, 8 * T);
     if (st != FEQL_OK) return st;
-    p.stack_x = make_tmap_f16_boxes(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB,
-                                    2 * (p.CT / 16)) == FEQL_OK;
-    if (!p.stack_x) st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * kT8, kG8DwTB);
+    p.stack_x = make_tmap_f16_boxes(&tm_x, x, N, static_cast<int64_t>(C) * T, kG8DwTB,
+                                    2 * (p.CT / 16), 8 * T) == FEQL_OK;
+    if (!p.stack_x) st = make_tmap_f16(&tm_x, x, N, static_cast<int64_t>(C) * T, kG8DwTB, 8 * T);
     if (st != FEQL_OK) return st;
     const int smem = g8_dw_smem(p).total + 1024;
     if (cudaFuncSetAttribute(tc_g8_dw_kernel<Gp>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -779,11 +791,11 @@ int g8_pass(const void *in, const void *What, const void *bias, void *out, int64
                            out, N, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t g8_dw_workspace_bytes(int64_t N, int C, int D) {
+size_t g8_dw_workspace_bytes(int64_t N, int C, int D, int T) {
   if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
-  return static_cast<size_t>(g8_dw_ws_floats(make_g8_dw_plan(N, C, D, dev.sms))) * 4;
+  return static_cast<size_t>(g8_dw_ws_floats(make_g8_dw_plan(N, C, D, dev.sms, T), T)) * 4;
 }
 
 template <class Gp>
@@ -1024,7 +1036,7 @@ size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int d
   if (T == 4) return feql_backward_dw_workspace_bytes(N, C, D, dtype);
   int path = 0;
   if (ct_route(T, dtype, &path) != FEQL_OK) return 0;
-  if (path == kCtTensor8) return g8_dw_workspace_bytes(N, C, D);
+  if (path == kCtTensor8) return g8_dw_workspace_bytes(N, C, D, 8);
   if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
@@ -1084,7 +1096,7 @@ int feql_p4m_backward_dx(const void *dy, const void *What, void *dx, int64_t N, 
 
 size_t feql_p4m_backward_dw_workspace_bytes(int64_t N, int C, int D, int dtype) {
   if (p4m_check(dtype) != FEQL_OK) return 0;
-  return g8_dw_workspace_bytes(N, C, D);
+  return g8_dw_workspace_bytes(N, C, D, 8);
 }
 
 int feql_p4m_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws,

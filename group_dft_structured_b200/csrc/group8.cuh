@@ -41,8 +41,70 @@
 
 namespace feql {
 
-constexpr int kT8 = 8;
 constexpr float kC8 = 0.70710678118654752f;  // sqrt(2)/2
+
+// Fibre geometry.  A TMA box row holds 8 channels x T group elements of one
+// token (16 T bytes).  T = 8: 128-byte rows under the 128-byte swizzle, one
+// 16-byte chunk per channel fibre; T = 6: 96-byte rows without swizzle,
+// 12-byte fibres (a channel pair is 24 bytes, 8-byte aligned).
+template <int T>
+struct G8Geo;
+
+template <>
+struct G8Geo<8> {
+  static constexpr int kRow = 128;
+  // Packed pairs v[t] = (channel 2p, channel 2p+1) at group element t of box row r.
+  __device__ static void pair(const uint8_t *row, int p, int r, __half2 (&v)[8]) {
+    const uint4 w0 = *reinterpret_cast<const uint4 *>(row + (((2 * p) ^ (r & 7)) << 4));
+    const uint4 w1 = *reinterpret_cast<const uint4 *>(row + (((2 * p + 1) ^ (r & 7)) << 4));
+    const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w}, b[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = __byte_perm(a[e], b[e], 0x5410), hi = __byte_perm(a[e], b[e], 0x7632);
+      v[2 * e] = *reinterpret_cast<const __half2 *>(&lo);
+      v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
+    }
+  }
+  // Channel c's fibre (packed fp16 pairs) into box row r.
+  __device__ static void put(uint8_t *row, int c, int r, const uint32_t (&h)[4]) {
+    *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+  // One fibre to global memory (16-byte aligned).
+  __device__ static void store(__half *dst, const uint32_t (&h)[4]) {
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+};
+
+template <>
+struct G8Geo<6> {
+  static constexpr int kRow = 96;
+  __device__ static void pair(const uint8_t *row, int p, int, __half2 (&v)[6]) {
+    const uint2 w0 = *reinterpret_cast<const uint2 *>(row + 24 * p);
+    const uint2 w1 = *reinterpret_cast<const uint2 *>(row + 24 * p + 8);
+    const uint2 w2 = *reinterpret_cast<const uint2 *>(row + 24 * p + 16);
+    // channel 2p: w0.x, w0.y, w1.x; channel 2p + 1: w1.y, w2.x, w2.y
+    const uint32_t a[3] = {w0.x, w0.y, w1.x}, b[3] = {w1.y, w2.x, w2.y};
+#pragma unroll
+    for (int e = 0; e < 3; ++e) {
+      const uint32_t lo = __byte_perm(a[e], b[e], 0x5410), hi = __byte_perm(a[e], b[e], 0x7632);
+      v[2 * e] = *reinterpret_cast<const __half2 *>(&lo);
+      v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
+    }
+  }
+  __device__ static void put(uint8_t *row, int c, int, const uint32_t (&h)[3]) {
+    uint32_t *w = reinterpret_cast<uint32_t *>(row + 12 * c);
+    w[0] = h[0];
+    w[1] = h[1];
+    w[2] = h[2];
+  }
+  // (4-byte aligned: fibres start at multiples of 12 bytes)
+  __device__ static void store(__half *dst, const uint32_t (&h)[3]) {
+    uint32_t *w = reinterpret_cast<uint32_t *>(dst);
+    w[0] = h[0];
+    w[1] = h[1];
+    w[2] = h[2];
+  }
+};
 
 // One tensor-core MMA of a table: accumulator column block, A operand plane,
 // B operand start (weight row block or x plane), N = 2 blocks (wide) or 1, and
@@ -55,6 +117,9 @@ struct G8Mma {
 // Cyclic group C_8
 // ---------------------------------------------------------------------------
 struct Cyclic8 {
+  static constexpr int kT = 8;        // group order: fibre length, planes, accumulator blocks
+  static constexpr int kFwdMmas = 8;  // entries of the fwd() and dw() tables
+  static constexpr int kDwMmas = 8;
   // Weight rows per output channel of a chunk: What0, What4 and for each complex
   // bin k = 1, 2, 3 at row block r_k = 2 + 3(k-1): Re_k, Im_k, -Re_k, so that
   // the window (Re_k ; Im_k) multiplies Re X_k and (Im_k ; -Re_k) the stored
@@ -181,6 +246,9 @@ struct Cyclic8 {
 // Point group D4 of p4m
 // ---------------------------------------------------------------------------
 struct Dihedral4 {
+  static constexpr int kT = 8;
+  static constexpr int kFwdMmas = 8;
+  static constexpr int kDwMmas = 8;
   // Weight rows per output channel of a chunk: A1, A2, B1, B2, then the 2 x 2
   // block of E with W^(E)[k][j] at row block 4 + 2k + j, so that the window
   // (W^[k][0] ; W^[k][1]) multiplies the plane x^(E)[i][k] into [Y^[i][0] | Y^[i][1]].
@@ -329,26 +397,16 @@ __host__ __device__ inline G8Layout make_g8_layout(int C, int D, int wrows) {
   return L;
 }
 
-// Two channels' 16-byte fibres (8 fp16 group values each) as 8 packed pairs:
-// v[t] = (channel q, channel q+1) at group element t.
-__device__ __forceinline__ void g8_pair_values(const uint4 &w0, const uint4 &w1, __half2 (&v)[8]) {
-  const uint32_t a[4] = {w0.x, w0.y, w0.z, w0.w}, b[4] = {w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint32_t lo = __byte_perm(a[e], b[e], 0x5410), hi = __byte_perm(a[e], b[e], 0x7632);
-    v[2 * e] = *reinterpret_cast<const __half2 *>(&lo);
-    v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
-  }
-}
-
-// Planes of two channels, packed: o[p] = plane p of (q, q+1), low half first.
+// Planes of the channel pair (2p, 2p+1) of box row r, packed: o[k] = plane k
+// of both channels, low half first.
 template <class Gp>
-__device__ __forceinline__ void g8_planes_pair(const uint4 &w0, const uint4 &w1, uint32_t (&o)[8]) {
-  __half2 v[8], r[8];
-  g8_pair_values(w0, w1, v);
-  Gp::planes_h2(v, r);
+__device__ __forceinline__ void g8_planes_pair(const uint8_t *row, int p, int r,
+                                               uint32_t (&o)[Gp::kT]) {
+  __half2 v[Gp::kT], w[Gp::kT];
+  G8Geo<Gp::kT>::pair(row, p, r, v);
+  Gp::planes_h2(v, w);
 #pragma unroll
-  for (int p = 0; p < 8; ++p) o[p] = *reinterpret_cast<const uint32_t *>(&r[p]);
+  for (int k = 0; k < Gp::kT; ++k) o[k] = *reinterpret_cast<const uint32_t *>(&w[k]);
 }
 
 // One thread per fp16 element of the tiled weight buffer (both directions).
@@ -373,17 +431,18 @@ __global__ void wfft_g8_kernel(const __half *__restrict__ W, uint8_t *__restrict
     float v = 0.f;
     if (o < P.Do && i < P.Ci) {
       const int d = dir == 0 ? o : i, c = dir == 0 ? i : o;
-      const __half *src = W + (static_cast<int64_t>(d) * C + c) * kT8;
-      float w[8], wr[Gp::kWRows];
+      const __half *src = W + (static_cast<int64_t>(d) * C + c) * Gp::kT;
+      float w[Gp::kT], wr[Gp::kWRows];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) w[t] = __half2float(src[t]);
+      for (int t = 0; t < Gp::kT; ++t) w[t] = __half2float(src[t]);
       Gp::weight_rows(w, dir, wr);
 #pragma unroll
       for (int r = 0; r < Gp::kWRows; ++r)
         if (r == sub) v = wr[r];
     }
     const int64_t base = (dir == 0 ? L.off_fwd : L.off_dx) + chunk * P.chunk_bytes;
-    // every weight plane divided by 8 (as the operand planes): no fp16 overflow for any finite W
+    // every weight plane divided by 8 (as the operand planes): no fp16 overflow for any
+    // finite W (a bin sums at most 8 values)
     *reinterpret_cast<__half *>(What + base + sw32_offset(row, k)) = __float2half_rn(0.125f * v);
   }
 }
@@ -410,21 +469,23 @@ __global__ void wfft_g8_kernel(const __half *__restrict__ W, uint8_t *__restrict
 //                and the warp issues one 4 KB TMA store (two boxes per warp)
 constexpr int kG8EpiWarps = 8;
 constexpr int kG8Threads = 64 + (8 + kG8EpiWarps) * 32;
-constexpr int kG8XChunk = kBM * kCK * kT8 * 2;  // 32 KB: 128 tokens x 16 channels x 8
-constexpr int kG8Box = kG8XChunk / 2;          // 16 KB: 8 channels
+// input chunk: 128 tokens x 16 channels x T (4 KB x T: two boxes of 8 channels),
+// rewritten in place as T planes of 128 tokens x 32 B
+template <int T>
+constexpr int g8_xchunk() { return kBM * kCK * T * 2; }
 constexpr int kG8Plane = kBM * kCK * 2;         // 4 KB: 128 tokens x 32 B
-constexpr int kG8OutBox = 32 * 128;             // 4 KB: 32 rows x 8 channels x 8
 constexpr int kG8MaxOut = 2;                    // staging boxes per epilogue warp (at most)
 
 struct G8FwdParams {
   const uint8_t *wt;   // weight chunks of this direction, [j][kc]
   const __half *bias;  // [Do] or nullptr
-  __half *out;         // [N][Do][8]
+  __half *out;         // [N][Do][T]
   int64_t N;
   int Ci, Do, BD, nD, nK, chunk_bytes;
   int nM, n_units;
   int nacc, acc_stride;
   int stages, stage_bytes, bias_floats;
+  int out_box;         // one staging box: 32 rows x 8 channels x T fp16
   int nout;            // staging boxes per epilogue warp: 2, or 1 when that leaves room for a third stage
 };
 
@@ -436,7 +497,7 @@ __host__ __device__ inline G8Smem g8_fwd_smem(const G8FwdParams &p) {
   G8Smem s;
   s.stage0 = 0;
   s.out0 = p.stages * p.stage_bytes;
-  s.bias = s.out0 + kG8EpiWarps * p.nout * kG8OutBox;
+  s.bias = s.out0 + kG8EpiWarps * p.nout * p.out_box;
   s.bars = s.bias + static_cast<int>(align_up(p.bias_floats * 4, 16));
   // full, tready, empty per stage; acc_full, acc_empty x2; final; tmem slot
   s.total = s.bars + (3 * p.stages + 4 + 1) * 8 + 16;
@@ -475,6 +536,9 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
+  constexpr int T = Gp::kT;
+  using Geo = G8Geo<T>;
+  constexpr int kChunk = g8_xchunk<T>(), kBox = kChunk / 2;
   const G8Smem L = g8_fwd_smem(p);
   float *sbias = reinterpret_cast<float *>(smem + L.bias);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
@@ -525,10 +589,10 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
           if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
           if (ok) {
             uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
-            mbar_arrive_expect_tx(&full[s], kG8XChunk + p.chunk_bytes);
-            tma_load_2d(st, &tm_in, kc * (kCK * kT8), m * kBM, &full[s]);
-            tma_load_2d(st + kG8Box, &tm_in, kc * (kCK * kT8) + 64, m * kBM, &full[s]);
-            bulk_load(st + kG8XChunk,
+            mbar_arrive_expect_tx(&full[s], kChunk + p.chunk_bytes);
+            tma_load_2d(st, &tm_in, kc * (kCK * T), m * kBM, &full[s]);
+            tma_load_2d(st + kBox, &tm_in, kc * (kCK * T) + 8 * T, m * kBM, &full[s]);
+            bulk_load(st + kChunk,
                       p.wt + (static_cast<int64_t>(j) * p.nK + kc) * p.chunk_bytes,
                       p.chunk_bytes, &full[s]);
           }
@@ -557,9 +621,9 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
           if (ok) ok = mbar_wait(&tready[s], ph);
           tc_fence_after();
           if (ok) {
-            const uint32_t xd = x0 + s * stage16, wd = xd + (kG8XChunk >> 4);
+            const uint32_t xd = x0 + s * stage16, wd = xd + (kChunk >> 4);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {  // the group's table: compile-time offsets
+            for (int e = 0; e < Gp::kFwdMmas; ++e) {  // the group's table: compile-time offsets
               const G8Mma t = Gp::fwd(e);
               mma_f16_lo(acc + t.acc * p.BD, xd + t.a * pl16, wd + t.b * w16, dhi,
                          t.wide ? id_2bd : id_bd, (kc > 0 || t.chained) ? 1u : 0u);
@@ -584,20 +648,18 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
       for (int kc = 0; kc < p.nK; ++kc) {
         if (ok) ok = mbar_wait(&full[s], ph);
         uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
-        const uint8_t *src = st + bx * kG8Box + r * 128;
-        uint32_t pw[8][4];  // [plane][channel pair], packed fp16
+        const uint8_t *src = st + bx * kBox + r * Geo::kRow;
+        uint32_t pw[T][4];  // [plane][channel pair], packed fp16
 #pragma unroll
-        for (int q = 0; q < 8; q += 2) {  // 16-byte chunk q = channel 8 bx + q, its 8 group elements
-          const uint4 r0 = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-          const uint4 r1 = *reinterpret_cast<const uint4 *>(src + (((q + 1) ^ (r & 7)) << 4));
-          uint32_t o[8];
-          g8_planes_pair<Gp>(r0, r1, o);
+        for (int q = 0; q < 4; ++q) {  // channels 8 bx + 2q, 8 bx + 2q + 1
+          uint32_t o[T];
+          g8_planes_pair<Gp>(src, q, r, o);
 #pragma unroll
-          for (int pp = 0; pp < 8; ++pp) pw[pp][q / 2] = o[pp];
+          for (int pp = 0; pp < T; ++pp) pw[pp][q] = o[pp];
         }
         named_bar_sync(2, 256);  // every row read before the planes overwrite it
 #pragma unroll
-        for (int pp = 0; pp < 8; ++pp)
+        for (int pp = 0; pp < T; ++pp)
           *reinterpret_cast<uint4 *>(st + pp * kG8Plane + r * 32 + (((bx ^ (r >> 2)) & 1) << 4)) =
               make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
         fence_proxy_async_smem();
@@ -613,7 +675,7 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
     const int groups = p.BD / 8;
     int last_g = -1;  // this team's last 8-channel group of a unit
     for (int g = team; g < groups; g += 2) last_g = g;
-    uint8_t *obase = smem + L.out0 + ew * p.nout * kG8OutBox;
+    uint8_t *obase = smem + L.out0 + ew * p.nout * p.out_box;
     int a = 0, oi = 0;
     uint32_t aph = 0;
     for (G8Units U(p); U.valid; U.next()) {
@@ -628,7 +690,7 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
       const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * p.acc_stride;
       for (int g = team; g < groups; g += 2) {
         const int d0 = j * p.BD + g * 8;
-        uint8_t *ob = obase + (p.nout == 2 ? (oi & 1) : 0) * kG8OutBox;
+        uint8_t *ob = obase + (p.nout == 2 ? (oi & 1) : 0) * p.out_box;
         if (d0 < p.Do) {
           if (lane == 0) {  // this box's last store has read it
             if (p.nout == 2)
@@ -640,10 +702,10 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // four output channels at a time
-          uint32_t Y[8][4];  // [accumulator block][column], in the group's plane order
+          uint32_t Y[T][4];  // [accumulator block][column], in the group's plane order
           __syncwarp();      // the TMEM loads are warp-collective
 #pragma unroll
-          for (int bk = 0; bk < 8; ++bk) tmem_ld4(tl + g * 8 + h * 4 + bk * p.BD, Y[bk]);
+          for (int bk = 0; bk < T; ++bk) tmem_ld4(tl + g * 8 + h * 4 + bk * p.BD, Y[bk]);
           tmem_ld_wait();
           if (h == 1 && g == last_g) {
             tc_fence_before();
@@ -652,23 +714,24 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
           }
           if (d0 >= p.Do) continue;  // whole group is padding
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {  // 16-byte chunk 4h + i of the row = channel d0 + 4h + i
+          for (int i = 0; i < 4; ++i) {  // fibre 4h + i of the row = channel d0 + 4h + i
             const int c = 4 * h + i;
-            float F[8], y[8];
+            float F[T], y[T];
 #pragma unroll
-            for (int bk = 0; bk < 8; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
+            for (int bk = 0; bk < T; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
             Gp::inverse(F, y, 64.f);  // planes and weights both carry 1/8
             const float bv = sbias[d0 + c];
-            *reinterpret_cast<uint4 *>(ob + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(pack_half2(y[0] + bv, y[1] + bv), pack_half2(y[2] + bv, y[3] + bv),
-                           pack_half2(y[4] + bv, y[5] + bv), pack_half2(y[6] + bv, y[7] + bv));
+            uint32_t hv[T / 2];
+#pragma unroll
+            for (int e = 0; e < T / 2; ++e) hv[e] = pack_half2(y[2 * e] + bv, y[2 * e + 1] + bv);
+            Geo::put(ob + lane * Geo::kRow, c, lane, hv);
           }
         }
         if (d0 >= p.Do) continue;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {  // the store clips rows past N and channels past Do
-          tma_store_2d(&tm_out, d0 * kT8, m * kBM + quad * 32, ob);
+          tma_store_2d(&tm_out, d0 * T, m * kBM + quad * 32, ob);
           bulk_commit();
         }
         ++oi;
@@ -706,7 +769,10 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
 // (N = 2 CT), i.e. Re G_k = a[c] + b[CT + c], Im G_k = a[CT + c] - b[c]:
 // 8 MMAs and 14 CT TMEM columns.
 constexpr int kG8DwTB = 32;                     // tokens per chunk (2 MMA K-steps)
-constexpr int kG8DwBox = kG8DwTB * 128;        // 4 KB: 32 tokens x 8 channels x 8
+// one box: 32 tokens x 8 channels x T (4 KB for T = 8); a pair of boxes holds
+// the same bytes as the pair's T planes of 32 tokens x 32 B
+template <int T>
+constexpr int g8_dw_box() { return kG8DwTB * 16 * T; }
 constexpr int kG8DwDySlots = 16;                // box slots for dy (the M = 128 operand spans 8 pairs)
 constexpr int kG8DwThreads = 64 + 8 * 32;
 constexpr int kG8DwMaxPer = 3;                  // (box, token) items per transform thread
@@ -721,7 +787,8 @@ struct G8DwParams {
   int slot_boxes;      // kG8DwDySlots + 2 * CT / 16
   int stack_dy, stack_x;  // 1: one 3-D load brings all of a chunk's dy (x) boxes
   int nqd_stack;       // boxes in the dy stack (those of the largest d tile)
-  float *ws;           // [splits][8][D][Cs]: G0, G4, Re G1, Im G1, Re G2, Im G2, Re G3, Im G3
+  int box_bytes;       // g8_dw_box<T>()
+  float *ws;           // [splits][T][D][Cs]: the T bin planes (C_8: G0, G4, Re G1, Im G1, ..., Im G3)
   float *ws_db;        // [splits][D]
 };
 
@@ -732,7 +799,7 @@ struct G8DwSmem {
 __host__ __device__ inline G8DwSmem g8_dw_smem(const G8DwParams &p) {
   G8DwSmem s;
   s.stage0 = 0;
-  s.bars = p.stages * p.slot_boxes * kG8DwBox;
+  s.bars = p.stages * p.slot_boxes * p.box_bytes;
   // full, tready, empty per stage; acc_full; tmem slot
   s.total = s.bars + (3 * p.stages + 1) * 8 + 16;
   return s;
@@ -745,6 +812,9 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
+  constexpr int T = Gp::kT;
+  using Geo = G8Geo<T>;
+  constexpr int kBox = g8_dw_box<T>();
   const G8DwSmem L = g8_dw_smem(p);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint64_t *full = bars;
@@ -767,7 +837,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
   int64_t t_end = t_begin + p.split_len;
   if (t_end > p.N) t_end = p.N;
   const int nch = t_begin < t_end ? static_cast<int>(cdiv(t_end - t_begin, kG8DwTB)) : 0;
-  const int xoff = kG8DwDySlots * kG8DwBox;  // x region of a stage
+  const int xoff = kG8DwDySlots * kBox;  // x region of a stage
   const int ncols = Gp::kDwBlocks * p.CT;
   const uint32_t tmem_cols = ncols <= 256 ? 256u : 512u;
 
@@ -800,22 +870,22 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
       for (int ch = 0; ch < nch; ++ch) {
         if (ok) ok = mbar_wait(&empty[s], ph ^ 1);
         if (ok) {
-          uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kG8DwBox;
+          uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kBox;
           const int32_t row = static_cast<int32_t>(t_begin + static_cast<int64_t>(ch) * kG8DwTB);
           // a stack lands whole (boxes past the last channel read as zeros)
           const int bd = p.stack_dy ? p.nqd_stack : nqd;
-          mbar_arrive_expect_tx(&full[s], (bd + nqc) * kG8DwBox);
+          mbar_arrive_expect_tx(&full[s], (bd + nqc) * kBox);
           if (p.stack_dy) {
             tma_load_3d(st, &tm_dy, 0, row, d0 / 8, &full[s]);
           } else {
             for (int q = 0; q < nqd; ++q)
-              tma_load_2d(st + q * kG8DwBox, &tm_dy, (d0 + 8 * q) * kT8, row, &full[s]);
+              tma_load_2d(st + q * kBox, &tm_dy, (d0 + 8 * q) * T, row, &full[s]);
           }
           if (p.stack_x) {
             tma_load_3d(st + xoff, &tm_x, 0, row, c0 / 8, &full[s]);
           } else {
             for (int q = 0; q < nqc; ++q)
-              tma_load_2d(st + xoff + q * kG8DwBox, &tm_x, (c0 + 8 * q) * kT8, row, &full[s]);
+              tma_load_2d(st + xoff + q * kBox, &tm_x, (c0 + 8 * q) * T, row, &full[s]);
           }
         }
         if (++s == p.stages) { s = 0; ph ^= 1; }
@@ -826,12 +896,12 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
     if (lane == 0) {
       const uint32_t id1 = instr_desc(128, p.CT, 0, 0, 1, 1);
       const uint32_t id2 = instr_desc(128, 2 * p.CT, 0, 0, 1, 1);
-      const uint64_t da = smem_desc(0, 2 * kG8DwBox, 256, kSw32);  // dy: pairs 8 KB apart
+      const uint64_t da = smem_desc(0, 2 * kBox, 256, kSw32);  // dy: pairs 2 boxes apart
       const uint64_t db = smem_desc(0, kG8DwTB * 32, 256, kSw32);  // x: pairs 1 KB apart
       const uint32_t dhi = desc_hi(da);
       const uint32_t a0 = desc_lo(desc_at(da, smem_u32(smem + L.stage0)));
       const uint32_t b0 = desc_lo(desc_at(db, smem_u32(smem + L.stage0 + xoff)));
-      const uint32_t stage16 = (p.slot_boxes * kG8DwBox) >> 4;
+      const uint32_t stage16 = (p.slot_boxes * kBox) >> 4;
       const uint32_t apl = (kG8DwTB * 32) >> 4, bpl = (npc * kG8DwTB * 32) >> 4;  // one plane
       int s = 0;
       uint32_t ph = 0;
@@ -846,7 +916,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
             const uint32_t A = sa + k * 32, B = sb + k * 32;
             const bool first = ch == 0 && k == 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {  // the group's table: compile-time offsets
+            for (int e = 0; e < Gp::kDwMmas; ++e) {  // the group's table: compile-time offsets
               const G8Mma t = Gp::dw(e);
               mma_f16_lo(tmem_base + t.acc * p.CT, A + t.a * apl, B + t.b * bpl, dhi,
                          t.wide ? id2 : id1, (first && !t.chained) ? 0u : 1u);
@@ -871,28 +941,26 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
     uint32_t ph = 0;
     for (int ch = 0; ch < nch; ++ch) {
       if (ok) ok = mbar_wait(&full[s], ph);
-      uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kG8DwBox;
-      uint32_t pw[kG8DwMaxPer][8][4];
+      uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kBox;
+      uint32_t pw[kG8DwMaxPer][T][4];
 #pragma unroll
       for (int k = 0; k < kG8DwMaxPer; ++k) {
         const int e = t + k * 256;
         const int bi = e / kG8DwTB, r = e % kG8DwTB;
         if (bi < nbox) {
-          const uint8_t *src = st + (bi < nqd ? bi * kG8DwBox : xoff + (bi - nqd) * kG8DwBox) +
-                               r * 128;
+          const uint8_t *src = st + (bi < nqd ? bi * kBox : xoff + (bi - nqd) * kBox) +
+                               r * Geo::kRow;
 #pragma unroll
-          for (int q = 0; q < 8; q += 2) {
-            const uint4 r0 = *reinterpret_cast<const uint4 *>(src + ((q ^ (r & 7)) << 4));
-            const uint4 r1 = *reinterpret_cast<const uint4 *>(src + (((q + 1) ^ (r & 7)) << 4));
-            uint32_t o[8];
-            g8_planes_pair<Gp>(r0, r1, o);
+          for (int q = 0; q < 4; ++q) {  // channels 2q, 2q + 1 of the box
+            uint32_t o[T];
+            g8_planes_pair<Gp>(src, q, r, o);
             if (do_db && bi < nqd) {  // bin 0 of the dy planes, as the MMAs see it
               const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&o[0]));
-              db_acc[k][q] += f.x;
-              db_acc[k][q + 1] += f.y;
+              db_acc[k][2 * q] += f.x;
+              db_acc[k][2 * q + 1] += f.y;
             }
 #pragma unroll
-            for (int pp = 0; pp < 8; ++pp) pw[k][pp][q / 2] = o[pp];
+            for (int pp = 0; pp < T; ++pp) pw[k][pp][q] = o[pp];
           }
         }
       }
@@ -905,11 +973,11 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
           const bool is_dy = bi < nqd;
           const int q2 = is_dy ? bi : bi - nqd;
           const int g = q2 / 2, hh = q2 % 2;
-          // dy pair g: plane pp at g x 8 KB + pp x 1 KB; x: plane-major (pp x npc + g) x 1 KB
-          uint8_t *pbase = is_dy ? st + g * 2 * kG8DwBox : st + xoff + g * kG8DwTB * 32;
+          // dy pair g: plane pp at g x 2 boxes + pp x 1 KB; x: plane-major (pp x npc + g) x 1 KB
+          uint8_t *pbase = is_dy ? st + g * 2 * kBox : st + xoff + g * kG8DwTB * 32;
           const int pstride = is_dy ? kG8DwTB * 32 : npc * kG8DwTB * 32;
 #pragma unroll
-          for (int pp = 0; pp < 8; ++pp)
+          for (int pp = 0; pp < T; ++pp)
             *reinterpret_cast<uint4 *>(pbase + pp * pstride + r * 32 + (((hh ^ (r >> 2)) & 1) << 4)) =
                 make_uint4(pw[k][pp][0], pw[k][pp][1], pw[k][pp][2], pw[k][pp][3]);
         }
@@ -927,7 +995,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
     const int d = quad * 32 + lane;  // row of the tile
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const int64_t plane = static_cast<int64_t>(p.D) * p.Cs;
-    float *dst = p.ws + static_cast<int64_t>(split) * 8 * plane + static_cast<int64_t>(d0 + d) * p.Cs + c0;
+    float *dst = p.ws + static_cast<int64_t>(split) * T * plane + static_cast<int64_t>(d0 + d) * p.Cs + c0;
     for (int g = half; g < p.CT / 8; g += 2) {  // 8-column steps
       uint32_t blk[Gp::kDwBlocks][8];  // accumulator block k, 8 columns of this step
       __syncwarp();  // the TMEM loads are warp-collective
@@ -935,18 +1003,18 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
       for (int k = 0; k < Gp::kDwBlocks; ++k) tmem_ld8(tl + k * p.CT + g * 8, blk[k]);
       tmem_ld_wait();
       if (d0 + d < p.D && c0 + g * 8 < p.C) {
-        float G[8][8];
+        float G[T][8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          float a[Gp::kDwBlocks], Gi[8];
+          float a[Gp::kDwBlocks], Gi[T];
 #pragma unroll
           for (int k = 0; k < Gp::kDwBlocks; ++k) a[k] = __uint_as_float(blk[k][i]);
           Gp::dw_planes(a, Gi);
 #pragma unroll
-          for (int bin = 0; bin < 8; ++bin) G[bin][i] = Gi[bin];
+          for (int bin = 0; bin < T; ++bin) G[bin][i] = Gi[bin];
         }
 #pragma unroll
-        for (int bin = 0; bin < 8; ++bin) {
+        for (int bin = 0; bin < T; ++bin) {
           float4 *o = reinterpret_cast<float4 *>(dst + bin * plane + g * 8);
           o[0] = make_float4(G[bin][0], G[bin][1], G[bin][2], G[bin][3]);
           o[1] = make_float4(G[bin][4], G[bin][5], G[bin][6], G[bin][7]);
@@ -997,35 +1065,41 @@ __global__ void __launch_bounds__(kRed8Out * kRed8Groups)
 g8_dw_reduce_kernel(const float *__restrict__ ws, const float *__restrict__ ws_db,
                      __half *__restrict__ dW, __half *__restrict__ db, int splits, int C, int D,
                      int Cs) {
-  __shared__ float part[kRed8Groups][kT8][kRed8Out];
+  constexpr int T = Gp::kT;
+  __shared__ float part[kRed8Groups][T][kRed8Out];
   const int64_t n = static_cast<int64_t>(D) * C;
   const int64_t plane = static_cast<int64_t>(D) * Cs;
   const int64_t nblk_w = cdiv(n, kRed8Out);
   const int lo = threadIdx.x % kRed8Out, grp = threadIdx.x / kRed8Out;
   if (blockIdx.x < nblk_w) {
     const int64_t e = blockIdx.x * static_cast<int64_t>(kRed8Out) + lo;
-    float G[kT8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float G[T];
+#pragma unroll
+    for (int k = 0; k < T; ++k) G[k] = 0.f;
     if (e < n) {
       const float *src = ws + (e / C) * Cs + (e % C);
       for (int s = grp; s < splits; s += kRed8Groups) {
-        const float *q = src + static_cast<int64_t>(s) * kT8 * plane;
+        const float *q = src + static_cast<int64_t>(s) * T * plane;
 #pragma unroll
-        for (int k = 0; k < kT8; ++k) G[k] += q[k * plane];
+        for (int k = 0; k < T; ++k) G[k] += q[k * plane];
       }
     }
 #pragma unroll
-    for (int k = 0; k < kT8; ++k) part[grp][k][lo] = G[k];
+    for (int k = 0; k < T; ++k) part[grp][k][lo] = G[k];
     __syncthreads();
     if (grp == 0 && e < n) {
-      float t[kT8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float t[T];
+#pragma unroll
+      for (int k = 0; k < T; ++k) t[k] = 0.f;
       for (int q = 0; q < kRed8Groups; ++q)
 #pragma unroll
-        for (int k = 0; k < kT8; ++k) t[k] += part[q][k][lo];
-      float y[kT8];
+        for (int k = 0; k < T; ++k) t[k] += part[q][k][lo];
+      float y[T];
       Gp::inverse(t, y, 64.f);  // x and dy planes both carry 1/8
-      *reinterpret_cast<uint4 *>(dW + e * kT8) =
-          make_uint4(pack_half2(y[0], y[1]), pack_half2(y[2], y[3]), pack_half2(y[4], y[5]),
-                     pack_half2(y[6], y[7]));
+      uint32_t hv[T / 2];
+#pragma unroll
+      for (int k = 0; k < T / 2; ++k) hv[k] = pack_half2(y[2 * k], y[2 * k + 1]);
+      G8Geo<T>::store(dW + e * T, hv);
     }
   } else if (db != nullptr) {
     const int64_t d = (blockIdx.x - nblk_w) * kRed8Out + lo;
