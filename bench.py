@@ -599,8 +599,8 @@ def per_config_report(F, torch, stream, reps):
     return out
 
 
-# The widened rows at full size: the C_8 and p4m layers and the two MLP blocks
-# on the tensor cores, C_6 on the CUDA cores (fp32 arithmetic on fp16 data).
+# The widened rows at full size: the C_8, C_6 and p4m layers and the two MLP
+# blocks, all on the tensor cores.
 WIDENING_RUNS = (6, 8, 10, 7, 9)
 # Nominal special-function throughput: 16 MUFU operations per SM per clock
 # (four per SM sub-partition), one tanh.approx.f16x2 (two values) per
@@ -614,7 +614,7 @@ def widening_report(F, torch, stream, reps, meas, nom, flush):
     CUDA-event timings with the L2 flushed before each, median and min, against
     the slower of its algorithmic bytes at HBM bandwidth and its Fourier-route
     FLOPs at the arithmetic peak of the units it runs on (tensor cores, or the
-    fp32 FMA pipes for C_6).  The MLP block also gets a special-function floor:
+    fp32 FMA pipes for a shape the CUDA-core kernels serve).  The MLP block also gets a special-function floor:
     its GELU takes one tanh per two hidden values."""
     import numpy as np
 
@@ -628,7 +628,8 @@ def widening_report(F, torch, stream, reps, meas, nom, flush):
         st = (setup_mlp if mlp else setup_layer)(args, w, 0, s, F, torch)
         calls, res = st["calls"], {}
         calls["wfft"]()
-        simt = w.T not in (4, 8)
+        # the tensor-core kernels serve T = 4, 8, and 6 when C and D are multiples of 4
+        simt = not (w.T in (4, 8) or (w.T == 6 and w.C % 4 == 0 and w.D % 4 == 0))
         for p in st["passes"]:
             for _ in range(3):
                 calls[p]()

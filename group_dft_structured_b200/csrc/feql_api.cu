@@ -633,18 +633,21 @@ int launch_mlp(const void *x, const uint8_t *wt, const __half *b1, const __half 
   return launch_status();
 }
 
-// Checks shared by the C_T entry points: a supported group order and mode.
-// Returns FEQL_OK for T = 8 in FEQL_FP16 (T = 4 is forwarded before this).
-// For T != 4: the tensor-core kernels serve T = 8 in FEQL_FP16, the CUDA-core
-// kernels every order 2..16 in the other modes (and every other order in fp16).
-enum CtPath { kCtTensor8 = 1, kCtSimt = 2 };
+// Checks shared by the C_T entry points: a supported group order and mode, and
+// the kernel family that serves them (T = 4 is forwarded before this).  In
+// FEQL_FP16 the tensor-core kernels serve T = 8, and T = 6 when C and D are
+// multiples of 4 (16-byte row strides for the tensor maps of 12-byte fibres);
+// the CUDA-core kernels every order 2..16 otherwise.
+enum CtPath { kCtTensor8 = 1, kCtSimt = 2, kCtTensor6 = 3 };
 
-int ct_route(int T, int dtype, int *path) {
+int ct_route(int T, int C, int D, int dtype, int *path) {
   if (!valid_dtype(dtype)) return FEQL_ERR_INVALID_ARG;
   if (T < 2 || T > kCtMaxT) return FEQL_ERR_UNSUPPORTED;
   const int dt = resolve(dtype);
   if (dt == FEQL_FP32_3XTF32) return FEQL_ERR_UNSUPPORTED;
-  *path = (T == 8 && dt == FEQL_FP16) ? kCtTensor8 : kCtSimt;
+  *path = kCtSimt;
+  if (dt == FEQL_FP16 && T == 8) *path = kCtTensor8;
+  if (dt == FEQL_FP16 && T == 6 && C % 4 == 0 && D % 4 == 0) *path = kCtTensor6;
   return FEQL_OK;
 }
 
@@ -980,8 +983,9 @@ int feql_backward_dw(const void *x, const void *dy, void *dW, void *db, void *ws
 size_t feql_ct_weight_fft_bytes(int T, int C, int D, int dtype) {
   if (T == 4) return feql_weight_fft_bytes(C, D, dtype);
   int path = 0;
-  if (ct_route(T, dtype, &path) != FEQL_OK || check_shape(C, D) != FEQL_OK) return 0;
+  if (ct_route(T, C, D, dtype, &path) != FEQL_OK || check_shape(C, D) != FEQL_OK) return 0;
   if (path == kCtTensor8) return g8_weight_fft_bytes<Cyclic8>(C, D);
+  if (path == kCtTensor6) return g8_weight_fft_bytes<Cyclic6>(C, D);
   return static_cast<size_t>(2) * T * C * D * 4;  // fp32 planes [dir][plane][Do][Ci]
 }
 
@@ -989,9 +993,10 @@ int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype
                        feql_stream stream) {
   if (T == 4) return feql_weight_fft(W, What, C, D, dtype, stream);
   int path = 0;
-  int st = ct_route(T, dtype, &path);
+  int st = ct_route(T, C, D, dtype, &path);
   if (st != FEQL_OK) return st;
   if (path == kCtTensor8) return g8_weight_fft<Cyclic8>(W, What, C, D, stream);
+  if (path == kCtTensor6) return g8_weight_fft<Cyclic6>(W, What, C, D, stream);
   if (W == nullptr || What == nullptr || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(What)) return FEQL_ERR_INVALID_ARG;
   DeviceInfo dev;
@@ -1005,9 +1010,10 @@ int feql_ct_weight_fft(int T, const void *W, void *What, int C, int D, int dtype
 static int ct_pass(int T, const void *in, const void *What, const void *bias, void *out, int64_t N,
                    int C, int D, int dtype, feql_stream stream, int dir) {
   int path = 0;
-  const int st = ct_route(T, dtype, &path);
+  const int st = ct_route(T, C, D, dtype, &path);
   if (st != FEQL_OK) return st;
   if (path == kCtTensor8) return g8_pass<Cyclic8>(in, What, bias, out, N, C, D, stream, dir);
+  if (path == kCtTensor6) return g8_pass<Cyclic6>(in, What, bias, out, N, C, D, stream, dir);
   if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return FEQL_ERR_INVALID_ARG;
   if (N > 0 && (in == nullptr || What == nullptr || out == nullptr)) return FEQL_ERR_INVALID_ARG;
   if (!aligned16(in) || !aligned16(What) || !aligned16(out)) return FEQL_ERR_INVALID_ARG;
@@ -1035,8 +1041,9 @@ int feql_ct_backward_dx(int T, const void *dy, const void *What, void *dx, int64
 size_t feql_ct_backward_dw_workspace_bytes(int T, int64_t N, int C, int D, int dtype) {
   if (T == 4) return feql_backward_dw_workspace_bytes(N, C, D, dtype);
   int path = 0;
-  if (ct_route(T, dtype, &path) != FEQL_OK) return 0;
+  if (ct_route(T, C, D, dtype, &path) != FEQL_OK) return 0;
   if (path == kCtTensor8) return g8_dw_workspace_bytes(N, C, D, 8);
+  if (path == kCtTensor6) return g8_dw_workspace_bytes(N, C, D, 6);
   if (N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK) return 0;
   DeviceInfo dev;
   if (device_info(&dev) != FEQL_OK) return 0;
@@ -1047,9 +1054,10 @@ int feql_ct_backward_dw(int T, const void *x, const void *dy, void *dW, void *db
                         size_t ws_bytes, int64_t N, int C, int D, int dtype, feql_stream stream) {
   if (T == 4) return feql_backward_dw(x, dy, dW, db, ws, ws_bytes, N, C, D, dtype, stream);
   int path = 0;
-  int st = ct_route(T, dtype, &path);
+  int st = ct_route(T, C, D, dtype, &path);
   if (st != FEQL_OK) return st;
   if (path == kCtTensor8) return g8_dw<Cyclic8>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
+  if (path == kCtTensor6) return g8_dw<Cyclic6>(x, dy, dW, db, ws, ws_bytes, N, C, D, stream);
   if (dW == nullptr || ws == nullptr || N < 0 || N > kMaxTokens || check_shape(C, D) != FEQL_OK)
     return FEQL_ERR_INVALID_ARG;
   if (N > 0 && (x == nullptr || dy == nullptr)) return FEQL_ERR_INVALID_ARG;

@@ -360,6 +360,123 @@ struct Dihedral4 {
 };
 
 // ---------------------------------------------------------------------------
+// Cyclic group C_6
+// ---------------------------------------------------------------------------
+// A non-dyadic order (twiddles cos(pi/3) = 1/2 and sin(pi/3) = sqrt(3)/2): the
+// real 6-point DFT keeps bins 0..3, bins 0 and 3 real, 1 and 2 complex:
+// 2 + 2 * 4 = 10 real N x C x D products instead of 36 (2(T-1)/T^2).
+//   a_s = v_s + v_{s+3},  b_s = v_s - v_{s+3}                  (s = 0, 1, 2)
+//   V0 = a0 + a1 + a2,  V2 = a0 - (a1 + a2)/2 - i c (a1 - a2),  c = sqrt(3)/2
+//   V3 = b0 - b1 + b2,  V1 = b0 + (b1 - b2)/2 - i c (b1 + b2)
+// planes V0, V3, Re V1, -Im V1, Re V2, -Im V2; inverse
+//   y_t = (Y0 + (-1)^t Y3)/6 + (1/3) sum_{k=1,2} (Re Y_k cos(pi k t/3) - Im Y_k sin(pi k t/3)).
+// Fibres are 12 bytes (G8Geo<6>); the layer needs C and D multiples of 4
+// (16-byte row strides for the tensor maps).
+constexpr float kS6 = 0.86602540378443865f;  // sqrt(3)/2
+
+struct Cyclic6 {
+  static constexpr int kT = 6;
+  static constexpr int kFwdMmas = 6;
+  static constexpr int kDwMmas = 6;
+  // Weight rows: What0, What3, then for bins k = 1, 2 at row block r_k = 2 + 3(k-1):
+  // Re_k, Im_k, -Re_k (the windows (Re_k ; Im_k) and (Im_k ; -Re_k), as for C_8).
+  static constexpr int kWRows = 8;
+  __host__ __device__ static constexpr G8Mma fwd(int e) {
+    switch (e) {
+      case 0: return G8Mma{0, 0, 0, 0, 0};
+      case 1: return G8Mma{1, 1, 1, 0, 0};
+      case 2: return G8Mma{2, 2, 2, 1, 0};
+      case 3: return G8Mma{2, 3, 3, 1, 1};
+      case 4: return G8Mma{4, 4, 5, 1, 0};
+      default: return G8Mma{4, 5, 6, 1, 1};
+    }
+  }
+  // dW (columns in CT units): G0, G3, then per complex bin a = Re dY_k [Re X_k | -Im X_k]
+  // and b = -Im dY_k [Re X_k | -Im X_k]
+  static constexpr int kDwBlocks = 10;
+  __host__ __device__ static constexpr G8Mma dw(int e) {
+    switch (e) {
+      case 0: return G8Mma{0, 0, 0, 0, 0};
+      case 1: return G8Mma{1, 1, 1, 0, 0};
+      case 2: return G8Mma{2, 2, 2, 1, 0};
+      case 3: return G8Mma{4, 3, 2, 1, 0};
+      case 4: return G8Mma{6, 4, 4, 1, 0};
+      default: return G8Mma{8, 5, 4, 1, 0};
+    }
+  }
+
+  __device__ static void planes(const float (&v)[6], float (&o)[6]) {
+    const float a0 = v[0] + v[3], a1 = v[1] + v[4], a2 = v[2] + v[5];
+    const float b0 = v[0] - v[3], b1 = v[1] - v[4], b2 = v[2] - v[5];
+    o[0] = a0 + a1 + a2;
+    o[1] = b0 - b1 + b2;
+    o[2] = b0 + 0.5f * (b1 - b2);
+    o[3] = kS6 * (b1 + b2);
+    o[4] = a0 - 0.5f * (a1 + a2);
+    o[5] = kS6 * (a1 - a2);
+  }
+
+  // Packed fp16 pairs, every plane divided by 8 (bin 0 sums six values) in the
+  // first stage, as for the order-8 groups.
+  __device__ static void planes_h2(const __half2 (&v)[6], __half2 (&o)[6]) {
+    const __half2 q = __float2half2_rn(0.125f), hf = __float2half2_rn(0.5f);
+    const __half2 c = __float2half2_rn(kS6);
+    __half2 a[3], b[3];
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      const __half2 u = __hmul2(v[t + 3], q);
+      a[t] = __hfma2(v[t], q, u);
+      b[t] = __hfma2(v[t], q, __hneg2(u));
+    }
+    o[0] = __hadd2(__hadd2(a[0], a[1]), a[2]);
+    o[1] = __hadd2(__hsub2(b[0], b[1]), b[2]);
+    o[2] = __hfma2(hf, __hsub2(b[1], b[2]), b[0]);
+    o[3] = __hmul2(c, __hadd2(b[1], b[2]));
+    o[4] = __hfma2(__hneg2(hf), __hadd2(a[1], a[2]), a[0]);
+    o[5] = __hmul2(c, __hsub2(a[1], a[2]));
+  }
+
+  // Group values, times s, from the accumulator blocks Y0, Y3, Re Y1, Im Y1, Re Y2, Im Y2.
+  __device__ static void inverse(const float (&F)[6], float (&y)[6], float s) {
+    const float e = s * (1.f / 6.f), h = s * (1.f / 3.f);
+    const float P = e * (F[0] + F[1]), Q = e * (F[0] - F[1]);
+    const float r1 = F[2], i1 = F[3], r2 = F[4], i2 = F[5];
+    const float u = 0.5f * (r1 - r2), w = kS6 * (i1 + i2), z = kS6 * (i1 - i2);
+    const float v = 0.5f * (r1 + r2);
+    y[0] = P + h * (r1 + r2);
+    y[1] = Q + h * (u - w);
+    y[2] = P - h * (v + z);
+    y[3] = Q + h * (r2 - r1);
+    y[4] = P + h * (z - v);
+    y[5] = Q + h * (u + w);
+  }
+
+  __device__ static void weight_rows(const float (&w)[6], int dir, float (&rows)[kWRows]) {
+    float pl[6];
+    planes(w, pl);  // planes hold -Im; weights want Im (conjugated for dX)
+    const float s = dir == 0 ? -1.f : 1.f;
+    rows[0] = pl[0];
+    rows[1] = pl[1];
+#pragma unroll
+    for (int bk = 0; bk < 2; ++bk) {
+      rows[2 + 3 * bk] = pl[2 + 2 * bk];
+      rows[3 + 3 * bk] = s * pl[3 + 2 * bk];
+      rows[4 + 3 * bk] = -pl[2 + 2 * bk];
+    }
+  }
+
+  __device__ static void dw_planes(const float (&a)[kDwBlocks], float (&G)[6]) {
+    G[0] = a[0];
+    G[1] = a[1];
+#pragma unroll
+    for (int bk = 0; bk < 2; ++bk) {
+      G[2 + 2 * bk] = a[2 + 4 * bk] + a[5 + 4 * bk];
+      G[3 + 2 * bk] = a[3 + 4 * bk] - a[4 + 4 * bk];
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
 // Plans and the Fourier-weight layout
 // ---------------------------------------------------------------------------
 // Per (output tile j, 16-channel chunk kc) a weight chunk of kWRows * BD rows x

@@ -75,7 +75,7 @@ WORKLOADS = {
                 "D is the hidden width, the output has C channels"),
     10: Workload(10, "c6_fwdbwd_fp16_swin_N401408_C16_D64", 401408, 16, 64, "fp16",
                  ("fwd", "dx", "dw"),
-                 "cyclic group C_6 (non-dyadic twiddles, CUDA-core kernels), Swin stage-1-like "
+                 "cyclic group C_6 (non-dyadic twiddles, 12-byte fibres), Swin stage-1-like "
                  "stream (96->384 unrolled)", T=6),
     9: Workload(9, "p4_mlp_fp16_vit_ti_N12608_C48_H192", 12608, 48, 192, "fp16", ("mlp",),
                 "ViT-Ti-like MLP block at 64x197 tokens (192->768->192 unrolled; weights "

@@ -158,7 +158,7 @@ def _g8_bytes(C, D, rows):
     return al(plan(C, D)) + al(plan(D, C))
 
 
-@pytest.mark.parametrize("C,D", [(12, 48), (8, 8), (40, 130), (64, 16)])
+@pytest.mark.parametrize("C,D", [(12, 48), (8, 8), (40, 130), (64, 16), (6, 40)])
 def test_order8_weight_buffer_sizes(lib, C, D):
     # C_8: 11 weight rows per output channel (W0, W4, (Re, Im, -Re) of bins 1..3); p4m: 8
     assert F.feql_ct_weight_fft_bytes(8, C, D, F.FEQL_FP16) == _g8_bytes(C, D, 11)
@@ -167,6 +167,12 @@ def test_order8_weight_buffer_sizes(lib, C, D):
     for T in (2, 3, 6, 8, 12, 16):  # CUDA-core orders: fp32 planes of both directions
         assert F.feql_ct_weight_fft_bytes(T, C, D, F.FEQL_FP32) == 2 * T * C * D * 4
     assert F.feql_p4m_weight_fft_bytes(C, D, F.FEQL_FP32) == 0
+    # C_6 in fp16: tensor cores (8 weight rows: W0, W3, (Re, Im, -Re) of bins 1, 2) when C
+    # and D are multiples of 4, else the CUDA-core planes
+    if C % 4 == 0 and D % 4 == 0:
+        assert F.feql_ct_weight_fft_bytes(6, C, D, F.FEQL_FP16) == _g8_bytes(C, D, 8)
+    else:
+        assert F.feql_ct_weight_fft_bytes(6, C, D, F.FEQL_FP16) == 2 * 6 * C * D * 4
 
 
 def test_mlp_weight_buffer_covers_both_layers(lib):

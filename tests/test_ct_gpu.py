@@ -1,4 +1,5 @@
-"""GPU parity of the cyclic-group C_8 kernels against the float64 C_T oracle.
+"""GPU parity of the cyclic-group tensor-core kernels (C_8, and C_6 with its
+non-dyadic twiddles and 12-byte fibres) against the float64 C_T oracle.
 
 Every test calls the library through the C ABI (ctypes); the oracle consumes
 the same dtype-rounded inputs.  Tolerance: max|err| / max|ref| <= 5e-3 (fp16
@@ -141,7 +142,8 @@ def test_ct_unsupported_orders_and_modes():
     assert F.feql_ct_weight_fft_bytes(1, 4, 4, FP16) == 0
     assert F.feql_ct_weight_fft_bytes(8, 4, 4, F.FEQL_FP32_3XTF32) == 0
     # the CUDA-core orders size their buffer as fp32 planes of both directions
-    assert F.feql_ct_weight_fft_bytes(6, 4, 4, FP16) == 2 * 6 * 4 * 4 * 4
+    assert F.feql_ct_weight_fft_bytes(6, 6, 6, FP16) == 2 * 6 * 6 * 6 * 4
+    assert F.feql_ct_weight_fft_bytes(3, 4, 4, FP16) == 2 * 3 * 4 * 4 * 4
     x = torch.zeros((16, 4, 17), dtype=torch.float16, device="cuda")
     W = torch.zeros(1 << 16, dtype=torch.uint8, device="cuda")
     y = torch.empty((16, 4, 17), dtype=torch.float16, device="cuda")
@@ -154,6 +156,88 @@ def test_ct_unsupported_orders_and_modes():
 def test_c8_workload_full_size():
     w = WORKLOADS[6]
     inp = workload_inputs(6)
+    out = run_c8(inp)
+    x, W, b, dy = (inp[k].astype(np.float64) for k in ("x", "W", "b", "dy"))
+    rows = np.r_[0:2048, w.N - 2048:w.N]  # sampled token rows for y and dx
+    assert O.rel_err(out["y"][rows], O.forward(x[rows], W, b)) <= TOL
+    assert O.rel_err(out["dx"][rows], O.backward_dx(dy[rows], W)) <= TOL
+    dW, db = O.backward_dw(x, dy)  # every token
+    assert O.rel_err(out["dW"], dW) <= TOL and O.rel_err(out["db"], db) <= TOL
+
+
+# C_6 on the tensor cores (C and D multiples of 4): forward tiles of <= 64 output
+# channels, 16-channel chunks with a ragged second box, ragged token tiles, dW tiles
+# of 128 d x 16/32 c; D = 132 and 20 take one TMA load per 8-channel box (no box stack)
+C6_SHAPES = [(300, 12, 48), (1, 8, 8), (129, 4, 40), (1000, 16, 64), (517, 32, 24),
+             (257, 40, 132), (70, 64, 16), (333, 20, 20)]
+
+
+@pytest.mark.parametrize("N,C,D", C6_SHAPES)
+def test_c6_tensor_cores_match_oracle(N, C, D):
+    inp = make_inputs(31, N, C, D, "fp16", T=6)
+    check_c8(run_c8(inp), inp)
+
+
+@pytest.mark.parametrize("C,D", [(6, 40), (12, 10)])
+def test_c6_other_channel_counts_take_the_cuda_cores(C, D):
+    # C or D not a multiple of 4: the 12-byte fibres' row strides would not be
+    # 16-byte multiples for the tensor maps; the CUDA-core kernels serve them
+    assert F.feql_ct_weight_fft_bytes(6, C, D, FP16) == 2 * 6 * C * D * 4
+    inp = make_inputs(32, 200, C, D, "fp16", T=6)
+    check_c8(run_c8(inp), inp)
+
+
+def test_c6_without_bias_and_zero_tokens():
+    N, C, D = 200, 12, 48
+    inp = make_inputs(33, N, C, D, "fp16", T=6)
+    x, W = dev(inp["x"]), dev(inp["W"])
+    What = Lyr.ct_weight_fft(W, FP16)
+    y = Lyr.ct_forward(x, What, None, D, FP16)
+    ref = O.forward(inp["x"].astype(np.float64), inp["W"].astype(np.float64), None)
+    assert O.rel_err(host(y), ref) <= TOL
+    x0 = torch.empty((0, C, 6), dtype=torch.float16, device="cuda")
+    dy0 = torch.empty((0, D, 6), dtype=torch.float16, device="cuda")
+    y0 = torch.full((1, D, 6), 7.0, dtype=torch.float16, device="cuda")
+    F.feql_ct_forward(6, x0, What, None, y0, 0, C, D, FP16)
+    dW, db = Lyr.ct_backward_dw(x0, dy0, FP16)
+    torch.cuda.synchronize()
+    assert torch.all(y0 == 7.0) and torch.all(dW == 0) and torch.all(db == 0)
+
+
+@pytest.mark.parametrize("r", [1, 2, 3])
+def test_c6_rotation_equivariance(r):
+    N, C, D = 500, 16, 32
+    inp = make_inputs(34, N, C, D, "fp16", T=6)
+    x, W, b = dev(inp["x"]), dev(inp["W"]), dev(inp["b"])
+    What = Lyr.ct_weight_fft(W, FP16)
+    y = host(Lyr.ct_forward(x, What, b, D, FP16))
+    yr = host(Lyr.ct_forward(torch.roll(x, r, dims=2).contiguous(), What, b, D, FP16))
+    assert O.rel_err(yr, np.roll(y, r, axis=2)) < 2e-3
+
+
+def test_c6_dw_is_deterministic_and_outputs_stay_in_their_buffers():
+    N, C, D = 3000, 12, 48
+    inp = make_inputs(35, N, C, D, "fp16", T=6)
+    x, W, b, dy = dev(inp["x"]), dev(inp["W"]), dev(inp["b"]), dev(inp["dy"])
+    a = Lyr.ct_backward_dw(x, dy, FP16)
+    c = Lyr.ct_backward_dw(x, dy, FP16)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+    What = Lyr.ct_weight_fft(W, FP16)
+    guard = 4096
+    for shape, fn in [((N, D, 6), lambda o: F.feql_ct_forward(6, x, What, b, o, N, C, D, FP16)),
+                      ((N, C, 6), lambda o: F.feql_ct_backward_dx(6, dy, What, o, N, C, D, FP16))]:
+        n = int(np.prod(shape))
+        buf = torch.full((n + 2 * guard,), -3.0, dtype=torch.float16, device="cuda")
+        fn(buf[guard:guard + n].view(shape))
+        torch.cuda.synchronize()
+        assert torch.all(buf[:guard] == -3.0) and torch.all(buf[guard + n:] == -3.0)
+
+
+@pytest.mark.slow
+def test_c6_workload_full_size():
+    w = WORKLOADS[10]
+    inp = workload_inputs(10)
     out = run_c8(inp)
     x, W, b, dy = (inp[k].astype(np.float64) for k in ("x", "W", "b", "dy"))
     rows = np.r_[0:2048, w.N - 2048:w.N]  # sampled token rows for y and dx
