@@ -614,8 +614,9 @@ def widening_report(F, torch, stream, reps, meas, nom, flush):
     CUDA-event timings with the L2 flushed before each, median and min, against
     the slower of its algorithmic bytes at HBM bandwidth and its Fourier-route
     FLOPs at the arithmetic peak of the units it runs on (tensor cores, or the
-    fp32 FMA pipes for a shape the CUDA-core kernels serve).  The MLP block also gets a special-function floor:
-    its GELU takes one tanh per two hidden values."""
+    fp32 FMA pipes for a shape the CUDA-core kernels serve).  The MLP block
+    also gets a special-function floor: its GELU takes one tanh per two hidden
+    values."""
     import numpy as np
 
     from group_dft_structured_b200.workloads import WORKLOADS

@@ -172,9 +172,12 @@ int feql_backward_dw_noalloc(const void *x, const void *dy, void *dW, void *db,
  *   y[n,d,t] = b[d] + sum_c sum_s W[d,c,(t-s) mod T] x[n,c,s]
  * T = 4 is the p4 layer: every call forwards to the function above with the
  * same arguments (all modes).  T = 8 in FEQL_FP16: tensor-core kernels (bins 0
- * and 4 real, 1..3 complex, 14 real products instead of 64).  Every order
+ * and 4 real, 1..3 complex, 14 real products instead of 64).  T = 6 in
+ * FEQL_FP16 with C and D multiples of 4: the same tensor-core kernels with the
+ * order-6 twiddles (bins 0 and 3 real, 1 and 2 complex, 10 real products
+ * instead of 36; the 12-byte fibres need 16-byte row strides).  Every order
  * 2 <= T <= 16 in FEQL_FP32 / FEQL_FP32_SIMT / FEQL_FP16_SIMT, and in
- * FEQL_FP16 for T other than 4 and 8: CUDA-core kernels of the same method
+ * FEQL_FP16 for the other orders and shapes: CUDA-core kernels of the same method
  * with the DFT twiddles of order T (non-dyadic for T = 3, 5, 6, 7, 12 ...;
  * (2T-2)/T^2 or, for odd T, (2T-1)/T^2 of the dense products), fp32
  * arithmetic on fp32 or fp16 data.  FEQL_FP32_3XTF32 and orders outside 2..16
