@@ -53,7 +53,9 @@ struct G8Geo;
 template <>
 struct G8Geo<8> {
   static constexpr int kRow = 128;
-  // Packed pairs v[t] = (channel 2p, channel 2p+1) at group element t of box row r.
+  // Channel pair p of the row as packed pairs: v[t] = (channel 2p, channel
+  // 2p+1) at group element t.  Chunk c of the row (channel c) sits at chunk
+  // c ^ (r & 7) (128-byte swizzle); each pair is two 16-byte loads of its own.
   __device__ static void pair(const uint8_t *row, int p, int r, __half2 (&v)[8]) {
     const uint4 w0 = *reinterpret_cast<const uint4 *>(row + (((2 * p) ^ (r & 7)) << 4));
     const uint4 w1 = *reinterpret_cast<const uint4 *>(row + (((2 * p + 1) ^ (r & 7)) << 4));
@@ -65,9 +67,12 @@ struct G8Geo<8> {
       v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
     }
   }
-  // Channel c's fibre (packed fp16 pairs) into box row r.
-  __device__ static void put(uint8_t *row, int c, int r, const uint32_t (&h)[4]) {
-    *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+  // Fibres of channels 4h..4h+3 (packed fp16 pairs) into box row r.
+  __device__ static void put4(uint8_t *row, int h, int r, const uint32_t (&f)[4][4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4 *>(row + (((4 * h + i) ^ (r & 7)) << 4)) =
+          make_uint4(f[i][0], f[i][1], f[i][2], f[i][3]);
   }
   // One fibre to global memory (16-byte aligned).
   __device__ static void store(__half *dst, const uint32_t (&h)[4]) {
@@ -75,27 +80,39 @@ struct G8Geo<8> {
   }
 };
 
+// 96-byte rows: the row is read as six 16-byte chunks (24 words, channel c in
+// words 3c..3c+2) and the fibres extracted with static indices; 16-byte
+// accesses of neighbouring rows (a 24-word pitch) conflict at most two ways.
 template <>
 struct G8Geo<6> {
   static constexpr int kRow = 96;
-  __device__ static void pair(const uint8_t *row, int p, int, __half2 (&v)[6]) {
-    const uint2 w0 = *reinterpret_cast<const uint2 *>(row + 24 * p);
-    const uint2 w1 = *reinterpret_cast<const uint2 *>(row + 24 * p + 8);
-    const uint2 w2 = *reinterpret_cast<const uint2 *>(row + 24 * p + 16);
-    // channel 2p: w0.x, w0.y, w1.x; channel 2p + 1: w1.y, w2.x, w2.y
-    const uint32_t a[3] = {w0.x, w0.y, w1.x}, b[3] = {w1.y, w2.x, w2.y};
+  __device__ static void pairs(const uint8_t *row, int, __half2 (&v)[4][6]) {
+    uint32_t w[24];
 #pragma unroll
-    for (int e = 0; e < 3; ++e) {
-      const uint32_t lo = __byte_perm(a[e], b[e], 0x5410), hi = __byte_perm(a[e], b[e], 0x7632);
-      v[2 * e] = *reinterpret_cast<const __half2 *>(&lo);
-      v[2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
+    for (int k = 0; k < 6; ++k) {
+      const uint4 c = *reinterpret_cast<const uint4 *>(row + 16 * k);
+      w[4 * k] = c.x;
+      w[4 * k + 1] = c.y;
+      w[4 * k + 2] = c.z;
+      w[4 * k + 3] = c.w;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+#pragma unroll
+      for (int e = 0; e < 3; ++e) {
+        const uint32_t a = w[6 * p + e], b = w[6 * p + 3 + e];  // channels 2p, 2p + 1
+        const uint32_t lo = __byte_perm(a, b, 0x5410), hi = __byte_perm(a, b, 0x7632);
+        v[p][2 * e] = *reinterpret_cast<const __half2 *>(&lo);
+        v[p][2 * e + 1] = *reinterpret_cast<const __half2 *>(&hi);
+      }
     }
   }
-  __device__ static void put(uint8_t *row, int c, int, const uint32_t (&h)[3]) {
-    uint32_t *w = reinterpret_cast<uint32_t *>(row + 12 * c);
-    w[0] = h[0];
-    w[1] = h[1];
-    w[2] = h[2];
+  // Channels 4h..4h+3 are words 12h..12h+11 of the row: three 16-byte chunks.
+  __device__ static void put4(uint8_t *row, int h, int, const uint32_t (&f)[4][3]) {
+    uint4 *dst = reinterpret_cast<uint4 *>(row + 48 * h);
+    dst[0] = make_uint4(f[0][0], f[0][1], f[0][2], f[1][0]);
+    dst[1] = make_uint4(f[1][1], f[1][2], f[2][0], f[2][1]);
+    dst[2] = make_uint4(f[2][2], f[3][0], f[3][1], f[3][2]);
   }
   // (4-byte aligned: fibres start at multiples of 12 bytes)
   __device__ static void store(__half *dst, const uint32_t (&h)[3]) {
@@ -514,16 +531,23 @@ __host__ __device__ inline G8Layout make_g8_layout(int C, int D, int wrows) {
   return L;
 }
 
-// Planes of the channel pair (2p, 2p+1) of box row r, packed: o[k] = plane k
-// of both channels, low half first.
+// Planes of the four channel pairs of box row r, packed: o[p][k] = plane k of
+// channels 2p, 2p+1, low half first.
+// (T = 8 loads pair by pair, each pair's two chunks whole; T = 6 loads the row
+// once, its fibres straddling the chunks.)
 template <class Gp>
-__device__ __forceinline__ void g8_planes_pair(const uint8_t *row, int p, int r,
-                                               uint32_t (&o)[Gp::kT]) {
-  __half2 v[Gp::kT], w[Gp::kT];
-  G8Geo<Gp::kT>::pair(row, p, r, v);
-  Gp::planes_h2(v, w);
+__device__ __forceinline__ void g8_planes_row(const uint8_t *row, int r,
+                                              uint32_t (&o)[4][Gp::kT]) {
+  __half2 v[4][Gp::kT];
+  if constexpr (Gp::kT == 6) G8Geo<6>::pairs(row, r, v);
 #pragma unroll
-  for (int k = 0; k < Gp::kT; ++k) o[k] = *reinterpret_cast<const uint32_t *>(&w[k]);
+  for (int p = 0; p < 4; ++p) {
+    if constexpr (Gp::kT == 8) G8Geo<8>::pair(row, p, r, v[p]);
+    __half2 w[Gp::kT];
+    Gp::planes_h2(v[p], w);
+#pragma unroll
+    for (int k = 0; k < Gp::kT; ++k) o[p][k] = *reinterpret_cast<const uint32_t *>(&w[k]);
+  }
 }
 
 // One thread per fp16 element of the tiled weight buffer (both directions).
@@ -766,19 +790,13 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
         if (ok) ok = mbar_wait(&full[s], ph);
         uint8_t *st = smem + L.stage0 + s * p.stage_bytes;
         const uint8_t *src = st + bx * kBox + r * Geo::kRow;
-        uint32_t pw[T][4];  // [plane][channel pair], packed fp16
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // channels 8 bx + 2q, 8 bx + 2q + 1
-          uint32_t o[T];
-          g8_planes_pair<Gp>(src, q, r, o);
-#pragma unroll
-          for (int pp = 0; pp < T; ++pp) pw[pp][q] = o[pp];
-        }
+        uint32_t pw[4][T];  // [channel pair][plane], packed fp16
+        g8_planes_row<Gp>(src, r, pw);
         named_bar_sync(2, 256);  // every row read before the planes overwrite it
 #pragma unroll
         for (int pp = 0; pp < T; ++pp)
           *reinterpret_cast<uint4 *>(st + pp * kG8Plane + r * 32 + (((bx ^ (r >> 2)) & 1) << 4)) =
-              make_uint4(pw[pp][0], pw[pp][1], pw[pp][2], pw[pp][3]);
+              make_uint4(pw[0][pp], pw[1][pp], pw[2][pp], pw[3][pp]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(&tready[s]);
@@ -830,19 +848,18 @@ tc_g8_fwd_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constan
             if (lane == 0 && ok) mbar_arrive(&acc_empty[a]);
           }
           if (d0 >= p.Do) continue;  // whole group is padding
+          uint32_t hv[4][T / 2];  // fibres of channels d0 + 4h .. d0 + 4h + 3, packed fp16
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {  // fibre 4h + i of the row = channel d0 + 4h + i
-            const int c = 4 * h + i;
+          for (int i = 0; i < 4; ++i) {
             float F[T], y[T];
 #pragma unroll
             for (int bk = 0; bk < T; ++bk) F[bk] = __uint_as_float(Y[bk][i]);
             Gp::inverse(F, y, 64.f);  // planes and weights both carry 1/8
-            const float bv = sbias[d0 + c];
-            uint32_t hv[T / 2];
+            const float bv = sbias[d0 + 4 * h + i];
 #pragma unroll
-            for (int e = 0; e < T / 2; ++e) hv[e] = pack_half2(y[2 * e] + bv, y[2 * e + 1] + bv);
-            Geo::put(ob + lane * Geo::kRow, c, lane, hv);
+            for (int e = 0; e < T / 2; ++e) hv[i][e] = pack_half2(y[2 * e] + bv, y[2 * e + 1] + bv);
           }
+          Geo::put4(ob + lane * Geo::kRow, h, lane, hv);
         }
         if (d0 >= p.Do) continue;
         fence_proxy_async_smem();
@@ -1059,7 +1076,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
     for (int ch = 0; ch < nch; ++ch) {
       if (ok) ok = mbar_wait(&full[s], ph);
       uint8_t *st = smem + L.stage0 + s * p.slot_boxes * kBox;
-      uint32_t pw[kG8DwMaxPer][T][4];
+      uint32_t pw[kG8DwMaxPer][4][T];  // [item][channel pair][plane], packed fp16
 #pragma unroll
       for (int k = 0; k < kG8DwMaxPer; ++k) {
         const int e = t + k * 256;
@@ -1067,17 +1084,14 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
         if (bi < nbox) {
           const uint8_t *src = st + (bi < nqd ? bi * kBox : xoff + (bi - nqd) * kBox) +
                                r * Geo::kRow;
+          g8_planes_row<Gp>(src, r, pw[k]);
+          if (do_db && bi < nqd) {  // bin 0 of the dy planes, as the MMAs see it
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {  // channels 2q, 2q + 1 of the box
-            uint32_t o[T];
-            g8_planes_pair<Gp>(src, q, r, o);
-            if (do_db && bi < nqd) {  // bin 0 of the dy planes, as the MMAs see it
-              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&o[0]));
+            for (int q = 0; q < 4; ++q) {  // channels 2q, 2q + 1 of the box
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&pw[k][q][0]));
               db_acc[k][2 * q] += f.x;
               db_acc[k][2 * q + 1] += f.y;
             }
-#pragma unroll
-            for (int pp = 0; pp < T; ++pp) pw[k][pp][q] = o[pp];
           }
         }
       }
@@ -1096,7 +1110,7 @@ tc_g8_dw_kernel(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant
 #pragma unroll
           for (int pp = 0; pp < T; ++pp)
             *reinterpret_cast<uint4 *>(pbase + pp * pstride + r * 32 + (((hh ^ (r >> 2)) & 1) << 4)) =
-                make_uint4(pw[k][pp][0], pw[k][pp][1], pw[k][pp][2], pw[k][pp][3]);
+                make_uint4(pw[k][0][pp], pw[k][1][pp], pw[k][2][pp], pw[k][3][pp]);
         }
       }
       fence_proxy_async_smem();
