@@ -36,14 +36,15 @@
  *    group-axis sums of the transform reach |G| max|v| (G the group: 4 for p4,
  *    6 for C_6, 8 for C_8 and p4m), so the fp16 operand planes and Fourier
  *    weights hold every bin divided by 4 (p4) or 8 (the others: an exact power
- *    of two that the fp32 epilogues undo); results are within the fp16 mode's tolerance whenever the outputs
- *    y, dx, dW and db themselves are finite in fp16 (an output beyond 65504
- *    becomes inf, as in any fp16 layer).  The MLP block likewise accepts
- *    every finite x, W1, W2, b1, b2 whose hidden activation h and output y
- *    are finite in fp16 (its hidden planes hold GELU(h) / 4).  Where a scaled
- *    value falls among the fp16 subnormals (below 2^-14) it is rounded to the
- *    subnormal spacing 2^-24, at most twice per butterfly stage: an absolute
- *    error per bin of at most 2^-21 for p4 and 2^-19 for the order-6 and -8 groups.
+ *    of two that the fp32 epilogues undo); results are within the fp16 mode's
+ *    tolerance whenever the outputs y, dx, dW and db themselves are finite in
+ *    fp16 (an output beyond 65504 becomes inf, as in any fp16 layer).  The MLP
+ *    block likewise accepts every finite x, W1, W2, b1, b2 whose hidden
+ *    activation h and output y are finite in fp16 (its hidden planes hold
+ *    GELU(h) / 4).  Where a scaled value falls among the fp16 subnormals (below
+ *    2^-14) it is rounded to the subnormal spacing 2^-24, at most twice per
+ *    butterfly stage: an absolute error per bin of at most 2^-21 for p4 and
+ *    2^-19 for the order-6 and -8 groups.
  */
 #ifndef FEQL_H
 #define FEQL_H
