@@ -1,15 +1,19 @@
-// group8.cuh — the EQ-Linear layer of a group of order 8 on the sm_100a tensor
-// cores, fp16 data with fp32 accumulation: the cyclic group C_8 (Cyclic8) and
-// the point group D4 of p4m (Dihedral4).
+// group8.cuh — the EQ-Linear layer of a group of order T = 8 or 6 on the
+// sm_100a tensor cores, fp16 data with fp32 accumulation: the cyclic group C_8
+// (Cyclic8), the point group D4 of p4m (Dihedral4) and the cyclic group C_6
+// (Cyclic6).
 //
 // Flash EQ-Linear states the method for a cyclic group of any order T (arXiv
 // abstract: cost 2(T-1)/T^2 of the dense layer), builds kernels for p4 and
 // names reflection groups as future work (technical summary, "Limitazioni e
-// Lavoro Futuro").  Both groups here have 8 elements, so a channel fibre is
-// 16 bytes of fp16 and its Fourier transform has 8 real components (planes);
-// per 16 channels the layer is 8 tensor-core MMAs into 8 BD accumulator
-// columns.  The kernels are templates over a group policy that supplies the
-// transform, its inverse, the weight planes and the MMA tables.
+// Lavoro Futuro").  A channel fibre is T fp16 values and its Fourier transform
+// has T real components (planes); per 16 channels the layer is one tensor-core
+// MMA per real bin and two per complex bin (8 for the order-8 groups, 6 for
+// C_6) into T BD accumulator columns.  The kernels are templates over a group
+// policy that supplies the order, the transform, its inverse, the weight
+// planes and the MMA tables, and over the fibre geometry of its order
+// (G8Geo: 16-byte fibres in swizzled 128-byte rows, or 12-byte fibres in
+// plain 96-byte rows).
 //
 // C_8: the real 8-point DFT keeps bins 0..4: bins 0 and 4 are real, 1, 2, 3
 // complex: 2 + 3*4 = 14 real N x C x D products instead of 64.
