@@ -454,8 +454,8 @@ NOMINAL = {"hbm_gbs": 8000.0, "tensor_tflops": 2250.0, "fp32_fma_tflops": 74.4,
            "tf32_tflops": 1125.0}
 
 # The five layer configurations, each with the passes its throughput is quoted
-# on (SURVEY of the method's workloads: forward for 1-3, dX and dW for 4,
-# forward and both gradients for 5; 3 also in fp32).
+# on (forward for 1-3, dX and dW for 4, forward and both gradients for 5; 3
+# also in fp32).
 # fp32 runs in both fp32 modes: CUDA cores ("fp32") and split TF32 on the tensor
 # cores ("fp32_3xtf32", three tf32 products per product).
 CONFIG_RUNS = [(1, "fp32", ("fwd",)), (1, "fp32_3xtf32", ("fwd",)), (2, "fp16", ("fwd",)),
