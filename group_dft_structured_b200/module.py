@@ -1,6 +1,6 @@
 """Drop-in PyTorch module for the equivariant linear layer of the cyclic group
-C_T (T = 4: the rotation group p4; T = 8) and of p4m (rotations and
-reflections, point group D4), with autograd.
+C_T (T = 4: the rotation group p4; any T in 2..16, T = 6 and 8 on the tensor
+cores) and of p4m (rotations and reflections, point group D4), with autograd.
 
 Flash EQ-Linear (arXiv abstract) presents the method as a plug-and-play
 replacement for the EQ-Linear layers of existing equivariant models: the layer
@@ -96,7 +96,8 @@ class EqLinear(torch.nn.Module):
     """Equivariant linear layer of C_T (or p4m) on features (..., C*T), group index innermost.
 
     Parameters: ``weight`` [D][C][T] and ``bias`` [D] (or None), in float16
-    (T = 4 or 8, p4m) or float32 (T = 4).  ``group="p4m"`` selects the point
+    (any T; the tensor cores serve T = 4, 8, p4m, and 6 with C and D multiples
+    of 4) or float32.  ``group="p4m"`` selects the point
     group D4 (T = 8: rotations (r, 0) at 0..3, reflected (r, 1) at 4..7).  The
     Fourier weight buffer is rebuilt when the weight changes (tracked by its
     storage and version counter), so it is computed once per optimizer step, or

@@ -129,7 +129,7 @@ def _host(t):
 
 
 CASES = [(4, "fp16", 300, 24, 96, 5e-3), (8, "fp16", 300, 12, 48, 5e-3),
-         (4, "fp32", 130, 16, 24, 1e-5)]
+         (6, "fp16", 300, 16, 64, 5e-3), (4, "fp32", 130, 16, 24, 1e-5)]
 
 
 @pytest.mark.gpu
@@ -152,7 +152,7 @@ def test_module_forward_and_autograd_match_oracle(T, dtype, N, C, D, tol):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("T", [4, 8])
+@pytest.mark.parametrize("T", [4, 6, 8])
 def test_module_gradient_subsets(T):
     _cuda_ready()
     N, C, D = 200, 8, 16
