@@ -31,3 +31,32 @@ def test_traffic_table_entries_are_positive_byte_counts():
         if name.startswith("_") or name == "source_hash":
             continue
         assert passes and all(isinstance(v, int) and v > 0 for v in passes.values()), name
+
+
+def test_traffic_table_matches_the_current_kernel_sources():
+    # the committed DRAM counters were taken on these kernels (bench.py reports
+    # them only while the hash matches; a kernel change needs a new capture)
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        table = json.load(f)
+    assert table["source_hash"] == bench.kernel_source_hash()
+
+
+def test_bench_mac_counts_equal_the_oracles_counted_products():
+    # the FLOPs behind the bench's TFLOP/s and rooflines are the real products
+    # the oracles count when they run the Fourier route
+    import numpy as np
+
+    from group_dft_structured_b200.workloads import Workload
+    from oracle import feql_ct_oracle as OC
+    from oracle import feql_p4m_oracle as OM
+
+    rng = np.random.default_rng(5)
+    N, C, D = 3, 5, 7
+    for T, group in ((4, "cyclic"), (6, "cyclic"), (8, "cyclic"), (8, "p4m")):
+        w = Workload(0, "t", N, C, D, "fp16", ("fwd",), "", T=T, group=group)
+        x, W = rng.standard_normal((N, C, T)), rng.standard_normal((D, C, T))
+        O = OM if group == "p4m" else OC
+        _, macs = O.fourier_forward_counted(x, W, None)
+        fourier, dense = bench.layer_macs(w)
+        assert fourier == macs, (T, group)
+        assert dense == T * T * N * C * D
